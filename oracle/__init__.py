@@ -1,0 +1,171 @@
+"""CPU oracle for the nested r-bit GEMM -- TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  The product library (``nested_bit_weight_b200``)
+never imports it and shares no code with it; the two meet only through the
+seeded generators in ``workloads.py``.
+
+Each function states the passage it follows.  The method's definitions come
+from the MatGPTQ pages (abstract of "MatGPTQ: Efficient and Accurate
+Inference over Nested Quantized Models": r-bit models are read from the
+parent by reading fewer bits, exactly r bits; author-page abstract of
+"MatGPTQ: Accurate and Efficient Post-Training Matryoshka Quantization": the
+most significant bits are sliced).  The dequantization formula and the
+tolerance are the hot-path statement this library is built to:
+
+    q_r = q >> (8 - r),   w = s_g * (2^(8-r) * q_r + 2^(7-r) - 128),
+    |Y - Y_ref| <= 8e-3 * |Y_ref| + 1e-3 * rms(Y_ref)  per element.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the plain-C oracle with gcc (-O2, OpenMP, no SIMD intrinsics)."""
+    if force or not os.path.exists(_LIB) or \
+            os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp",
+                               "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        lib.oracle_pack.argtypes = [P, I64, I64, P]
+        lib.oracle_unpack.argtypes = [P, I64, I64, I, P]
+        lib.oracle_gemm_f64.argtypes = [P, P, P, I64, I64, I64, I, P]
+        lib.oracle_gemm_f64_at.argtypes = [P, P, P, I64, I, I64, P, P, P]
+        lib.oracle_threads.restype = I
+        for f in (lib.oracle_pack, lib.oracle_unpack, lib.oracle_gemm_f64,
+                  lib.oracle_gemm_f64_at):
+            f.restype = None
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def threads() -> int:
+    return int(_load().oracle_threads())
+
+
+# ---------------------------------------------------------------- definitions
+
+def slice_codes(codes: np.ndarray, r: int) -> np.ndarray:
+    """Top r bits of each 8-bit parent code (MSB slicing, integer floor)."""
+    if not 1 <= r <= 8:
+        raise ValueError("r must be in 1..8")
+    return (codes.astype(np.uint8) >> np.uint8(8 - r)).astype(np.uint8)
+
+
+def level(q_r: np.ndarray, r: int) -> np.ndarray:
+    """v_r = 2^(8-r) q_r + 2^(7-r) - 128, exact in fp64."""
+    return (2.0 ** (8 - r)) * q_r.astype(np.float64) + 2.0 ** (7 - r) - 128.0
+
+
+def scales_f16(s: np.ndarray) -> np.ndarray:
+    """The stored scale: fp32 s rounded to fp16 (round-to-nearest-even)."""
+    with np.errstate(over="ignore"):
+        return np.asarray(s, np.float32).astype(np.float16)
+
+
+def dequant(codes: np.ndarray, s: np.ndarray, r: int) -> np.ndarray:
+    """W_r[n, k] = s16[n, k // 128] * v_r(q_r[n, k]) in fp64."""
+    s16 = scales_f16(s).astype(np.float64)
+    v = level(slice_codes(codes, r), r)
+    return v * np.repeat(s16, 128, axis=1)
+
+
+# ------------------------------------------------------------- plain-C kernels
+
+def pack(codes: np.ndarray) -> np.ndarray:
+    """8 MSB-first bit planes, uint32 [8, N, K/32]."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    N, K = codes.shape
+    out = np.empty((8, N, K // 32), np.uint32)
+    _load().oracle_pack(_ptr(codes), N, K, _ptr(out))
+    return out
+
+
+def unpack(planes: np.ndarray, r: int, N: int, K: int) -> np.ndarray:
+    """r-bit codes read from the first r planes, uint8 [N, K]."""
+    planes = np.ascontiguousarray(planes, np.uint32)
+    if planes.size < r * N * (K // 32):
+        raise ValueError("plane buffer too small")
+    out = np.empty((N, K), np.uint8)
+    _load().oracle_unpack(_ptr(planes), N, K, r, _ptr(out))
+    return out
+
+
+def gemm(X: np.ndarray, codes: np.ndarray, s: np.ndarray, r: int) -> np.ndarray:
+    """Y = X . W_r^T with fp64 accumulation in ascending k; Y is [M, N] fp64.
+
+    X holds bf16 values (any float dtype holding them exactly); s is the fp32
+    scale, rounded to its stored fp16 value here.
+    """
+    X = np.ascontiguousarray(X, np.float64)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    s16 = np.ascontiguousarray(scales_f16(s).astype(np.float64))
+    M, K = X.shape
+    N = codes.shape[0]
+    Y = np.empty((M, N), np.float64)
+    _load().oracle_gemm_f64(_ptr(X), _ptr(codes), _ptr(s16), M, N, K, r, _ptr(Y))
+    return Y
+
+
+def gemm_at(X, codes, s, r, ms, ns) -> np.ndarray:
+    """Y[ms[i], ns[i]] for a list of output positions (same definition)."""
+    X = np.ascontiguousarray(X, np.float64)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    s16 = np.ascontiguousarray(scales_f16(s).astype(np.float64))
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.empty(ms.shape[0], np.float64)
+    _load().oracle_gemm_f64_at(_ptr(X), _ptr(codes), _ptr(s16), X.shape[1], r,
+                               ms.shape[0], _ptr(ms), _ptr(ns), _ptr(out))
+    return out
+
+
+# ------------------------------------------------------------------ tolerance
+
+REL_TOL = 8e-3
+RMS_TOL = 1e-3
+
+
+def tolerance(Yref: np.ndarray, rms: float | None = None) -> np.ndarray:
+    """Per-element bound 8e-3 |Y_ref| + 1e-3 rms(Y_ref) (rms over all of Y)."""
+    Yref = np.asarray(Yref, np.float64)
+    if rms is None:
+        rms = float(np.sqrt(np.mean(Yref * Yref))) if Yref.size else 0.0
+    return REL_TOL * np.abs(Yref) + RMS_TOL * rms
+
+
+def violation_ratio(Y, Yref, rms: float | None = None) -> float:
+    """max |Y - Y_ref| / bound; <= 1 means every element passes."""
+    Y = np.asarray(Y, np.float64)
+    Yref = np.asarray(Yref, np.float64)
+    if Yref.size == 0:
+        return 0.0
+    tol = tolerance(Yref, rms)
+    err = np.abs(Y - Yref)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(tol > 0, err / tol, np.where(err > 0, np.inf, 0.0))
+    return float(ratio.max())

@@ -1,0 +1,125 @@
+/*
+ * Plain CPU oracle for the nested r-bit GEMM (TEST INFRASTRUCTURE ONLY).
+ *
+ * Only tests/, __graft_entry__.smoke() and bench.py's cpu_baseline leg call
+ * this code.  It shares nothing with the CUDA library: no header, no table,
+ * no helper.  It is written for obviousness, not speed: every loop follows
+ * the definition directly.
+ *
+ * Definitions followed (MatGPTQ, "Efficient and Accurate Inference over
+ * Nested Quantized Models", abstract: lower-precision models are read from
+ * the higher-precision parent by reading fewer bits, and an r-bit model reads
+ * exactly r bits; MatGPTQ author page abstract: the most significant bits
+ * are sliced at inference time):
+ *
+ *   slice:   q_r = q >> (8 - r)                         (top r bits of q)
+ *   level:   v_r = 2^(8-r) * q_r + 2^(7-r) - 128
+ *   weight:  w[n,k] = s16[n, k/128] * v_r[n,k]
+ *   output:  Y[m,n] = sum_k X[m,k] * w[n,k]   (fp64, ascending k)
+ *
+ * Bit-plane layout (the exact-r-bit storage): planes[p][n][K/32] of uint32,
+ * p = 0..7; plane p holds bit (7 - p) of the parent code (most significant
+ * plane first) and bit j of word w of row n holds the code at k = 32*w + j.
+ * An r-bit model is the first r planes.
+ */
+#include <stdint.h>
+#include <stddef.h>
+
+/* Build the 8 planes bit by bit from the parent codes. */
+void oracle_pack(const uint8_t *codes, int64_t N, int64_t K, uint32_t *planes)
+{
+    int64_t W = K / 32;
+    for (int p = 0; p < 8; ++p) {
+        for (int64_t n = 0; n < N; ++n) {
+            for (int64_t w = 0; w < W; ++w) {
+                uint32_t word = 0;
+                for (int j = 0; j < 32; ++j) {
+                    uint8_t q = codes[n * K + 32 * w + j];
+                    uint32_t bit = (q >> (7 - p)) & 1u;
+                    word |= bit << j;
+                }
+                planes[((int64_t)p * N + n) * W + w] = word;
+            }
+        }
+    }
+}
+
+/* Read back the r-bit codes q_r from the first r planes. */
+void oracle_unpack(const uint32_t *planes, int64_t N, int64_t K, int r,
+                   uint8_t *codes_r)
+{
+    int64_t W = K / 32;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned q = 0;
+            for (int p = 0; p < r; ++p) {
+                uint32_t word = planes[((int64_t)p * N + n) * W + k / 32];
+                unsigned bit = (word >> (k % 32)) & 1u;
+                q = (q << 1) | bit;      /* plane 0 is the most significant */
+            }
+            codes_r[n * K + k] = (uint8_t)q;
+        }
+    }
+}
+
+/* The dequantized level of an r-bit code, exactly, in fp64. */
+static double level(unsigned q_r, int r)
+{
+    double a = (double)(1u << (8 - r));                 /* 2^(8-r) */
+    double b = (r == 8) ? 0.5 : (double)(1u << (7 - r)); /* 2^(7-r) */
+    return a * (double)q_r + b - 128.0;
+}
+
+/*
+ * Y[m, n] for every (m, n): X is M x K (bf16 values widened to fp64),
+ * codes N x K (parent, 8-bit), s16 N x (K/128) (the fp16-stored scales
+ * widened to fp64).  The r-bit slice is taken inside.
+ */
+void oracle_gemm_f64(const double *X, const uint8_t *codes, const double *s16,
+                     int64_t M, int64_t N, int64_t K, int r, double *Y)
+{
+    int64_t G = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                unsigned q_r = (unsigned)codes[n * K + k] >> (8 - r);
+                double w = s16[n * G + k / 128] * level(q_r, r);
+                acc += X[m * K + k] * w;
+            }
+            Y[m * N + n] = acc;
+        }
+    }
+}
+
+/* The same definition for a list of (m, n) output positions only. */
+void oracle_gemm_f64_at(const double *X, const uint8_t *codes,
+                        const double *s16, int64_t K, int r,
+                        int64_t count, const int64_t *ms, const int64_t *ns,
+                        double *out)
+{
+    int64_t G = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = ms[i], n = ns[i];
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned q_r = (unsigned)codes[n * K + k] >> (8 - r);
+            double w = s16[n * G + k / 128] * level(q_r, r);
+            acc += X[m * K + k] * w;
+        }
+        out[i] = acc;
+    }
+}
+
+/* Number of OpenMP threads the gemm loops use (1 without OpenMP). */
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
