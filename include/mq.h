@@ -1,0 +1,155 @@
+/*
+ * libmq -- nested (Matryoshka) r-bit weight GEMM for NVIDIA B200 (sm_100a).
+ *
+ * One 8-bit parent checkpoint serves every bit-width r = 1..8: the r-bit
+ * model is the top r bits of each parent code ("MatGPTQ: Efficient and
+ * Accurate Inference over Nested Quantized Models", abstract: lower-precision
+ * models are read from the parent by reading fewer bits, and the refined
+ * representation makes an r-bit model read exactly r bits; "MatGPTQ:
+ * Accurate and Efficient Post-Training Matryoshka Quantization", abstract:
+ * the most significant bits are sliced at inference time, with kernels for
+ * slicing and mixed-precision execution).
+ *
+ * Definitions used by every call:
+ *   q      parent code, uint8, N x K row-major (N output features, K inputs)
+ *   q_r    = q >> (8 - r)                               (top r bits)
+ *   v_r    = 2^(8-r) * q_r + 2^(7-r) - 128              (dequantized level)
+ *   s      per-group scale, one per 128 consecutive k, stored as fp16
+ *   W_r    [n, k] = s[n, k / 128] * v_r[n, k]
+ *   Y      = X . W_r^T, X is M x K bf16 row-major, Y is M x N bf16 row-major
+ *
+ * Storage ("bit planes"): planes[p][n][K/32] of uint32, p = 0..7, plane p
+ * holds bit (7 - p) of q (most significant plane first), and bit j of word w
+ * of row n holds the code of column k = 32 w + j.  One aligned 16-byte vector
+ * is one 128-column group of one plane.  The r-bit model is the prefix made
+ * of the first r planes (r * N * K / 8 bytes), so it reads exactly r bits
+ * per weight; planes of a weight set are always N * K / 32 words apart.
+ *
+ * Conventions:
+ *   - All pointers named *_dev are device pointers; the caller owns every
+ *     buffer and every stream.  The library allocates no device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *   - Calls are asynchronous on `stream` unless stated otherwise.  Argument
+ *     errors are returned before anything is launched.  Launch failures
+ *     return MQ_ERR_CUDA; the CUDA error text is kept for mq_last_error_string.
+ *   - fp16 and bf16 values are passed as their uint16_t bit patterns.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef MQ_H_
+#define MQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MQ_API __attribute__((visibility("default")))
+#else
+#define MQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MQ_OK = 0,
+    MQ_ERR_INVALID_ARG = 1,   /* null pointer, bad size, r or group out of range */
+    MQ_ERR_UNSUPPORTED = 2,   /* valid request the library does not serve (e.g. a scale that overflows fp16) */
+    MQ_ERR_MISALIGNED = 3,    /* pointer not 16-byte aligned */
+    MQ_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    MQ_ERR_TIMEOUT = 5,       /* a bounded device-side wait expired */
+    MQ_ERR_WORKSPACE = 6      /* workspace missing or smaller than mq_gemm_workspace_bytes */
+} mq_status;
+
+/* A view of an r-bit weight set inside a bit-plane buffer (no ownership). */
+typedef struct {
+    const uint32_t *planes;   /* device: plane 0 of the buffer; first r planes are read */
+    const uint16_t *scales;   /* device: fp16 scales, N x (K / group), row-major */
+    int64_t N;                /* output features (rows of W) */
+    int64_t K;                /* input features, multiple of 128 */
+    int32_t group;            /* columns per scale; must be 128 */
+    int32_t r;                /* bits per weight, 1..8 */
+} mq_weights;
+
+/* Bytes of the first r planes: r * N * K / 8 (0 on invalid arguments). */
+MQ_API size_t mq_plane_bytes(int64_t N, int64_t K, int r);
+
+/* Bytes of the fp16 scales: 2 * N * (K / group) (0 on invalid arguments). */
+MQ_API size_t mq_scale_bytes(int64_t N, int64_t K, int group);
+
+/*
+ * Pack parent codes into the 8 bit planes and round the scales to fp16.
+ * Follows the exact-r-bit storage of the MatGPTQ abstract (Table 1, "Exact
+ * r-bit loading"; "single multi-precision checkpoint").
+ *   codes_dev   uint8 N x K (row-major), the 8-bit parent codes
+ *   scales_dev  fp32 N x (K/group), the per-group scales
+ *   planes_out  uint32 [8][N][K/32] (mq_plane_bytes(N, K, 8) bytes)
+ *   scales_out  fp16 bits N x (K/group), round-to-nearest-even of scales_dev
+ * Preconditions: N >= 1, K >= 128, K % 128 == 0, group == 128, all four
+ * pointers 16-byte aligned, buffers do not overlap.
+ * Synchronous: returns after the work on `stream` has finished, because it
+ * reports MQ_ERR_UNSUPPORTED when any scale is negative, NaN or rounds to an
+ * fp16 infinity (the outputs are then unspecified).
+ */
+MQ_API mq_status mq_pack(const uint8_t *codes_dev, const float *scales_dev,
+                  int64_t N, int64_t K, int group,
+                  uint32_t *planes_out, uint16_t *scales_out, void *stream);
+
+/*
+ * Select the r-bit model of a parent: host-only, O(1), no device work and no
+ * copy.  `out` refers to the first r planes of `parent`'s buffer and to the
+ * same scales, so it lives as long as the parent's buffers.  MSB slicing per
+ * the MatGPTQ author-page abstract.  parent->r must be >= r (slicing is
+ * nested: the slice of a slice is the slice of the parent).
+ */
+MQ_API mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out);
+
+/*
+ * Bytes of device workspace mq_gemm needs for this problem (0 if none).
+ * The workspace holds split-K partial sums and arrival counters.
+ */
+MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+
+/*
+ * Y = X . W_r^T (MatGPTQ abstract: kernels for the nested format that serve
+ * batch sizes beyond one).  M <= 8 runs the split-K CUDA-core GEMV; M >= 9
+ * runs the tcgen05 tensor-core GEMM.
+ *   X_dev      bf16 M x K row-major
+ *   w          r-bit view (from mq_slice, or a parent with r = 8)
+ *   Y_dev      bf16 M x N row-major (written, not accumulated)
+ *   workspace  device buffer of at least mq_gemm_workspace_bytes(M, N, K, r)
+ *              bytes, zero-filled before its first use; every call leaves it
+ *              zero-filled again.  May be NULL when that size is 0.  Calls
+ *              that run concurrently must not share a workspace.
+ * Preconditions: M >= 1, w->N >= 1, w->K == K, K % 128 == 0, w->group == 128,
+ * 1 <= w->r <= 8, X/Y/planes/scales/workspace 16-byte aligned, Y does not
+ * overlap the inputs.  M == 0 is accepted and does nothing.
+ * The fp32 accumulation order is fixed, so results are deterministic.
+ */
+MQ_API mq_status mq_gemm(const uint16_t *X_dev, const mq_weights *w,
+                  int64_t M, int64_t N, int64_t K, uint16_t *Y_dev,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Test helper: codes_out[n, k] = q_r[n, k] read back from the first r planes
+ * (uint8 N x K row-major, device).  Same preconditions as mq_gemm on `w`.
+ */
+MQ_API mq_status mq_unpack(const mq_weights *w, uint8_t *codes_out, void *stream);
+
+/* Status of the most recent failing call on this host thread (MQ_OK if none). */
+MQ_API mq_status mq_last_error(void);
+
+/* Text of the most recent failure on this host thread (never NULL). */
+MQ_API const char *mq_last_error_string(void);
+
+/* Fixed description of a status code (never NULL). */
+MQ_API const char *mq_status_string(mq_status s);
+
+/* Library version, e.g. "0.1.0". */
+MQ_API const char *mq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MQ_H_ */

@@ -1,0 +1,172 @@
+"""Python binding of libmq (nested r-bit weight GEMM on B200).
+
+Argument marshalling only: every computation runs in libmq's CUDA kernels.
+The function names follow the C ABI in include/mq.h (mq_pack, mq_slice,
+mq_gemm, mq_unpack, ...).  PyTorch supplies device memory and streams.
+
+If libmq.so has not been built, importing this package raises; there is no
+CPU or PyTorch fallback for any step.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "MQError", "MqWeights", "NestedWeights", "lib", "library_path",
+    "mq_plane_bytes", "mq_scale_bytes", "mq_pack", "mq_slice", "mq_gemm",
+    "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libmq.so")
+
+MQ_OK = 0
+STATUS = {0: "MQ_OK", 1: "MQ_ERR_INVALID_ARG", 2: "MQ_ERR_UNSUPPORTED",
+          3: "MQ_ERR_MISALIGNED", 4: "MQ_ERR_CUDA", 5: "MQ_ERR_TIMEOUT",
+          6: "MQ_ERR_WORKSPACE"}
+
+
+class MQError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+class MqWeights(ctypes.Structure):
+    """Mirror of the C struct mq_weights (a view, owns nothing)."""
+    _fields_ = [("planes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+                ("group", ctypes.c_int32), ("r", ctypes.c_int32)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(library_path):
+        raise ImportError(
+            f"{library_path} is missing: build it with "
+            "`python -m nested_bit_weight_b200._build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(library_path)
+    P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    W = ctypes.POINTER(MqWeights)
+    sig = {
+        "mq_plane_bytes": (SZ, [I64, I64, I]),
+        "mq_scale_bytes": (SZ, [I64, I64, I]),
+        "mq_pack": (I, [P, P, I64, I64, I, P, P, P]),
+        "mq_slice": (I, [W, I, W]),
+        "mq_gemm_workspace_bytes": (SZ, [I64, I64, I64, I]),
+        "mq_gemm": (I, [P, W, I64, I64, I64, P, P, SZ, P]),
+        "mq_unpack": (I, [W, P, P]),
+        "mq_last_error": (I, []),
+        "mq_last_error_string": (ctypes.c_char_p, []),
+        "mq_status_string": (ctypes.c_char_p, [I]),
+        "mq_version": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int) -> None:
+    if status != MQ_OK:
+        raise MQError(status, lib.mq_last_error_string().decode())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+# ------------------------------------------------------------------ raw C ABI
+
+def mq_plane_bytes(N: int, K: int, r: int) -> int:
+    return lib.mq_plane_bytes(N, K, r)
+
+
+def mq_scale_bytes(N: int, K: int, group: int = 128) -> int:
+    return lib.mq_scale_bytes(N, K, group)
+
+
+def mq_gemm_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return lib.mq_gemm_workspace_bytes(M, N, K, r)
+
+
+def mq_version() -> str:
+    return lib.mq_version().decode()
+
+
+def mq_pack(codes, scales, planes_out, scales_out, stream=None) -> None:
+    """codes uint8 [N, K], scales fp32 [N, K/128] -> planes_out (>= 8 planes
+    of uint32 words), scales_out (fp16 or int16 [N, K/128]); all on device."""
+    N, K = codes.shape
+    _check(lib.mq_pack(codes.data_ptr(), scales.data_ptr(), N, K, 128,
+                       planes_out.data_ptr(), scales_out.data_ptr(), _stream(stream)))
+
+
+def mq_slice(parent: MqWeights, r: int) -> MqWeights:
+    out = MqWeights()
+    _check(lib.mq_slice(ctypes.byref(parent), r, ctypes.byref(out)))
+    return out
+
+
+def mq_gemm(X, w: MqWeights, Y, workspace=None, stream=None) -> None:
+    """Y[M, N] = X[M, K] . W_r^T (bf16 device tensors)."""
+    M, K = X.shape
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.mq_gemm(X.data_ptr(), ctypes.byref(w), M, w.N, K, Y.data_ptr(),
+                       ws_ptr, ws_bytes, _stream(stream)))
+
+
+def mq_unpack(w: MqWeights, codes_out, stream=None) -> None:
+    _check(lib.mq_unpack(ctypes.byref(w), codes_out.data_ptr(), _stream(stream)))
+
+
+# ------------------------------------------------------------- owning helpers
+
+class NestedWeights:
+    """A packed 8-bit parent (device tensors) and its r-bit views."""
+
+    def __init__(self, planes, scales16, N: int, K: int):
+        self.planes, self.scales16, self.N, self.K = planes, scales16, N, K
+        self.parent = MqWeights(planes.data_ptr(), scales16.data_ptr(), N, K, 128, 8)
+
+    def view(self, r: int) -> MqWeights:
+        return mq_slice(self.parent, r)
+
+
+def pack_parent(codes, scales, stream=None) -> NestedWeights:
+    """Allocate the 8-plane buffer and fp16 scales with torch, then mq_pack."""
+    import torch
+    N, K = codes.shape
+    planes = torch.empty(mq_plane_bytes(N, K, 8) // 4, dtype=torch.int32, device=codes.device)
+    s16 = torch.empty((N, K // 128), dtype=torch.float16, device=codes.device)
+    mq_pack(codes, scales, planes, s16, stream)
+    return NestedWeights(planes, s16, N, K)
+
+
+_ws_cache: dict = {}
+
+
+def gemm(X, weights: NestedWeights, r: int, Y=None, stream=None):
+    """Y = X . W_r^T with a cached, zero-initialised workspace per device."""
+    import torch
+    M, K = X.shape
+    w = weights.view(r)
+    if Y is None:
+        Y = torch.empty((M, weights.N), dtype=torch.bfloat16, device=X.device)
+    need = mq_gemm_workspace_bytes(M, weights.N, K, r)
+    ws = None
+    if need:
+        key = X.device.index
+        ws = _ws_cache.get(key)
+        if ws is None or ws.numel() < need:
+            ws = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=X.device)
+            _ws_cache[key] = ws
+    mq_gemm(X, w, Y, ws, stream)
+    return Y

@@ -1,0 +1,154 @@
+// C-ABI entry points of libmq that are not kernels: argument checks, the
+// O(1) slice, sizes, dispatch between the GEMV and the tensor-core GEMM, and
+// error reporting.
+#include <stdarg.h>
+#include <string.h>
+
+#include "mq_common.cuh"
+
+namespace mq {
+
+static thread_local mq_status g_last = MQ_OK;
+static thread_local char g_msg[512] = "no error";
+
+void set_error(mq_status s, const char *fmt, ...) {
+    g_last = s;
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+    va_end(ap);
+}
+
+mq_status cuda_fail(cudaError_t e, const char *where) {
+    set_error(MQ_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+    return MQ_ERR_CUDA;
+}
+
+// Driver calls reached through the runtime's entry-point query, so the library
+// has no link-time dependency on libcuda (it loads on machines without a GPU).
+typedef int (*CtxGetCurrentFn)(void **);
+typedef int (*CtxGetDeviceFn)(int *);
+
+static int current_context_device() {
+    static CtxGetCurrentFn get_ctx = nullptr;
+    static CtxGetDeviceFn get_dev = nullptr;
+    static bool looked_up = false;
+    if (!looked_up) {
+        cudaDriverEntryPointQueryResult q;
+        cudaGetDriverEntryPoint("cuCtxGetCurrent", (void **)&get_ctx, cudaEnableDefault, &q);
+        cudaGetDriverEntryPoint("cuCtxGetDevice", (void **)&get_dev, cudaEnableDefault, &q);
+        looked_up = true;
+    }
+    void *ctx = nullptr;
+    int dev = -1;
+    if (!get_ctx || !get_dev || get_ctx(&ctx) != 0 || !ctx || get_dev(&dev) != 0) return -1;
+    return dev;
+}
+
+mq_status bind_device(cudaStream_t st) {
+    static thread_local cudaStream_t last_stream = nullptr;
+    if (st != nullptr && st == last_stream) return MQ_OK;
+    int dev = -1;
+    if (st != nullptr) {
+        cudaError_t e = cudaStreamGetDevice(st, &dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamGetDevice");
+    } else {
+        dev = current_context_device();   // legacy stream: the caller's context
+        if (dev < 0) return MQ_OK;
+    }
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess || cur != dev) {
+        cudaError_t e = cudaSetDevice(dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaSetDevice");
+    }
+    last_stream = st;
+    return MQ_OK;
+}
+
+mq_status check_weights(const mq_weights *w, int64_t N, int64_t K) {
+    if (!w) return fail(MQ_ERR_INVALID_ARG, "weights view is NULL");
+    if (!w->planes || !w->scales)
+        return fail(MQ_ERR_INVALID_ARG, "weights view has a NULL buffer");
+    if (w->r < 1 || w->r > 8) return fail(MQ_ERR_INVALID_ARG, "r must be in 1..8");
+    if (w->group != kGroup) return fail(MQ_ERR_INVALID_ARG, "group must be 128");
+    if (w->N != N || w->K != K)
+        return fail(MQ_ERR_INVALID_ARG, "weights view shape differs from (N, K)");
+    if (N < 1 || K < kGroup || K % kGroup)
+        return fail(MQ_ERR_INVALID_ARG, "need N >= 1 and K a positive multiple of 128");
+    if (!aligned16(w->planes) || !aligned16(w->scales))
+        return fail(MQ_ERR_MISALIGNED, "planes and scales must be 16-byte aligned");
+    return MQ_OK;
+}
+
+}  // namespace mq
+
+using namespace mq;
+
+extern "C" {
+
+size_t mq_plane_bytes(int64_t N, int64_t K, int r) {
+    if (N < 1 || K < kGroup || K % kGroup || r < 1 || r > 8) return 0;
+    return (size_t)r * (size_t)N * (size_t)K / 8;
+}
+
+size_t mq_scale_bytes(int64_t N, int64_t K, int group) {
+    if (N < 1 || K < kGroup || K % kGroup || group != kGroup) return 0;
+    return 2 * (size_t)N * (size_t)(K / group);
+}
+
+mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out) {
+    if (!parent || !out) return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_slice");
+    if (r < 1 || r > 8) return fail(MQ_ERR_INVALID_ARG, "r must be in 1..8");
+    if (parent->r < r)
+        return fail(MQ_ERR_INVALID_ARG, "cannot slice to more bits than the parent has");
+    mq_status s = check_weights(parent, parent->N, parent->K);
+    if (s != MQ_OK) return s;
+    *out = *parent;   // same buffer: the first r planes are the r-bit model
+    out->r = r;
+    return MQ_OK;
+}
+
+size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+    if (M < 1 || N < 1 || K < kGroup || K % kGroup || r < 1 || r > 8) return 0;
+    if (M <= kGemvMaxM) return gemv_workspace_bytes(M, N, K, r);
+    return gemm_tc_workspace_bytes(M, N, K, r);
+}
+
+mq_status mq_gemm(const uint16_t *X, const mq_weights *w, int64_t M, int64_t N,
+                  int64_t K, uint16_t *Y, void *workspace, size_t workspace_bytes,
+                  void *stream) {
+    mq_status s = check_weights(w, N, K);
+    if (s != MQ_OK) return s;
+    if (M < 0) return fail(MQ_ERR_INVALID_ARG, "M must be >= 0");
+    if (M == 0) return MQ_OK;
+    if (!X || !Y) return fail(MQ_ERR_INVALID_ARG, "X or Y is NULL");
+    if (!aligned16(X) || !aligned16(Y) || (workspace && !aligned16(workspace)))
+        return fail(MQ_ERR_MISALIGNED, "X, Y and workspace must be 16-byte aligned");
+    size_t need = mq_gemm_workspace_bytes(M, N, K, w->r);
+    if (need && (!workspace || workspace_bytes < need))
+        return fail(MQ_ERR_WORKSPACE, "workspace smaller than mq_gemm_workspace_bytes");
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((s = bind_device(st)) != MQ_OK) return s;
+    if (M <= kGemvMaxM) return launch_gemv(X, w, M, Y, workspace, workspace_bytes, st);
+    return launch_gemm_tc(X, w, M, Y, workspace, workspace_bytes, st);
+}
+
+mq_status mq_last_error(void) { return g_last; }
+const char *mq_last_error_string(void) { return g_msg; }
+
+const char *mq_status_string(mq_status s) {
+    switch (s) {
+        case MQ_OK: return "ok";
+        case MQ_ERR_INVALID_ARG: return "invalid argument";
+        case MQ_ERR_UNSUPPORTED: return "unsupported";
+        case MQ_ERR_MISALIGNED: return "misaligned pointer";
+        case MQ_ERR_CUDA: return "CUDA error";
+        case MQ_ERR_TIMEOUT: return "device wait timed out";
+        case MQ_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+const char *mq_version(void) { return "0.1.0"; }
+
+}  // extern "C"

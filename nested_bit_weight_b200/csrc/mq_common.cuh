@@ -1,0 +1,47 @@
+// Internal helpers shared by the libmq translation units (not installed).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "../../include/mq.h"
+
+namespace mq {
+
+constexpr int kGroup = 128;          // columns per scale
+constexpr int kPlanes = 8;           // planes in a parent buffer
+
+// Per-host-thread record of the last failure (mq_last_error*).
+void set_error(mq_status s, const char *fmt, ...);
+inline mq_status fail(mq_status s, const char *what) {
+    set_error(s, "%s", what);
+    return s;
+}
+mq_status cuda_fail(cudaError_t e, const char *where);
+
+inline bool aligned16(const void *p) {
+    return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;
+}
+
+// Make the stream's device current for this library's runtime (the library
+// links its own CUDA runtime, whose current device is not the caller's).
+mq_status bind_device(cudaStream_t st);
+
+// Validate a weight view against (N, K); returns MQ_OK or the failing status.
+mq_status check_weights(const mq_weights *w, int64_t N, int64_t K);
+
+// Kernel launchers (each returns MQ_OK or MQ_ERR_CUDA after the launch).
+size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+mq_status launch_gemv(const uint16_t *X, const mq_weights *w, int64_t M,
+                      uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
+size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M,
+                         uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
+
+// Largest M served by the CUDA-core GEMV; larger M runs the tcgen05 GEMM.
+constexpr int kGemvMaxM = 8;
+
+}  // namespace mq

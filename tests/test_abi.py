@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+bad arguments with the documented status before touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nested_bit_weight_b200 as mq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names |= set(re.findall(r"MQ_API[^;(]*?\b(mq_\w+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert {"mq_pack", "mq_slice", "mq_gemm", "mq_unpack"} <= names
+    raw = ctypes.CDLL(mq.library_path)
+    for n in sorted(names):
+        assert hasattr(raw, n), n
+
+
+def test_sizes():
+    assert mq.mq_plane_bytes(4096, 4096, 2) == 2 * 4096 * 4096 // 8
+    assert mq.mq_plane_bytes(4096, 4096, 8) == 4096 * 4096
+    assert mq.mq_scale_bytes(4096, 4096) == 2 * 4096 * 32
+    assert mq.mq_plane_bytes(4, 100, 2) == 0          # K not a multiple of 128
+    assert mq.mq_plane_bytes(4, 128, 9) == 0
+    assert mq.mq_scale_bytes(4, 256, 64) == 0
+    assert mq.mq_gemm_workspace_bytes(0, 4, 128, 2) == 0
+    assert mq.mq_version() == "0.1.0"
+
+
+FAKE = 0x10000   # an aligned address; these calls must fail before any access
+
+
+def _parent(N=64, K=256, r=8, planes=FAKE, scales=FAKE * 2):
+    return mq.MqWeights(planes, scales, N, K, 128, r)
+
+
+def test_slice_is_a_prefix_view():
+    p = _parent()
+    for r in range(1, 9):
+        v = mq.mq_slice(p, r)
+        assert (v.planes, v.scales, v.N, v.K, v.group, v.r) == (p.planes, p.scales, 64, 256, 128, r)
+    v4 = mq.mq_slice(p, 4)
+    assert mq.mq_slice(v4, 2).r == 2                  # nested
+    with pytest.raises(mq.MQError) as e:
+        mq.mq_slice(v4, 5)                            # more bits than the parent has
+    assert e.value.status == 1
+    for bad in (0, 9):
+        with pytest.raises(mq.MQError):
+            mq.mq_slice(p, bad)
+
+
+def _gemm_status(M=1, N=64, K=256, r=4, X=FAKE, Y=FAKE, w=None, ws=None, wsb=0):
+    w = w if w is not None else _parent(N, K, r)
+    return mq.lib.mq_gemm(X, ctypes.byref(w), M, N, K, Y, ws, wsb, None)
+
+
+def test_gemm_argument_errors_before_launch():
+    assert _gemm_status(M=0) == 0                                 # nothing to do
+    assert _gemm_status(X=None) == 1
+    assert _gemm_status(X=FAKE + 2) == 3                          # misaligned X
+    assert _gemm_status(Y=FAKE + 8) == 3
+    assert _gemm_status(w=_parent(planes=FAKE + 4)) == 3
+    assert _gemm_status(N=32, w=_parent(N=64)) == 1                 # view shape mismatch
+    assert _gemm_status(w=mq.MqWeights(FAKE, FAKE, 64, 200, 128, 4), K=200) == 1
+    assert _gemm_status(w=mq.MqWeights(FAKE, FAKE, 64, 256, 64, 4)) == 1   # group
+    assert _gemm_status(w=mq.MqWeights(FAKE, FAKE, 64, 256, 128, 0)) == 1  # r
+    assert _gemm_status(M=-1) == 1
+    need = mq.mq_gemm_workspace_bytes(1, 64, 1 << 16, 2)
+    assert need > 0
+    assert _gemm_status(N=64, K=1 << 16, r=2, ws=None) == 6
+    assert _gemm_status(N=64, K=1 << 16, r=2, ws=FAKE, wsb=need - 1) == 6
+    assert mq.lib.mq_status_string(6) == b"workspace missing or too small"
+
+
+def test_pack_unpack_argument_errors():
+    L = mq.lib
+    assert L.mq_pack(None, FAKE, 4, 128, 128, FAKE, FAKE, None) == 1
+    assert L.mq_pack(FAKE, FAKE, 4, 100, 128, FAKE, FAKE, None) == 1
+    assert L.mq_pack(FAKE, FAKE, 4, 128, 64, FAKE, FAKE, None) == 1
+    assert L.mq_pack(FAKE + 1, FAKE, 4, 128, 128, FAKE, FAKE, None) == 3
+    w = _parent()
+    assert L.mq_unpack(ctypes.byref(w), None, None) == 1
+    assert L.mq_unpack(ctypes.byref(w), FAKE + 3, None) == 3
+    assert L.mq_unpack(None, FAKE, None) == 1
+    assert b"16-byte" in L.mq_last_error_string() or L.mq_last_error() == 1

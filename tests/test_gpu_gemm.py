@@ -1,0 +1,118 @@
+"""GPU parity of mq_gemm against the fp64 CPU oracle.
+
+Pass criterion (per element): |Y - Y_ref| <= 8e-3 |Y_ref| + 1e-3 rms(Y_ref),
+rms over the whole output (oracle.violation_ratio <= 1).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(codes, s, xbits, r, parent=None):
+    import torch
+    import nested_bit_weight_b200 as mq
+    if parent is None:
+        parent = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    X = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = mq.gemm(X, parent, r)
+    torch.cuda.synchronize()
+    return Y.float().cpu().numpy().astype(np.float64), parent
+
+
+def _case(N, K, M, r, seed, outliers=False):
+    codes, s, _ = wl.gen_weights(N, K, seed)
+    xbits, X = wl.gen_x(M, K, seed, outlier_channels=outliers)
+    Y, _ = _run(codes, s, xbits, r)
+    Yref = oracle.gemm(X, codes, s, r)
+    return oracle.violation_ratio(Y, Yref)
+
+
+@pytest.mark.parametrize("r", [8, 7, 6, 5, 4, 3, 2, 1])
+def test_single_layer_512(r):
+    # the 512 x 512 single-layer workload at M = 1, seed 0
+    assert _case(512, 512, 1, r, wl.layer_seed(0, 0)) <= 1.0
+
+
+def test_golden_samples_config0():
+    import json, os
+    g = json.load(open(os.path.join(os.path.dirname(__file__), "golden",
+                                    "config0_samples.json")))
+    codes, s, _ = wl.gen_weights(512, 512, wl.layer_seed(0, 0))
+    xbits, X = wl.gen_x(1, 512, wl.layer_seed(0, 0))
+    parent = None
+    for r, vals in g["Y"].items():
+        Y, parent = _run(codes, s, xbits, int(r), parent)
+        ref = np.array([float.fromhex(v) for v in vals])
+        Yref_full = oracle.gemm(X, codes, s, int(r))[0]
+        rms = float(np.sqrt(np.mean(Yref_full ** 2)))
+        assert oracle.violation_ratio(Y[0, g["columns"]], ref, rms) <= 1.0
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("r", [2, 3, 4, 8])
+@pytest.mark.parametrize("N,K", [(37, 384), (300, 1408), (1, 128), (130, 2048)])
+def test_gemv_ragged(N, K, M, r):
+    assert _case(N, K, M, r, seed=N * 7 + K + M) <= 1.0
+
+
+@pytest.mark.parametrize("M", [9, 12, 15, 16, 33, 64])
+@pytest.mark.parametrize("r", [2, 4, 8])
+def test_batched_ragged(M, r):
+    assert _case(200, 640, M, r, seed=M + r) <= 1.0
+
+
+@pytest.mark.parametrize("kind", ["zeros", "ones", "alternating", "single_bit"])
+@pytest.mark.parametrize("r", [1, 2, 3, 4, 8])
+def test_adversarial_codes(kind, r):
+    N, K, M = 64, 512, 3
+    codes = wl.adversarial_codes(kind, N, K)
+    s = wl.gen_scales(N, K, seed=5, zero_groups=17)
+    xbits, X = wl.gen_x(M, K, seed=5)
+    Y, _ = _run(codes, s, xbits, r)
+    Yref = oracle.gemm(X, codes, s, r)
+    assert oracle.violation_ratio(Y, Yref) <= 1.0
+
+
+def test_all_zero_scales_give_zero():
+    N, K = 16, 256
+    codes = wl.adversarial_codes("random", N, K)
+    s = np.zeros((N, K // 128), np.float32)
+    xbits, _ = wl.gen_x(2, K, seed=1)
+    Y, _ = _run(codes, s, xbits, 4)
+    assert np.all(Y == 0.0)
+
+
+def test_deterministic_and_workspace_reusable():
+    # split-K shape: the arrival tickets must be back at zero after each call,
+    # otherwise a later call would skip the final reduction (NaN survives)
+    import torch
+    import nested_bit_weight_b200 as mq
+    N, K = 1024, 14336
+    assert mq.mq_gemm_workspace_bytes(1, N, K, 3) > 0
+    codes, s, _ = wl.gen_weights(N, K, seed=9)
+    xbits, X = wl.gen_x(1, K, seed=9)
+    parent = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    Xd = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+    outs = []
+    for _ in range(3):
+        Y = torch.full((1, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        mq.gemm(Xd, parent, 3, Y=Y)
+        outs.append(Y.float().cpu().numpy())
+    assert not np.isnan(outs[0]).any()
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+    assert oracle.violation_ratio(outs[0], oracle.gemm(X, codes, s, 3)) <= 1.0
+
+
+LLAMA = [(l.name, l.N, l.K) for l in wl.LLAMA8B]
+
+
+@pytest.mark.parametrize("r", [4, 3, 2])
+@pytest.mark.parametrize("name,N,K", LLAMA)
+def test_llama_layers_full_m1(name, N, K, r):
+    # full-size decode layers at M = 1: every output against the oracle
+    seed = wl.layer_seed(1, [l[0] for l in LLAMA].index(name))
+    assert _case(N, K, 1, r, seed) <= 1.0
