@@ -118,9 +118,11 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  *   w          r-bit view (from mq_slice, or a parent with r = 8)
  *   Y_dev      bf16 M x N row-major (written, not accumulated)
  *   workspace  device buffer of at least mq_gemm_workspace_bytes(M, N, K, r)
- *              bytes, zero-filled before its first use; every call leaves it
- *              zero-filled again.  May be NULL when that size is 0.  Calls
- *              that run concurrently must not share a workspace.
+ *              bytes whose first 64 KiB (arrival tickets) are zero-filled
+ *              before its first use; every call leaves those 64 KiB zero
+ *              again, so one workspace serves calls of any shape in stream
+ *              order.  May be NULL when the size is 0.  Calls that run
+ *              concurrently must not share a workspace.
  * Preconditions: M >= 1, w->N >= 1, w->K == K, K % 128 == 0, w->group == 128,
  * 1 <= w->r <= 8, X/Y/planes/scales/workspace 16-byte aligned, Y does not
  * overlap the inputs.  M == 0 is accepted and does nothing.

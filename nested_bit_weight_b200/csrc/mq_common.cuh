@@ -13,6 +13,9 @@ namespace mq {
 
 constexpr int kGroup = 128;          // columns per scale
 constexpr int kPlanes = 8;           // planes in a parent buffer
+// Split-K arrival tickets live in the first kTicketBytes of every workspace;
+// each call returns the tickets it used to zero.
+constexpr size_t kTicketBytes = 64 * 1024;
 
 // Per-host-thread record of the last failure (mq_last_error*).
 void set_error(mq_status s, const char *fmt, ...);

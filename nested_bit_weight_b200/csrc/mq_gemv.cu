@@ -22,7 +22,7 @@ constexpr int kXPad = 4;                 // floats of padding per staged group
 struct GemvPlan {
     int MB, Gc, RT, KS, B;               // B = row blocks per CTA
     int64_t tiles;                       // CTAs along N
-    size_t part_bytes, ws_bytes;
+    size_t part_bytes, ws_bytes;          // part_bytes: offset of the partial sums
 };
 
 int pow2_floor(int64_t v) { int p = 1; while ((int64_t)p * 2 <= v) p *= 2; return p; }
@@ -47,8 +47,10 @@ GemvPlan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     }
     p.tiles = (N + (int64_t)p.B * p.RT - 1) / ((int64_t)p.B * p.RT);
     if (p.KS > 1) {
-        p.part_bytes = ((size_t)p.KS * M * N * sizeof(float) + 255) & ~(size_t)255;
-        p.ws_bytes = p.part_bytes + (((size_t)p.tiles * sizeof(unsigned) + 255) & ~(size_t)255);
+        // tickets first, at a fixed place: a call with a different shape must
+        // never find another call's partial sums where its tickets live
+        p.part_bytes = kTicketBytes;
+        p.ws_bytes = kTicketBytes + (((size_t)p.KS * M * N * sizeof(float) + 255) & ~(size_t)255);
     }
     return p;
 }
@@ -305,9 +307,11 @@ mq_status launch_gemv(const uint16_t *X, const mq_weights *w, int64_t M, uint16_
                       void *ws, size_t ws_bytes, cudaStream_t st) {
     const GemvPlan p = make_plan(M, w->N, w->K, w->r);
     if (p.ws_bytes > ws_bytes) return fail(MQ_ERR_WORKSPACE, "GEMV workspace too small");
-    float *part = p.KS > 1 ? reinterpret_cast<float *>(ws) : nullptr;
-    unsigned *tickets = p.KS > 1
-        ? reinterpret_cast<unsigned *>(static_cast<char *>(ws) + p.part_bytes) : nullptr;
+    if (p.KS > 1 && p.tiles > (int64_t)(kTicketBytes / sizeof(unsigned)))
+        return fail(MQ_ERR_UNSUPPORTED, "too many row tiles for the split-K ticket region");
+    unsigned *tickets = p.KS > 1 ? reinterpret_cast<unsigned *>(ws) : nullptr;
+    float *part = p.KS > 1
+        ? reinterpret_cast<float *>(static_cast<char *>(ws) + kTicketBytes) : nullptr;
     const size_t smem = (size_t)p.MB * p.Gc * (kGroup + kXPad) * sizeof(float);
     dim3 grid((unsigned)p.tiles, (unsigned)p.KS);
     GemvFn fn = pick(w->r, p.MB, p.RT);

@@ -116,3 +116,21 @@ def test_llama_layers_full_m1(name, N, K, r):
     # full-size decode layers at M = 1: every output against the oracle
     seed = wl.layer_seed(1, [l[0] for l in LLAMA].index(name))
     assert _case(N, K, 1, r, seed) <= 1.0
+
+
+def test_workspace_shared_across_shapes():
+    # a larger split-K call followed by a smaller one on the same workspace
+    import torch
+    import nested_bit_weight_b200 as mq
+    N, K = 37, 384
+    codes, s, _ = wl.gen_weights(N, K, seed=77)
+    parent = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    need = max(mq.mq_gemm_workspace_bytes(M, N, K, r) for M in (1, 8) for r in (2, 3))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    for M, r in ((8, 2), (1, 3), (8, 3), (1, 2)):
+        xbits, X = wl.gen_x(M, K, seed=M)
+        Xd = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        mq.mq_gemm(Xd, parent.view(r), Y, ws)
+        Yh = Y.float().cpu().numpy()
+        assert oracle.violation_ratio(Yh, oracle.gemm(X, codes, s, r)) <= 1.0
