@@ -112,8 +112,8 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
 /*
  * Y = X . W_r^T (MatGPTQ abstract: kernels for the nested format that serve
- * batch sizes beyond one).  M <= 8 runs the split-K CUDA-core GEMV; M >= 9
- * runs the tcgen05 tensor-core GEMM.
+ * batch sizes beyond one).  M <= 8 runs a split-K GEMV (see
+ * mq_set_gemv_variant); M >= 9 runs the tcgen05 tensor-core GEMM.
  *   X_dev      bf16 M x K row-major
  *   w          r-bit view (from mq_slice, or a parent with r = 8)
  *   Y_dev      bf16 M x N row-major (written, not accumulated)
@@ -131,6 +131,24 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 MQ_API mq_status mq_gemm(const uint16_t *X_dev, const mq_weights *w,
                   int64_t M, int64_t N, int64_t K, uint16_t *Y_dev,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Kernels for M <= 8 (both compute the same Y within the stated tolerance). */
+enum {
+    MQ_GEMV_MMA = 0,   /* default: bf16 operands built in registers, warp MMA m16n8k16 */
+    MQ_GEMV_SIMT = 1   /* CUDA-core fp32 FMA GEMV with warp-shuffle reduction */
+};
+
+/*
+ * Choose the M <= 8 kernel for later mq_gemm calls in this process (host
+ * only, no device work).  Returns MQ_ERR_INVALID_ARG for an unknown value.
+ * Both variants follow the same definition of Y (MatGPTQ abstract: kernels
+ * for slicing and mixed-precision execution); they differ only in which
+ * units do the multiply-adds.
+ */
+MQ_API mq_status mq_set_gemv_variant(int variant);
+
+/* The M <= 8 kernel in use (MQ_GEMV_MMA or MQ_GEMV_SIMT). */
+MQ_API int mq_get_gemv_variant(void);
 
 /*
  * Test helper: codes_out[n, k] = q_r[n, k] read back from the first r planes

@@ -16,6 +16,7 @@ __all__ = [
     "MQError", "MqWeights", "NestedWeights", "lib", "library_path",
     "mq_plane_bytes", "mq_scale_bytes", "mq_pack", "mq_slice", "mq_gemm",
     "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
+    "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_MMA", "GEMV_SIMT",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -60,6 +61,8 @@ def _load() -> ctypes.CDLL:
         "mq_last_error_string": (ctypes.c_char_p, []),
         "mq_status_string": (ctypes.c_char_p, [I]),
         "mq_version": (ctypes.c_char_p, []),
+        "mq_set_gemv_variant": (I, [I]),
+        "mq_get_gemv_variant": (I, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -94,6 +97,17 @@ def mq_scale_bytes(N: int, K: int, group: int = 128) -> int:
 
 def mq_gemm_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
     return lib.mq_gemm_workspace_bytes(M, N, K, r)
+
+
+GEMV_MMA, GEMV_SIMT = 0, 1
+
+
+def mq_set_gemv_variant(variant: int) -> None:
+    _check(lib.mq_set_gemv_variant(variant))
+
+
+def mq_get_gemv_variant() -> int:
+    return lib.mq_get_gemv_variant()
 
 
 def mq_version() -> str:

@@ -9,6 +9,7 @@
 namespace mq {
 
 static thread_local mq_status g_last = MQ_OK;
+static int g_gemv_variant = MQ_GEMV_MMA;   // process-wide kernel choice for M <= 8
 static thread_local char g_msg[512] = "no error";
 
 void set_error(mq_status s, const char *fmt, ...) {
@@ -110,7 +111,10 @@ mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out) {
 
 size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
     if (M < 1 || N < 1 || K < kGroup || K % kGroup || r < 1 || r > 8) return 0;
-    if (M <= kGemvMaxM) return gemv_workspace_bytes(M, N, K, r);
+    if (M <= kGemvMaxM) {
+        const size_t a = gemv_workspace_bytes(M, N, K, r), b = gemv_mma_workspace_bytes(M, N, K, r);
+        return a > b ? a : b;
+    }
     return gemm_tc_workspace_bytes(M, N, K, r);
 }
 
@@ -129,9 +133,22 @@ mq_status mq_gemm(const uint16_t *X, const mq_weights *w, int64_t M, int64_t N,
         return fail(MQ_ERR_WORKSPACE, "workspace smaller than mq_gemm_workspace_bytes");
     cudaStream_t st = (cudaStream_t)stream;
     if ((s = bind_device(st)) != MQ_OK) return s;
-    if (M <= kGemvMaxM) return launch_gemv(X, w, M, Y, workspace, workspace_bytes, st);
+    if (M <= kGemvMaxM) {
+        if (__atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) == MQ_GEMV_SIMT)
+            return launch_gemv(X, w, M, Y, workspace, workspace_bytes, st);
+        return launch_gemv_mma(X, w, M, Y, workspace, workspace_bytes, st);
+    }
     return launch_gemm_tc(X, w, M, Y, workspace, workspace_bytes, st);
 }
+
+mq_status mq_set_gemv_variant(int variant) {
+    if (variant != MQ_GEMV_MMA && variant != MQ_GEMV_SIMT)
+        return fail(MQ_ERR_INVALID_ARG, "unknown GEMV variant");
+    __atomic_store_n(&g_gemv_variant, variant, __ATOMIC_RELAXED);
+    return MQ_OK;
+}
+
+int mq_get_gemv_variant(void) { return __atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED); }
 
 mq_status mq_last_error(void) { return g_last; }
 const char *mq_last_error_string(void) { return g_msg; }

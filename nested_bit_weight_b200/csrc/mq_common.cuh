@@ -40,6 +40,9 @@ mq_status check_weights(const mq_weights *w, int64_t N, int64_t K);
 size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 mq_status launch_gemv(const uint16_t *X, const mq_weights *w, int64_t M,
                       uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
+size_t gemv_mma_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+mq_status launch_gemv_mma(const uint16_t *X, const mq_weights *w, int64_t M,
+                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M,
                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);

@@ -52,11 +52,42 @@ def test_golden_samples_config0():
         assert oracle.violation_ratio(Y[0, g["columns"]], ref, rms) <= 1.0
 
 
+@pytest.fixture(params=["mma", "simt"])
+def gemv_variant(request):
+    import nested_bit_weight_b200 as mq
+    old = mq.mq_get_gemv_variant()
+    mq.mq_set_gemv_variant(mq.GEMV_MMA if request.param == "mma" else mq.GEMV_SIMT)
+    yield request.param
+    mq.mq_set_gemv_variant(old)
+
+
 @pytest.mark.parametrize("M", [1, 2, 3, 4, 5, 6, 7, 8])
-@pytest.mark.parametrize("r", [2, 3, 4, 8])
+@pytest.mark.parametrize("r", [1, 2, 3, 4, 5, 6, 7, 8])
 @pytest.mark.parametrize("N,K", [(37, 384), (300, 1408), (1, 128), (130, 2048)])
-def test_gemv_ragged(N, K, M, r):
+def test_gemv_ragged(N, K, M, r, gemv_variant):
     assert _case(N, K, M, r, seed=N * 7 + K + M) <= 1.0
+
+
+@pytest.mark.parametrize("r", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_gemv_one_hot_columns(r, gemv_variant):
+    # X = e_k picks column k of W_r: every column position of a group, exactly
+    # up to the bf16 rounding of the output
+    import torch
+    import nested_bit_weight_b200 as mq
+    N, K = 48, 256
+    codes = wl.adversarial_codes("random", N, K, seed=r)
+    s = wl.gen_scales(N, K, seed=r)
+    parent = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    W = oracle.dequant(codes, s, r)
+    M = 8
+    for k0 in range(0, K, M):
+        X = np.zeros((M, K), np.float32)
+        for m in range(M):
+            X[m, k0 + m] = 1.0
+        Xd = torch.from_numpy(X).cuda().to(torch.bfloat16)
+        Y = mq.gemm(Xd, parent, r).float().cpu().numpy()
+        want = W[:, k0:k0 + M].T
+        assert np.allclose(Y, want, rtol=2 ** -8, atol=0), (r, k0)
 
 
 @pytest.mark.parametrize("M", [9, 12, 15, 16, 33, 64])
@@ -112,7 +143,7 @@ LLAMA = [(l.name, l.N, l.K) for l in wl.LLAMA8B]
 
 @pytest.mark.parametrize("r", [4, 3, 2])
 @pytest.mark.parametrize("name,N,K", LLAMA)
-def test_llama_layers_full_m1(name, N, K, r):
+def test_llama_layers_full_m1(name, N, K, r, gemv_variant):
     # full-size decode layers at M = 1: every output against the oracle
     seed = wl.layer_seed(1, [l[0] for l in LLAMA].index(name))
     assert _case(N, K, 1, r, seed) <= 1.0
