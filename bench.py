@@ -309,14 +309,15 @@ def run_mq(args, ws_n, rank, local):
         "metric": METRIC, "value": round(ws_n * sb / (ms_per_step * 1e-3) / 1e9, 2),
         "unit": "GB/s", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u1-u4 planes, bf16 x, fp32 accumulate",
+        "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded; weights, codes and X per the layer recipe)",
         "config": config_dict(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "gemv_kernel (all 21 launches of the step)",
+                     "kernel": "mq_gemm M<=8 call: bfrag prep + gemv_mma_kernel, "
+                               "all 21 calls of the step",
                      "frac_of_8TBps": round(achieved / 8000.0, 4)},
         "e2e": {"value": round(ws_n * sb / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

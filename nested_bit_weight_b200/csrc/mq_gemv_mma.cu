@@ -1,364 +1,464 @@
-// Batch M <= 8: bit planes -> bf16 operand fragments in registers -> mma.sync.
+// Batch M <= 8: bit planes -> u8 operand fragments in registers -> int8 MMA.
 //
-// Why not CUDA-core FMAs: turning a weight into a float costs integer/logic
-// instructions, which B200 issues at half the fp32 rate, and the multiply-add
-// then costs one more instruction per weight and batch row.  Here a single
-// LOP3 builds two bf16 operands, and the warp-level MMA m16n8k16 (16 weight
-// rows x 8 batch rows x 16 columns) does every multiply-add; its n = 8 covers
-// M = 1..8 at the same cost.
+// Turning a weight into an operand costs integer/logic instructions, which
+// B200 issues at half the fp32 rate; a CUDA-core FMA then costs one more
+// instruction per weight and batch row.  Here one mask builds four u8
+// operands (one per byte), and the warp MMA m16n8k32 (16 weight rows x 8
+// columns x 32 inputs, u8 x s8 -> s32) does every multiply-add exactly.
 //
-// Operand construction.  Each lane owns one 32-column word of a 128-column
-// group for weight rows g and g + 8 (g = lane / 4, word t = lane % 4), reads
-// exactly r plane words per row (the r-bit model reads r bits per weight), and
-// rearranges them into "field words" whose fields hold the r-bit code q (or
-// 2q / a 4-bit part of it).  A field of width W at bit position p of a bf16
-// mantissa gives the exact bf16 value
-//          A = 1 + field * 2^(p - 7)          (bits 0x3F80 | field << p)
-// and the matching X operand is x * 2^(7 - p) (exact power-of-two scaling),
-// so A * B = x * 2^(7 - p) + x * field.  Per group g and batch row m:
-//     D = C0 + 2^e sum_k x q,   C0 = sum of the B operands of the group,
-//     sum_k x v_r = alpha (D - C0) + c_r S,  alpha = 2^(8 - r - e),
-//     c_r = 2^(7 - r) - 128,  S = sum_k x,
-// hence  y[n, m] += s[n, g] (alpha D - E[g, m]),  E = alpha C0 - c_r S.
-// A prep kernel writes the B fragments and E for the call; the main kernel
-// streams the planes, issues the MMAs and applies the group scales in fp32.
+// Weights: each lane owns one 32-column word of a 128-column group for rows g
+// and g + 8 (g = lane / 4, word t = lane % 4), reads exactly r plane words per
+// row, and builds eight u8x4 registers whose bytes are the r-bit codes q
+// (times 2^e, e = 1 for r = 3 and 8 - r for r >= 5) of known columns.
+//
+// X: per batch row m and group g, x = 2^(E-6) (a1 + 2^-7 a2 + 2^-14 a3) with
+// E = floor(log2 max|x|) and int8 slices a_j; bf16 x has 8 significant bits,
+// so the three slices are exact for every x within 2^-13 of the group's
+// largest (smaller ones keep an error below 2^(E-20)).  The slices are the MMA
+// columns c = 3m + j, so M <= 8 needs at most three 8-column tiles.
+//
+// Per group:  D_c = sum_k a_j(m, k) * field_k  (exact int32), and
+//   y[n, m] += s[n, g] * ( sum_j fac[g, c] D_c + c_r S[g, m] ),
+//   fac = 2^(8 - r - e + E - 6 - 7j),  c_r = 2^(7-r) - 128,  S = sum_k x.
+// A prep kernel writes the B fragments, fac and the c_r S terms; the main
+// kernel streams the planes, issues the MMAs and applies scales in fp32.
 #include "mq_common.cuh"
+#include "mq_bits.cuh"
 
 namespace mq {
 namespace {
 
-// ----------------------------------------------------------- operand tables
-// One register = two bf16 operands: field f of the low half and the field
-// at the same place in the high half of field word `fw` after a right shift.
-struct Entry { int fw, shift, p, f; };
-
-template <int R> struct Layout;   // field words, registers per row, fields
-
-// r = 1: the plane word itself, 1-bit fields, column k = f.
-template <> struct Layout<1> {
-    static constexpr int W = 1, NFW = 1, NREG = 16, E_EXP = 0;
-    __host__ __device__ static constexpr Entry entry(int i) {
-        return i < 7 ? Entry{0, 0, i, i} : i < 14 ? Entry{0, 7, i - 7, i} : Entry{0, 14, i - 14, i};
-    }
-    __host__ __device__ static constexpr int col(int fw, int f) { return f; }
-    __host__ __device__ static constexpr int part(int fw) { return 0; }
-};
-
-// r = 2: 2-bit fields q; word 0 holds even columns (k = 2f), word 1 odd.
-template <> struct Layout<2> {
-    static constexpr int W = 2, NFW = 2, NREG = 16, E_EXP = 0;
-    __host__ __device__ static constexpr Entry entry(int i) {
-        const int w = i / 8, j = i % 8;
-        return j < 3 ? Entry{w, 0, 2 * j, j} : j < 6 ? Entry{w, 6, 2 * (j - 3), j}
-                                                 : Entry{w, 12, 2 * (j - 6), j};
-    }
-    __host__ __device__ static constexpr int col(int fw, int f) { return 2 * f + fw; }
-    __host__ __device__ static constexpr int part(int fw) { return 0; }
-};
-
-// r = 3, 4: nibble fields (q, or 2q for r = 3); word d holds k = 4f + d.
-// r >= 5: words 0..3 hold the top nibble of q << (8 - r), words 4..7 the
-// bottom one (weighted 16 : 1 through the X operand).
-template <int R> struct Layout {
-    static constexpr int W = 4, NFW = R <= 4 ? 4 : 8, NREG = R <= 4 ? 16 : 32;
-    static constexpr int E_EXP = R == 3 ? 1 : R >= 5 ? 8 - R : 0;
-    __host__ __device__ static constexpr Entry entry(int i) {
-        return Entry{i / 4, 4 * (i % 4), 0, i % 4};
-    }
-    __host__ __device__ static constexpr int col(int fw, int f) { return 4 * f + (fw & 3); }
-    __host__ __device__ static constexpr int part(int fw) { return (R >= 5 && fw < 4) ? 1 : 0; }
-};
-
-template <int R> __host__ __device__ constexpr int fields_per_half() {
-    return 16 / Layout<R>::W;
+// ----------------------------------------------------------- operand layout
+// Register i (0..7) of a row word; byte b holds column col_of<R>(i, b).
+template <int R> __host__ __device__ constexpr int col_of(int i, int b) {
+    return R == 1 ? 8 * b + i                                   // bit i of byte b
+         : R == 2 ? 2 * (4 * b + (i & 3)) + (i >> 2)            // pair field 4b + j
+         : R <= 4 ? 4 * (2 * b + (i & 1)) + (i >> 1)            // nibble 2b + j of class d
+                  : 8 * b + i;                                   // byte word e = i
+}
+template <int R> __host__ __device__ constexpr int field_exp() {
+    return R == 3 ? 1 : R >= 5 ? 8 - R : 0;
 }
 
-// Field words from the r plane words of one 32-column word.
 template <int R>
-__device__ __forceinline__ void field_words(const uint32_t (&P)[8], uint32_t (&F)[8]) {
+__device__ __forceinline__ void operand_bytes(const uint32_t (&P)[8], uint32_t (&A)[8]) {
     if constexpr (R == 1) {
-        F[0] = P[0];
-    } else if constexpr (R == 2) {
-        F[0] = ((P[0] << 1) & 0xAAAAAAAAu) | (P[1] & 0x55555555u);
-        F[1] = (P[0] & 0xAAAAAAAAu) | ((P[1] >> 1) & 0x55555555u);
-    } else {
 #pragma unroll
-        for (int half = 0; half < (R <= 4 ? 1 : 2); ++half) {
-            const uint32_t p0 = P[4 * half], p1 = 4 * half + 1 < R ? P[4 * half + 1] : 0u;
-            const uint32_t p2 = 4 * half + 2 < R ? P[4 * half + 2] : 0u;
-            const uint32_t p3 = 4 * half + 3 < R ? P[4 * half + 3] : 0u;
-            const uint32_t x0 = ((p0 << 1) & 0xAAAAAAAAu) | (p1 & 0x55555555u);   // k even
-            const uint32_t x1 = (p0 & 0xAAAAAAAAu) | ((p1 >> 1) & 0x55555555u);   // k odd
-            const uint32_t y0 = ((p2 << 1) & 0xAAAAAAAAu) | (p3 & 0x55555555u);
-            const uint32_t y1 = (p2 & 0xAAAAAAAAu) | ((p3 >> 1) & 0x55555555u);
-            F[4 * half + 0] = ((x0 << 2) & 0xCCCCCCCCu) | (y0 & 0x33333333u);
-            F[4 * half + 1] = ((x1 << 2) & 0xCCCCCCCCu) | (y1 & 0x33333333u);
-            F[4 * half + 2] = (x0 & 0xCCCCCCCCu) | ((y0 >> 2) & 0x33333333u);
-            F[4 * half + 3] = (x1 & 0xCCCCCCCCu) | ((y1 >> 2) & 0x33333333u);
-        }
+        for (int i = 0; i < 8; ++i) A[i] = (P[0] >> i) & 0x01010101u;
+    } else if constexpr (R == 2) {
+        const uint32_t F[2] = {pair_even(P[0], P[1]), pair_odd(P[0], P[1])};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) A[i] = (F[i >> 2] >> (2 * (i & 3))) & 0x03030303u;
+    } else if constexpr (R <= 4) {
+        uint32_t N[4];
+        nibble_words<R>(P, 0, N);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) A[i] = (N[i >> 1] >> (4 * (i & 1))) & 0x0F0F0F0Fu;
+    } else {
+        byte_words<R>(P, A);
     }
 }
 
-// bf16 pair for register i: (field words >> shift) & mask | 1.0 (x2).
-template <int R>
-__device__ __forceinline__ uint32_t operand_reg(const uint32_t (&F)[8], int i) {
-    constexpr int W = Layout<R>::W;
-    const Entry e = Layout<R>::entry(i);
-    const uint32_t fmask = ((1u << W) - 1u) << e.p;
-    return ((F[e.fw] >> e.shift) & (fmask | (fmask << 16))) | 0x3F803F80u;
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
-                                               uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
 template <int R>
-__host__ __device__ constexpr float level_offset() { return (float)(1 << 7 >> (R - 1)) * 0.5f - 128.0f; }
+__host__ __device__ constexpr float level_offset() {   // c_r = 2^(7-r) - 128
+    return (float)(128 >> (R - 1)) * 0.5f - 128.0f;
+}
+
+constexpr int kCols = 24;                 // 8 batch rows x 3 slices
 
 // ------------------------------------------------------------ prep kernel
-// B fragments of every group (bf16 pairs, per lane in MMA order) and E[g, m].
+// One block (256 threads) per group.  Writes, for NT column tiles:
+//   bq[g][nt][h][lane][4]  u32 B fragments (h: MMA steps 2h, 2h+1; b0, b1 each)
+//   fac[g][24], off[g][24] floats (off = c_r S on slice-0 columns, else 0)
 template <int R>
 __global__ void __launch_bounds__(256)
-bfrag_kernel(const __nv_bfloat16 *__restrict__ X, int M, int64_t K,
-             uint32_t *__restrict__ bfrag, float *__restrict__ Eg) {
-    using L = Layout<R>;
-    constexpr int NREG = L::NREG, FPH = fields_per_half<R>();
-    const int64_t G = K / kGroup;
-    const int64_t total = G * 32 * NREG;                       // one uint32 per thread
-    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < total;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-        const int i = (int)(idx % NREG);                        // register (2s + half)
-        const int lane = (int)((idx / NREG) % 32);
-        const int64_t grp = idx / (NREG * 32);
-        const int m = lane >> 2, t = lane & 3;
-        const Entry e = L::entry(i);
-        float v[2] = {0.f, 0.f};
+xslice_kernel(const __nv_bfloat16 *__restrict__ X, int M, int64_t K, int NT,
+              uint32_t *__restrict__ bq, float *__restrict__ fac, float *__restrict__ off) {
+    __shared__ int8_t a[kCols][kGroup];       // slice j of batch row m at column k
+    __shared__ int e_grp[8];
+    __shared__ float s_grp[8];
+    const int64_t grp = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // warp m: exponent, sum and the three slices of batch row m
+    {
+        const int m = warp;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
         if (m < M) {
+            const uint2 raw = *reinterpret_cast<const uint2 *>(X + (int64_t)m * K + grp * kGroup + 4 * lane);
+            x[0] = __uint_as_float(raw.x << 16);
+            x[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+            x[2] = __uint_as_float(raw.y << 16);
+            x[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+        }
+        float amax = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+        float s = (x[0] + x[1]) + (x[2] + x[3]);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int f = e.f + h * FPH;
-                const int64_t k = grp * kGroup + 32 * t + L::col(e.fw, f);
-                const float sc = (float)(1 << (7 - e.p)) * (L::part(e.fw) ? 16.f : 1.f);
-                v[h] = __bfloat162float(X[(int64_t)m * K + k]) * sc;
-            }
+        for (int o = 16; o >= 1; o >>= 1) {
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            s += __shfl_xor_sync(0xffffffffu, s, o);
         }
-        __nv_bfloat162 b = __floats2bfloat162_rn(v[0], v[1]);   // exact: power-of-two scale
-        bfrag[idx] = *reinterpret_cast<uint32_t *>(&b);
+        // E = floor(log2 amax) from the exponent field (amax is a bf16 value)
+        const int E = amax > 0.f ? (int)((__float_as_uint(amax) >> 23) & 0xFF) - 127 : 0;
+        if (lane == 0) { e_grp[m] = E; s_grp[m] = s; }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            // exact splitting: every step subtracts a representable multiple
+            const float v1 = ldexpf(x[u], 6 - E);                    // |v1| < 128
+            const float a1 = truncf(v1);
+            const float v2 = (v1 - a1) * 128.f;
+            const float a2 = truncf(v2);
+            const float a3 = truncf((v2 - a2) * 128.f);
+            a[3 * m + 0][4 * lane + u] = (int8_t)a1;
+            a[3 * m + 1][4 * lane + u] = (int8_t)a2;
+            a[3 * m + 2][4 * lane + u] = (int8_t)a3;
+        }
     }
-    // E[g, m] = alpha * C0 - c_r * S, with C0 the sum of the group's B operands
-    constexpr float alpha = (float)(1 << (8 - R - L::E_EXP));
-    for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < G * 8;
-         idx += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t grp = idx / 8;
-        const int m = (int)(idx % 8);
-        float c0 = 0.f, s = 0.f;
-        if (m < M) {
-            for (int t = 0; t < 4; ++t)
-                for (int i = 0; i < NREG; ++i) {
-                    const Entry e = L::entry(i);
-                    for (int h = 0; h < 2; ++h) {
-                        const int f = e.f + h * FPH;
-                        const float x = __bfloat162float(
-                            X[(int64_t)m * K + grp * kGroup + 32 * t + L::col(e.fw, f)]);
-                        c0 += x * (float)(1 << (7 - e.p)) * (L::part(e.fw) ? 16.f : 1.f);
-                        s += x;
-                    }
-                }
+    __syncthreads();
+    // B fragments: lane L = (column-in-tile cg, word t); step st uses the
+    // bytes of registers 2 st (b0) and 2 st + 1 (b1)
+    for (int idx = threadIdx.x; idx < NT * 2 * 32 * 4; idx += blockDim.x) {
+        const int w = idx & 3, L = (idx >> 2) & 31, h = (idx >> 7) & 1, nt = idx >> 8;
+        const int cg = L >> 2, t = L & 3;
+        const int c = 8 * nt + cg;
+        const int st = 2 * h + (w >> 1), reg = 2 * st + (w & 1);
+        uint32_t v = 0;
+        if (c < 3 * M) {
+#pragma unroll
+            for (int b = 0; b < 4; ++b)
+                v |= (uint32_t)(uint8_t)a[c][32 * t + col_of<R>(reg, b)] << (8 * b);
         }
-        Eg[idx] = alpha * c0 - level_offset<R>() * s;
+        bq[((grp * NT + nt) * 2 + h) * 128 + L * 4 + w] = v;
+    }
+    if (threadIdx.x < kCols) {
+        const int c = threadIdx.x, m = c / 3, j = c % 3;
+        float f = 0.f, o = 0.f;
+        if (m < M) {
+            f = ldexpf(1.f, 8 - R - field_exp<R>() + e_grp[m] - 6 - 7 * j);
+            o = j == 0 ? level_offset<R>() * s_grp[m] : 0.f;
+        }
+        fac[grp * kCols + c] = f;
+        off[grp * kCols + c] = o;
     }
 }
 
 // ------------------------------------------------------------- main kernel
-constexpr int kMmaWarps = 4;
-constexpr int kBatch = 2;               // groups loaded per pipeline stage
+// Persistent CTAs per K slice (blockIdx.y).  The CTA stages the slice's B
+// fragments, fac and off once; each warp owns 16-row tiles and pulls a tile's
+// plane bytes (16 rows x r planes x the slice's groups) into shared memory
+// with bulk async copies issued by one lane, one tile ahead (two stages per
+// warp), so a whole tile of HBM reads is in flight while it computes the last.
+constexpr int kMmaWarps = 8;
 
-__device__ __forceinline__ uint32_t ld_plane(const uint32_t *p) {
-    uint32_t v;
-    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
-    return v;
+template <int R> __host__ __device__ constexpr int slice_groups() { return R >= 6 ? 2 : 16 / R; }
+
+// Row stride (words) of a staged tile: 4 (mod 8), so the 8 rows x 4 words a
+// warp reads at once fall in 32 distinct banks.
+__host__ __device__ constexpr int stage_row_words(int r, int gpt) {
+    return ((r * gpt * 4) % 8 == 0) ? r * gpt * 4 + 4 : r * gpt * 4;
 }
 
-// One warp: 16 weight rows x a range of groups.  Warp task w -> (tile, split).
-template <int R>
+template <int R, int NT> struct MmaSmem {
+    static constexpr int GPT = slice_groups<R>();
+    static constexpr int RS = stage_row_words(R, GPT);
+    static constexpr size_t bq = 0;
+    static constexpr size_t fac = bq + (size_t)GPT * NT * 1024;
+    static constexpr size_t off = fac + (size_t)GPT * kCols * 4;
+    static constexpr size_t red = off + (size_t)GPT * kCols * 4;
+    static constexpr size_t stages = red + (size_t)kMmaWarps * 16 * kCols * 4;
+    static constexpr size_t stage_bytes = (size_t)16 * RS * 4;
+    static constexpr size_t bars = stages + (size_t)kMmaWarps * 2 * stage_bytes;
+    static constexpr size_t total = bars + (1 + 2 * kMmaWarps) * 8;
+};
+
+__device__ unsigned int g_gemv_timeout;
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void bar_init(uint64_t *b, uint32_t n) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(b)), "r"(n));
+}
+__device__ __forceinline__ void bar_expect(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_addr(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *b) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(b)) : "memory");
+}
+// Bounded wait on an mbarrier phase (the hint lets the thread sleep).
+__device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) {
+    for (uint32_t i = 0; i < (1u << 22); ++i) {
+        uint32_t ok;
+        asm volatile("{\n .reg .pred p;\n"
+                     " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 1000000;\n"
+                     " selp.u32 %0, 1, 0, p;\n}"
+                     : "=r"(ok) : "r"(smem_addr(b)), "r"(parity) : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+template <int R, int NT>
 __global__ void __launch_bounds__(kMmaWarps * 32)
-gemv_mma_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ scales,
-                const uint32_t *__restrict__ bfrag, const float *__restrict__ Eg,
-                int M, int64_t N, int64_t K, int64_t tiles, int KS, int gpt,
-                float *__restrict__ part, unsigned *__restrict__ tickets,
-                __nv_bfloat16 *__restrict__ Y) {
-    using L = Layout<R>;
-    constexpr int NREG = L::NREG, STEPS = NREG / 2;
-    constexpr float alpha = (float)(1 << (8 - R - L::E_EXP));
-    const int lane = threadIdx.x & 31;
-    const int64_t task = (int64_t)blockIdx.x * kMmaWarps + (threadIdx.x >> 5);
-    if (task >= tiles * KS) return;
-    const int64_t tile = task / KS;
-    const int ks = (int)(task % KS);
+gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ scales,
+               const uint32_t *__restrict__ bq, const float *__restrict__ facg,
+               const float *__restrict__ offg, int M, int64_t N, int64_t K, int64_t tiles,
+               float *__restrict__ part, unsigned *__restrict__ tickets,
+               __nv_bfloat16 *__restrict__ Y) {
+    using S = MmaSmem<R, NT>;
+    constexpr int GPT = S::GPT, RS = S::RS, JS = (GPT + 3) / 4;
+    constexpr int kStageWords = (int)(S::stage_bytes / 4);
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint4 *sB = reinterpret_cast<const uint4 *>(smem + S::bq);
+    const float *sF = reinterpret_cast<const float *>(smem + S::fac);
+    const float *sO = reinterpret_cast<const float *>(smem + S::off);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + S::bars);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
+    float *red = reinterpret_cast<float *>(smem + S::red) + warp * 16 * kCols;
+    const int KS = gridDim.y, ks = blockIdx.y;
     const int64_t G = K / kGroup;
-    const int64_t g0 = (int64_t)ks * gpt;
-    const int64_t g1 = g0 + gpt < G ? g0 + gpt : G;
-    const int64_t n_lo = tile * 16 + g, n_hi = n_lo + 8;
-    const bool ok_lo = n_lo < N, ok_hi = n_hi < N;
+    const int64_t g0 = (int64_t)ks * GPT;
+    const int ng = (int)((g0 + GPT < G ? g0 + GPT : G) - g0);
     const int64_t plane_words = N * (K / 32);
-    const uint32_t *row_lo = planes + (ok_lo ? n_lo : 0) * (K / 32) + t;
-    const uint32_t *row_hi = planes + (ok_hi ? n_hi : 0) * (K / 32) + t;
-    const bool bvalid = g < M;
+    uint32_t *const stage0 = reinterpret_cast<uint32_t *>(smem + S::stages + 2 * warp * S::stage_bytes);
+    uint64_t *wbar = bars + 1 + 2 * warp;
 
-    float y[4] = {0.f, 0.f, 0.f, 0.f};
-    uint32_t w[2][kBatch][2][R];          // [buffer][group][row][plane]
-    float sc[2][kBatch][2];
+    if (threadIdx.x == 0) {
+        bar_init(&bars[0], 1);
+        for (int i = 0; i < 2 * kMmaWarps; ++i) bar_init(&bars[1 + i], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t bb = (uint32_t)ng * NT * 1024, fb = (uint32_t)ng * kCols * 4;
+        bar_expect(&bars[0], bb + 2 * fb);
+        bulk_g2s(smem + S::bq, bq + g0 * NT * 256, bb, &bars[0]);
+        bulk_g2s(smem + S::fac, facg + g0 * kCols, fb, &bars[0]);
+        bulk_g2s(smem + S::off, offg + g0 * kCols, fb, &bars[0]);
+    }
 
-    auto load = [&](int buf, int64_t gb) {
+    const int64_t stride = (int64_t)gridDim.x * kMmaWarps;
+    int64_t tile = (int64_t)blockIdx.x * kMmaWarps + warp;
+
+    // One tile's plane rows into stage `st` (lane 0); each lane prefetches the
+    // scales of groups 4j + t for its rows g and g + 8.
+    float nsc[2][JS];
+    auto issue = [&](int st, int64_t tl) {
+        if (lane == 0) {
+            int rows = 0;
+            for (int rr = 0; rr < 16; ++rr) rows += (tl * 16 + rr < N);
+            bar_expect(wbar + st, (uint32_t)(rows * R * ng * 16));
+            for (int rr = 0; rr < rows; ++rr) {
+                const int64_t n = tl * 16 + rr;
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int64_t gg = gb + j;
-            const bool in = gg < g1;
-#pragma unroll
-            for (int p = 0; p < R; ++p) {
-                w[buf][j][0][p] = (in && ok_lo) ? ld_plane(row_lo + p * plane_words + gg * 4) : 0u;
-                w[buf][j][1][p] = (in && ok_hi) ? ld_plane(row_hi + p * plane_words + gg * 4) : 0u;
+                for (int p = 0; p < R; ++p)
+                    bulk_g2s(stage0 + st * kStageWords + rr * RS + p * GPT * 4,
+                             planes + p * plane_words + n * (K / 32) + g0 * 4,
+                             (uint32_t)ng * 16, wbar + st);
             }
-            sc[buf][j][0] = (in && ok_lo) ? __half2float(scales[n_lo * G + gg]) : 0.f;
-            sc[buf][j][1] = (in && ok_hi) ? __half2float(scales[n_hi * G + gg]) : 0.f;
+        }
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+            const int64_t n = tl * 16 + g + 8 * hr;
+#pragma unroll
+            for (int j = 0; j < JS; ++j) {
+                const int grp = 4 * j + t;
+                nsc[hr][j] = (n < N && grp < ng) ? __half2float(scales[n * G + g0 + grp]) : 0.f;
+            }
         }
     };
 
-    auto compute = [&](int buf, int64_t gb) {
+    uint32_t phase_bits = 0u;
+    bool ok = true;
+    if (tile < tiles) issue(0, tile);
+    if (!bar_wait(&bars[0], 0)) ok = false;
+    int st = 0;
+    float csc[2][JS];
+    for (; tile < tiles && ok; tile += stride) {
 #pragma unroll
-        for (int j = 0; j < kBatch; ++j) {
-            const int64_t gg = gb + j;
-            if (gg >= g1) break;
-            uint32_t F[2][8], P[8];
+        for (int hr = 0; hr < 2; ++hr)
 #pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
+            for (int j = 0; j < JS; ++j) csc[hr][j] = nsc[hr][j];
+        const int64_t next = tile + stride;
+        __syncwarp();
+        if (next < tiles) issue(st ^ 1, next);
+        if (!bar_wait(wbar + st, (phase_bits >> st) & 1u)) { ok = false; break; }
+        phase_bits ^= 1u << st;
+        const uint32_t *sw = stage0 + st * kStageWords;
+
+        float y[NT][4];
 #pragma unroll
-                for (int p = 0; p < 8; ++p) P[p] = p < R ? w[buf][j][rr][p] : 0u;
-                field_words<R>(P, F[rr]);
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) y[nt][i] = 0.f;
+#pragma unroll
+        for (int grp = 0; grp < GPT; ++grp) {
+            if (grp >= ng) break;
+            uint32_t A[2][8], P[8];
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+#pragma unroll
+                for (int p = 0; p < 8; ++p)
+                    P[p] = p < R ? sw[(g + 8 * hr) * RS + p * GPT * 4 + grp * 4 + t] : 0u;
+                operand_bytes<R>(P, A[hr]);
             }
-            const uint4 *bp = reinterpret_cast<const uint4 *>(bfrag + (gg * 32 + lane) * NREG);
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            const float s_lo = __shfl_sync(0xffffffffu, csc[0][grp / 4], g * 4 + (grp & 3));
+            const float s_hi = __shfl_sync(0xffffffffu, csc[1][grp / 4], g * 4 + (grp & 3));
 #pragma unroll
-            for (int q4 = 0; q4 < NREG / 4; ++q4) {
-                const uint4 b = bvalid ? __ldg(bp + q4) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int hs = 0; hs < 2; ++hs) {         // two MMA steps per uint4
-                    const int s = 2 * q4 + hs;
-                    uint32_t a[4];
-                    a[0] = operand_reg<R>(F[0], 2 * s);
-                    a[1] = operand_reg<R>(F[1], 2 * s);
-                    a[2] = operand_reg<R>(F[0], 2 * s + 1);
-                    a[3] = operand_reg<R>(F[1], 2 * s + 1);
-                    mma_bf16_16816(d, a, hs ? b.z : b.x, hs ? b.w : b.y);
-                }
+            for (int nt = 0; nt < NT; ++nt) {
+                int da[4] = {0, 0, 0, 0}, db[4] = {0, 0, 0, 0};
+                const uint4 b0 = sB[((grp * NT + nt) * 2 + 0) * 32 + lane];
+                const uint4 b1 = sB[((grp * NT + nt) * 2 + 1) * 32 + lane];
+                uint32_t a[4];
+                a[0] = A[0][0]; a[1] = A[1][0]; a[2] = A[0][1]; a[3] = A[1][1];
+                mma_u8s8(da, a, b0.x, b0.y);
+                a[0] = A[0][2]; a[1] = A[1][2]; a[2] = A[0][3]; a[3] = A[1][3];
+                mma_u8s8(db, a, b0.z, b0.w);
+                a[0] = A[0][4]; a[1] = A[1][4]; a[2] = A[0][5]; a[3] = A[1][5];
+                mma_u8s8(da, a, b1.x, b1.y);
+                a[0] = A[0][6]; a[1] = A[1][6]; a[2] = A[0][7]; a[3] = A[1][7];
+                mma_u8s8(db, a, b1.z, b1.w);
+                const float2 f = *reinterpret_cast<const float2 *>(sF + grp * kCols + 8 * nt + 2 * t);
+                const float2 o = *reinterpret_cast<const float2 *>(sO + grp * kCols + 8 * nt + 2 * t);
+                y[nt][0] = fmaf(s_lo, fmaf(f.x, (float)(da[0] + db[0]), o.x), y[nt][0]);
+                y[nt][1] = fmaf(s_lo, fmaf(f.y, (float)(da[1] + db[1]), o.y), y[nt][1]);
+                y[nt][2] = fmaf(s_hi, fmaf(f.x, (float)(da[2] + db[2]), o.x), y[nt][2]);
+                y[nt][3] = fmaf(s_hi, fmaf(f.y, (float)(da[3] + db[3]), o.y), y[nt][3]);
             }
-            const float2 e = *reinterpret_cast<const float2 *>(Eg + gg * 8 + 2 * t);
-            y[0] = fmaf(sc[buf][j][0], fmaf(alpha, d[0], -e.x), y[0]);
-            y[1] = fmaf(sc[buf][j][0], fmaf(alpha, d[1], -e.y), y[1]);
-            y[2] = fmaf(sc[buf][j][1], fmaf(alpha, d[2], -e.x), y[2]);
-            y[3] = fmaf(sc[buf][j][1], fmaf(alpha, d[3], -e.y), y[3]);
         }
-    };
+        st ^= 1;
 
-    // two register buffers, static indices: load one stage ahead
-    load(0, g0);
-    for (int64_t gb = g0; gb < g1; gb += 2 * kBatch) {
-        if (gb + kBatch < g1) load(1, gb + kBatch);
-        compute(0, gb);
-        if (gb + kBatch >= g1) break;
-        if (gb + 2 * kBatch < g1) load(0, gb + 2 * kBatch);
-        compute(1, gb + kBatch);
+        // ---- columns -> batch rows: Y[m, n] = sum_j column 3m + j
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int c = 8 * nt + 2 * t;
+            red[g * kCols + c] = y[nt][0];
+            red[g * kCols + c + 1] = y[nt][1];
+            red[(g + 8) * kCols + c] = y[nt][2];
+            red[(g + 8) * kCols + c + 1] = y[nt][3];
+        }
+        __syncwarp();
+        float out[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {                      // 16 M <= 128 outputs
+            const int idx = lane + 32 * q, rr = idx & 15, m = idx >> 4;
+            out[q] = idx < 16 * M ? red[rr * kCols + 3 * m] + red[rr * kCols + 3 * m + 1] +
+                                        red[rr * kCols + 3 * m + 2]
+                                  : 0.f;
+        }
+        __syncwarp();
+        if (KS == 1) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int idx = lane + 32 * q, rr = idx & 15, m = idx >> 4;
+                const int64_t n = tile * 16 + rr;
+                if (idx < 16 * M && n < N) Y[(int64_t)m * N + n] = __float2bfloat16_rn(out[q]);
+            }
+            continue;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int idx = lane + 32 * q, rr = idx & 15, m = idx >> 4;
+            const int64_t n = tile * 16 + rr;
+            if (idx < 16 * M && n < N) part[((int64_t)ks * M + m) * N + n] = out[q];
+        }
+        __threadfence();
+        __syncwarp();
+        unsigned last = 0;
+        if (lane == 0) last = atomicAdd(&tickets[tile], 1u) == (unsigned)KS - 1;
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) continue;
+        __threadfence();
+        for (int idx = lane; idx < 16 * M; idx += 32) {      // fixed-order sum
+            const int rr = idx & 15, m = idx >> 4;
+            const int64_t n = tile * 16 + rr;
+            if (n >= N) continue;
+            float acc = 0.f;
+            for (int z = 0; z < KS; ++z) acc += __ldcg(part + ((int64_t)z * M + m) * N + n);
+            Y[(int64_t)m * N + n] = __float2bfloat16_rn(acc);
+        }
+        if (lane == 0) tickets[tile] = 0u;
     }
-    (void)STEPS;
-
-    // ---- outputs: lane holds rows (n_lo, n_hi) x batch rows (2t, 2t+1)
-    const int m0 = 2 * t;
-    if (KS == 1) {
-        if (ok_lo && m0 < M) Y[(int64_t)m0 * N + n_lo] = __float2bfloat16_rn(y[0]);
-        if (ok_lo && m0 + 1 < M) Y[(int64_t)(m0 + 1) * N + n_lo] = __float2bfloat16_rn(y[1]);
-        if (ok_hi && m0 < M) Y[(int64_t)m0 * N + n_hi] = __float2bfloat16_rn(y[2]);
-        if (ok_hi && m0 + 1 < M) Y[(int64_t)(m0 + 1) * N + n_hi] = __float2bfloat16_rn(y[3]);
-        return;
-    }
-    float *pk = part + (int64_t)ks * M * N;
-    if (ok_lo && m0 < M) pk[(int64_t)m0 * N + n_lo] = y[0];
-    if (ok_lo && m0 + 1 < M) pk[(int64_t)(m0 + 1) * N + n_lo] = y[1];
-    if (ok_hi && m0 < M) pk[(int64_t)m0 * N + n_hi] = y[2];
-    if (ok_hi && m0 + 1 < M) pk[(int64_t)(m0 + 1) * N + n_hi] = y[3];
-    __threadfence();
-    __syncwarp();
-    unsigned last = 0;
-    if (lane == 0) last = atomicAdd(&tickets[tile], 1u) == (unsigned)KS - 1;
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (!last) return;
-    __threadfence();
-    // the last warp of this tile sums the KS partials in fixed order
-    for (int idx = lane; idx < 16 * M; idx += 32) {
-        const int m = idx / 16;
-        const int64_t n = tile * 16 + idx % 16;
-        if (n >= N) continue;
-        float a = 0.f;
-        for (int z = 0; z < KS; ++z) a += __ldcg(part + ((int64_t)z * M + m) * N + n);
-        Y[(int64_t)m * N + n] = __float2bfloat16_rn(a);
-    }
-    if (lane == 0) tickets[tile] = 0u;
+    if (!ok && lane == 0) atomicOr(&g_gemv_timeout, 1u);
 }
 
 struct MmaPlan {
-    int KS, gpt;
-    int64_t tiles, tasks;
-    size_t part_off, bfrag_off, e_off, ws_bytes;
+    int KS, NT;
+    int64_t tiles, ctas_x;
+    size_t part_off, bq_off, fac_off, off_off, ws_bytes;
 };
+
+int plan_gpt(int r) { return r >= 6 ? 2 : 16 / r; }
 
 MmaPlan mma_plan(int64_t M, int64_t N, int64_t K, int r) {
     MmaPlan p{};
     const int64_t G = K / kGroup;
+    const int gpt = plan_gpt(r);
+    p.NT = (int)((3 * M + 7) / 8);
     p.tiles = (N + 15) / 16;
-    const int64_t want = 148 * 16;                   // warp tasks to fill the GPU
-    int64_t ks = (want + p.tiles - 1) / p.tiles;
-    int64_t cap = G / 4 > 1 ? G / 4 : 1;
-    if (ks > cap) ks = cap;
-    if (ks < 1) ks = 1;
-    p.gpt = (int)((G + ks - 1) / ks);
-    p.KS = (int)((G + p.gpt - 1) / p.gpt);
-    p.tasks = p.tiles * p.KS;
-    const int nreg = r <= 4 ? 16 : 32;
+    p.KS = (int)((G + gpt - 1) / gpt);
+    int64_t cap = (2 * 148) / p.KS;
+    if (cap < 1) cap = 1;
+    p.ctas_x = (p.tiles + kMmaWarps - 1) / kMmaWarps;
+    if (p.ctas_x > cap) p.ctas_x = cap;
     p.part_off = kTicketBytes;
     size_t off = p.part_off + (p.KS > 1 ? (size_t)p.KS * M * N * sizeof(float) : 0);
-    p.bfrag_off = (off + 255) & ~(size_t)255;
-    off = p.bfrag_off + (size_t)G * 32 * nreg * sizeof(uint32_t);
-    p.e_off = (off + 255) & ~(size_t)255;
-    p.ws_bytes = p.e_off + (size_t)G * 8 * sizeof(float);
+    p.bq_off = (off + 255) & ~(size_t)255;
+    off = p.bq_off + (size_t)G * p.NT * 1024;
+    p.fac_off = (off + 255) & ~(size_t)255;
+    off = p.fac_off + (size_t)G * kCols * sizeof(float);
+    p.off_off = (off + 255) & ~(size_t)255;
+    p.ws_bytes = p.off_off + (size_t)G * kCols * sizeof(float);
     return p;
 }
 
-template <int R>
-mq_status run_mma(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y, char *ws,
-                  const MmaPlan &p, cudaStream_t st) {
-    uint32_t *bfrag = reinterpret_cast<uint32_t *>(ws + p.bfrag_off);
-    float *Eg = reinterpret_cast<float *>(ws + p.e_off);
+template <int R, int NT>
+mq_status run_i8(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y, char *ws,
+                 const MmaPlan &p, cudaStream_t st) {
+    uint32_t *bq = reinterpret_cast<uint32_t *>(ws + p.bq_off);
+    float *fac = reinterpret_cast<float *>(ws + p.fac_off);
+    float *off = reinterpret_cast<float *>(ws + p.off_off);
     const int64_t G = w->K / kGroup;
-    const int64_t work = G * 32 * Layout<R>::NREG;
-    int grid = (int)((work + 255) / 256);
-    if (grid > 148 * 8) grid = 148 * 8;
-    bfrag_kernel<R><<<grid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X), (int)M,
-                                          w->K, bfrag, Eg);
+    xslice_kernel<R><<<(unsigned)G, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16 *>(X),
+                                                  (int)M, w->K, NT, bq, fac, off);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "bfrag_kernel");
-    const unsigned blocks = (unsigned)((p.tasks + kMmaWarps - 1) / kMmaWarps);
-    gemv_mma_kernel<R><<<blocks, kMmaWarps * 32, 0, st>>>(
-        w->planes, reinterpret_cast<const __half *>(w->scales), bfrag, Eg, (int)M, w->N, w->K,
-        p.tiles, p.KS, p.gpt, reinterpret_cast<float *>(ws + p.part_off),
-        reinterpret_cast<unsigned *>(ws), reinterpret_cast<__nv_bfloat16 *>(Y));
+    if (e != cudaSuccess) return cuda_fail(e, "xslice_kernel");
+    constexpr size_t smem = MmaSmem<R, NT>::total;
+    static bool attr_set = false;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(gemv_i8_kernel<R, NT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        attr_set = true;
+    }
+    dim3 grid((unsigned)p.ctas_x, (unsigned)p.KS);
+    gemv_i8_kernel<R, NT><<<grid, kMmaWarps * 32, smem, st>>>(
+        w->planes, reinterpret_cast<const __half *>(w->scales), bq, fac, off, (int)M, w->N, w->K,
+        p.tiles, reinterpret_cast<float *>(ws + p.part_off), reinterpret_cast<unsigned *>(ws),
+        reinterpret_cast<__nv_bfloat16 *>(Y));
     e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "gemv_mma_kernel");
+    if (e != cudaSuccess) return cuda_fail(e, "gemv_i8_kernel");
     return MQ_OK;
+}
+
+template <int R>
+mq_status run_r(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y, char *ws,
+                const MmaPlan &p, cudaStream_t st) {
+    if (p.NT == 1) return run_i8<R, 1>(X, w, M, Y, ws, p, st);
+    if (p.NT == 2) return run_i8<R, 2>(X, w, M, Y, ws, p, st);
+    return run_i8<R, 3>(X, w, M, Y, ws, p, st);
 }
 
 }  // namespace
@@ -373,16 +473,17 @@ mq_status launch_gemv_mma(const uint16_t *X, const mq_weights *w, int64_t M, uin
     if (p.ws_bytes > ws_bytes) return fail(MQ_ERR_WORKSPACE, "GEMV workspace too small");
     if (p.KS > 1 && p.tiles > (int64_t)(kTicketBytes / sizeof(unsigned)))
         return fail(MQ_ERR_UNSUPPORTED, "too many row tiles for the split-K ticket region");
+    if (p.KS > 65535) return fail(MQ_ERR_UNSUPPORTED, "K too large");
     char *b = static_cast<char *>(ws);
     switch (w->r) {
-        case 1: return run_mma<1>(X, w, M, Y, b, p, st);
-        case 2: return run_mma<2>(X, w, M, Y, b, p, st);
-        case 3: return run_mma<3>(X, w, M, Y, b, p, st);
-        case 4: return run_mma<4>(X, w, M, Y, b, p, st);
-        case 5: return run_mma<5>(X, w, M, Y, b, p, st);
-        case 6: return run_mma<6>(X, w, M, Y, b, p, st);
-        case 7: return run_mma<7>(X, w, M, Y, b, p, st);
-        default: return run_mma<8>(X, w, M, Y, b, p, st);
+        case 1: return run_r<1>(X, w, M, Y, b, p, st);
+        case 2: return run_r<2>(X, w, M, Y, b, p, st);
+        case 3: return run_r<3>(X, w, M, Y, b, p, st);
+        case 4: return run_r<4>(X, w, M, Y, b, p, st);
+        case 5: return run_r<5>(X, w, M, Y, b, p, st);
+        case 6: return run_r<6>(X, w, M, Y, b, p, st);
+        case 7: return run_r<7>(X, w, M, Y, b, p, st);
+        default: return run_r<8>(X, w, M, Y, b, p, st);
     }
 }
 

@@ -1,9 +1,8 @@
 // Bit-plane packer and its inverse (exact-r-bit storage of the MatGPTQ
 // abstract and Table 1, "Exact r-bit loading").
 //
-// pack: one warp turns 32 consecutive codes of a row into one word of each of
-// the 8 planes with warp ballots (lane j votes bit j), so every store is a
-// full word and every plane row is written contiguously.
+// pack: a warp turns 32 consecutive codes of a row into one word of each of
+// the 8 planes with warp ballots (lane j votes bit j of its code).
 #include "mq_common.cuh"
 
 namespace mq {
@@ -13,22 +12,31 @@ __device__ unsigned int g_pack_bad;   // set when a scale is not storable
 __global__ void __launch_bounds__(256)
 pack_kernel(const uint8_t *__restrict__ codes, int64_t N, int64_t K,
             uint32_t *__restrict__ planes) {
+    // one warp per (row, block of 32 words): chunk c's ballots land in lane c,
+    // so each plane's 32 words leave as one coalesced 128-byte store
     const int lane = threadIdx.x & 31;
     const int64_t W = K / 32;                        // words per plane row
-    const int64_t total = N * W;                     // (row, word) pairs
+    const int64_t blocks_per_row = (W + 31) / 32;
+    const int64_t total = N * blocks_per_row;
     const int64_t plane_words = N * W;
     int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t i = warp; i < total; i += nwarps) {
-        const int64_t n = i / W, w = i - n * W;
-        const unsigned c = codes[n * K + 32 * w + lane];
-        uint32_t mine = 0;
+        const int64_t n = i / blocks_per_row, w0 = (i % blocks_per_row) * 32;
+        uint32_t mine[kPlanes] = {0, 0, 0, 0, 0, 0, 0, 0};
+        for (int c = 0; c < 32 && w0 + c < W; ++c) {
+            const unsigned q = codes[n * K + 32 * (w0 + c) + lane];
 #pragma unroll
-        for (int p = 0; p < kPlanes; ++p) {
-            const uint32_t word = __ballot_sync(0xffffffffu, (c >> (7 - p)) & 1u);
-            if (lane == p) mine = word;
+            for (int p = 0; p < kPlanes; ++p) {
+                const uint32_t word = __ballot_sync(0xffffffffu, (q >> (7 - p)) & 1u);
+                if (lane == c) mine[p] = word;
+            }
         }
-        if (lane < kPlanes) planes[(int64_t)lane * plane_words + i] = mine;
+        if (w0 + lane < W) {
+#pragma unroll
+            for (int p = 0; p < kPlanes; ++p)
+                planes[(int64_t)p * plane_words + n * W + w0 + lane] = mine[p];
+        }
     }
 }
 
@@ -100,8 +108,7 @@ extern "C" mq_status mq_pack(const uint8_t *codes, const float *scales, int64_t 
     cudaError_t e = cudaMemcpyToSymbolAsync(g_pack_bad, &zero, sizeof(zero), 0,
                                             cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "mq_pack reset");
-    const int64_t words = N * (K / 32);
-    pack_kernel<<<grid_for(words * 32, 256), 256, 0, st>>>(codes, N, K, planes_out);
+    pack_kernel<<<grid_for(N * ((K / 32 + 31) / 32) * 32, 256), 256, 0, st>>>(codes, N, K, planes_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pack_kernel");
     const int64_t ns = N * (K / kGroup);
     scales_kernel<<<grid_for(ns, 256), 256, 0, st>>>(scales, ns,
