@@ -22,6 +22,10 @@
 //   fac = 2^(8 - r - e + E - 6 - 7j),  c_r = 2^(7-r) - 128,  S = sum_k x.
 // A prep kernel writes the B fragments, fac and the c_r S terms; the main
 // kernel streams the planes, issues the MMAs and applies scales in fp32.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <string.h>
+
 #include "mq_common.cuh"
 #include "mq_bits.cuh"
 
@@ -86,6 +90,8 @@ xslice_kernel(const __nv_bfloat16 *__restrict__ X, int M, int64_t K, int NT,
     __shared__ int8_t a[kCols][kGroup];       // slice j of batch row m at column k
     __shared__ int e_grp[8];
     __shared__ float s_grp[8];
+    // the GEMV kernel may start now: it streams weights until it needs our output
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int64_t grp = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // warp m: exponent, sum and the three slices of batch row m
@@ -158,25 +164,23 @@ xslice_kernel(const __nv_bfloat16 *__restrict__ X, int M, int64_t K, int NT,
 // warp), so a whole tile of HBM reads is in flight while it computes the last.
 constexpr int kMmaWarps = 8;
 
-template <int R> __host__ __device__ constexpr int slice_groups() { return R >= 6 ? 2 : 16 / R; }
+// Groups per K slice: a tile row of one plane is 16 GPT bytes = one TMA
+// swizzle span (128, 64 or 32 bytes).
+template <int R> __host__ __device__ constexpr int slice_groups() { return R <= 2 ? 8 : R <= 4 ? 4 : 2; }
 
-// Row stride (words) of a staged tile: 4 (mod 8), so the 8 rows x 4 words a
-// warp reads at once fall in 32 distinct banks.
-__host__ __device__ constexpr int stage_row_words(int r, int gpt) {
-    return ((r * gpt * 4) % 8 == 0) ? r * gpt * 4 + 4 : r * gpt * 4;
-}
 
 template <int R, int NT> struct MmaSmem {
     static constexpr int GPT = slice_groups<R>();
-    static constexpr int RS = stage_row_words(R, GPT);
-    static constexpr size_t bq = 0;
+    static constexpr int ROWB = 16 * GPT;                 // bytes of one plane row of a tile
+    static constexpr size_t stage_bytes = (size_t)R * 16 * ROWB;   // the TMA box
+    static constexpr size_t stages = 0;                   // 1024-aligned (swizzle period)
+    static constexpr size_t bq = stages + (size_t)kMmaWarps * 2 * ((stage_bytes + 256 + 1023) & ~(size_t)1023);
     static constexpr size_t fac = bq + (size_t)GPT * NT * 1024;
     static constexpr size_t off = fac + (size_t)GPT * kCols * 4;
     static constexpr size_t red = off + (size_t)GPT * kCols * 4;
-    static constexpr size_t stages = red + (size_t)kMmaWarps * 16 * kCols * 4;
-    static constexpr size_t stage_bytes = (size_t)16 * RS * 4;
-    static constexpr size_t bars = stages + (size_t)kMmaWarps * 2 * stage_bytes;
-    static constexpr size_t total = bars + (1 + 2 * kMmaWarps) * 8;
+    static constexpr size_t bars = red + (size_t)kMmaWarps * 16 * kCols * 4;
+    static constexpr size_t stage_pitch = (stage_bytes + 256 + 1023) & ~(size_t)1023;
+    static constexpr size_t total = bars + (1 + 2 * kMmaWarps) * 8 + 1024;   // + base alignment
 };
 
 __device__ unsigned int g_gemv_timeout;
@@ -196,6 +200,30 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(b)) : "memory");
 }
+// One 3-D TMA box (words x rows x planes) of the plane tensor into shared memory.
+__device__ __forceinline__ void tma_box3(void *dst, const CUtensorMap *map, int x, int y, int z,
+                                         uint64_t *b) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];"
+        ::"r"(smem_addr(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_addr(b)) : "memory");
+}
+
+// One 2-D TMA box (elements x rows) into shared memory.
+__device__ __forceinline__ void tma_box2(void *dst, const CUtensorMap *map, int x, int y, uint64_t *b) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];"
+        ::"r"(smem_addr(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_addr(b)) : "memory");
+}
+
+// Arrival ticket: acquire-release add at GPU scope, returns the old value.
+__device__ __forceinline__ unsigned ticket_add_acq_rel(unsigned *p) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old;
+}
+
 // Bounded wait on an mbarrier phase (the hint lets the thread sleep).
 __device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) {
     for (uint32_t i = 0; i < (1u << 22); ++i) {
@@ -210,16 +238,19 @@ __device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) {
 }
 
 template <int R, int NT>
-__global__ void __launch_bounds__(kMmaWarps * 32)
-gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ scales,
-               const uint32_t *__restrict__ bq, const float *__restrict__ facg,
-               const float *__restrict__ offg, int M, int64_t N, int64_t K, int64_t tiles,
-               float *__restrict__ part, unsigned *__restrict__ tickets,
+__global__ void __launch_bounds__(kMmaWarps * 32, 2)
+gemv_i8_kernel(const __grid_constant__ CUtensorMap tmap, const __grid_constant__ CUtensorMap smap,
+               int scales_tma, const __half *__restrict__ scales, const uint32_t *__restrict__ bq,
+               const float *__restrict__ facg, const float *__restrict__ offg, int M, int64_t N,
+               int64_t K, int64_t tiles, float *__restrict__ part, unsigned *__restrict__ tickets,
                __nv_bfloat16 *__restrict__ Y) {
     using S = MmaSmem<R, NT>;
-    constexpr int GPT = S::GPT, RS = S::RS, JS = (GPT + 3) / 4;
-    constexpr int kStageWords = (int)(S::stage_bytes / 4);
-    extern __shared__ __align__(128) uint8_t smem[];
+    constexpr int GPT = S::GPT;
+    constexpr int kStageWords = (int)(S::stage_pitch / 4);
+    constexpr int ROWW = S::ROWB / 4;                       // words per tile row of a plane
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const uint4 *sB = reinterpret_cast<const uint4 *>(smem + S::bq);
     const float *sF = reinterpret_cast<const float *>(smem + S::fac);
     const float *sO = reinterpret_cast<const float *>(smem + S::off);
@@ -231,9 +262,11 @@ gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ s
     const int64_t G = K / kGroup;
     const int64_t g0 = (int64_t)ks * GPT;
     const int ng = (int)((g0 + GPT < G ? g0 + GPT : G) - g0);
-    const int64_t plane_words = N * (K / 32);
-    uint32_t *const stage0 = reinterpret_cast<uint32_t *>(smem + S::stages + 2 * warp * S::stage_bytes);
+    const int soff = (int)(g0 & 7);                         // first group inside the scale box
+    uint32_t *const stage0 = reinterpret_cast<uint32_t *>(smem + S::stages + 2 * warp * S::stage_pitch);
     uint64_t *wbar = bars + 1 + 2 * warp;
+    // 16-byte chunk of a row after the TMA swizzle (rows g and g + 8 agree)
+    const int swz = GPT == 8 ? (g & 7) : GPT == 4 ? ((g >> 1) & 3) : ((g >> 2) & 1);
 
     if (threadIdx.x == 0) {
         bar_init(&bars[0], 1);
@@ -241,6 +274,40 @@ gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ s
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
+
+    // Tiles of this warp: blockIdx.x + gridDim.x * (warp + kMmaWarps * j), so
+    // every CTA (and SM) gets the same number of tiles within one.
+    const int64_t stride = (int64_t)gridDim.x * kMmaWarps;
+    int64_t tile = blockIdx.x + (int64_t)gridDim.x * warp;
+
+    // One tile into stage `st`: planes (and scales) by TMA from lane 0; rows
+    // >= N and groups >= G arrive zero-filled.  Without a scale tensor map
+    // (G not a multiple of 8) lanes 0..15 copy their row's scales.
+    auto issue = [&](int st, int64_t tl) {
+        uint32_t *dst = stage0 + st * kStageWords;
+        if (lane == 0) {
+            bar_expect(wbar + st, (uint32_t)S::stage_bytes + (scales_tma ? 256u : 0u));
+            tma_box3(dst, &tmap, (int)(g0 * 4), (int)(tl * 16), 0, wbar + st);
+            if (scales_tma)
+                tma_box2(reinterpret_cast<uint8_t *>(dst) + S::stage_bytes, &smap,
+                         (int)(g0 - soff), (int)(tl * 16), wbar + st);
+        }
+        if (!scales_tma && lane < 16) {
+            const int64_t n = tl * 16 + lane;
+            __half *sd = reinterpret_cast<__half *>(reinterpret_cast<uint8_t *>(dst) + S::stage_bytes);
+#pragma unroll
+            for (int grp = 0; grp < GPT; ++grp)
+                sd[lane * 8 + soff + grp] = (n < N && grp < ng) ? scales[n * G + g0 + grp]
+                                                                : __float2half(0.f);
+        }
+    };
+
+    uint32_t phase_bits = 0u;
+    bool ok = true;
+    if (tile < tiles) issue(0, tile);
+    // Everything above reads only the weights; X-derived operands come from
+    // the preceding prep kernel of this call.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     if (threadIdx.x == 0) {
         const uint32_t bb = (uint32_t)ng * NT * 1024, fb = (uint32_t)ng * kCols * 4;
         bar_expect(&bars[0], bb + 2 * fb);
@@ -248,55 +315,17 @@ gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ s
         bulk_g2s(smem + S::fac, facg + g0 * kCols, fb, &bars[0]);
         bulk_g2s(smem + S::off, offg + g0 * kCols, fb, &bars[0]);
     }
-
-    const int64_t stride = (int64_t)gridDim.x * kMmaWarps;
-    int64_t tile = (int64_t)blockIdx.x * kMmaWarps + warp;
-
-    // One tile's plane rows into stage `st` (lane 0); each lane prefetches the
-    // scales of groups 4j + t for its rows g and g + 8.
-    float nsc[2][JS];
-    auto issue = [&](int st, int64_t tl) {
-        if (lane == 0) {
-            int rows = 0;
-            for (int rr = 0; rr < 16; ++rr) rows += (tl * 16 + rr < N);
-            bar_expect(wbar + st, (uint32_t)(rows * R * ng * 16));
-            for (int rr = 0; rr < rows; ++rr) {
-                const int64_t n = tl * 16 + rr;
-#pragma unroll
-                for (int p = 0; p < R; ++p)
-                    bulk_g2s(stage0 + st * kStageWords + rr * RS + p * GPT * 4,
-                             planes + p * plane_words + n * (K / 32) + g0 * 4,
-                             (uint32_t)ng * 16, wbar + st);
-            }
-        }
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-            const int64_t n = tl * 16 + g + 8 * hr;
-#pragma unroll
-            for (int j = 0; j < JS; ++j) {
-                const int grp = 4 * j + t;
-                nsc[hr][j] = (n < N && grp < ng) ? __half2float(scales[n * G + g0 + grp]) : 0.f;
-            }
-        }
-    };
-
-    uint32_t phase_bits = 0u;
-    bool ok = true;
-    if (tile < tiles) issue(0, tile);
     if (!bar_wait(&bars[0], 0)) ok = false;
     int st = 0;
-    float csc[2][JS];
     for (; tile < tiles && ok; tile += stride) {
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr)
-#pragma unroll
-            for (int j = 0; j < JS; ++j) csc[hr][j] = nsc[hr][j];
         const int64_t next = tile + stride;
         __syncwarp();
         if (next < tiles) issue(st ^ 1, next);
         if (!bar_wait(wbar + st, (phase_bits >> st) & 1u)) { ok = false; break; }
         phase_bits ^= 1u << st;
+        __syncwarp();
         const uint32_t *sw = stage0 + st * kStageWords;
+        const __half *ss = reinterpret_cast<const __half *>(reinterpret_cast<const uint8_t *>(sw) + S::stage_bytes);
 
         float y[NT][4];
 #pragma unroll
@@ -311,31 +340,31 @@ gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ s
             for (int hr = 0; hr < 2; ++hr) {
 #pragma unroll
                 for (int p = 0; p < 8; ++p)
-                    P[p] = p < R ? sw[(g + 8 * hr) * RS + p * GPT * 4 + grp * 4 + t] : 0u;
+                    P[p] = p < R ? sw[(p * 16 + g + 8 * hr) * ROWW + ((grp ^ swz) << 2) + t] : 0u;
                 operand_bytes<R>(P, A[hr]);
             }
-            const float s_lo = __shfl_sync(0xffffffffu, csc[0][grp / 4], g * 4 + (grp & 3));
-            const float s_hi = __shfl_sync(0xffffffffu, csc[1][grp / 4], g * 4 + (grp & 3));
+            const float s_lo = __half2float(ss[g * 8 + soff + grp]);
+            const float s_hi = __half2float(ss[(g + 8) * 8 + soff + grp]);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                int da[4] = {0, 0, 0, 0}, db[4] = {0, 0, 0, 0};
+                int d[4] = {0, 0, 0, 0};
                 const uint4 b0 = sB[((grp * NT + nt) * 2 + 0) * 32 + lane];
                 const uint4 b1 = sB[((grp * NT + nt) * 2 + 1) * 32 + lane];
                 uint32_t a[4];
                 a[0] = A[0][0]; a[1] = A[1][0]; a[2] = A[0][1]; a[3] = A[1][1];
-                mma_u8s8(da, a, b0.x, b0.y);
+                mma_u8s8(d, a, b0.x, b0.y);
                 a[0] = A[0][2]; a[1] = A[1][2]; a[2] = A[0][3]; a[3] = A[1][3];
-                mma_u8s8(db, a, b0.z, b0.w);
+                mma_u8s8(d, a, b0.z, b0.w);
                 a[0] = A[0][4]; a[1] = A[1][4]; a[2] = A[0][5]; a[3] = A[1][5];
-                mma_u8s8(da, a, b1.x, b1.y);
+                mma_u8s8(d, a, b1.x, b1.y);
                 a[0] = A[0][6]; a[1] = A[1][6]; a[2] = A[0][7]; a[3] = A[1][7];
-                mma_u8s8(db, a, b1.z, b1.w);
+                mma_u8s8(d, a, b1.z, b1.w);
                 const float2 f = *reinterpret_cast<const float2 *>(sF + grp * kCols + 8 * nt + 2 * t);
                 const float2 o = *reinterpret_cast<const float2 *>(sO + grp * kCols + 8 * nt + 2 * t);
-                y[nt][0] = fmaf(s_lo, fmaf(f.x, (float)(da[0] + db[0]), o.x), y[nt][0]);
-                y[nt][1] = fmaf(s_lo, fmaf(f.y, (float)(da[1] + db[1]), o.y), y[nt][1]);
-                y[nt][2] = fmaf(s_hi, fmaf(f.x, (float)(da[2] + db[2]), o.x), y[nt][2]);
-                y[nt][3] = fmaf(s_hi, fmaf(f.y, (float)(da[3] + db[3]), o.y), y[nt][3]);
+                y[nt][0] = fmaf(s_lo, fmaf(f.x, (float)d[0], o.x), y[nt][0]);
+                y[nt][1] = fmaf(s_lo, fmaf(f.y, (float)d[1], o.y), y[nt][1]);
+                y[nt][2] = fmaf(s_hi, fmaf(f.x, (float)d[2], o.x), y[nt][2]);
+                y[nt][3] = fmaf(s_hi, fmaf(f.y, (float)d[3], o.y), y[nt][3]);
             }
         }
         st ^= 1;
@@ -374,10 +403,9 @@ gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ s
             const int64_t n = tile * 16 + rr;
             if (idx < 16 * M && n < N) part[((int64_t)ks * M + m) * N + n] = out[q];
         }
-        __threadfence();
-        __syncwarp();
+        __syncwarp();                      // the warp's partials before lane 0's release
         unsigned last = 0;
-        if (lane == 0) last = atomicAdd(&tickets[tile], 1u) == (unsigned)KS - 1;
+        if (lane == 0) last = ticket_add_acq_rel(&tickets[tile]) == (unsigned)KS - 1;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) continue;
         __threadfence();
@@ -394,13 +422,81 @@ gemv_i8_kernel(const uint32_t *__restrict__ planes, const __half *__restrict__ s
     if (!ok && lane == 0) atomicOr(&g_gemv_timeout, 1u);
 }
 
+// Tensor map of the fp16 scales [N][G] with a 16 x 8 box; needs G % 8 == 0
+// (row pitch a multiple of 16 bytes).
+mq_status scale_map(const mq_weights *w, CUtensorMap *out, bool *ok) {
+    const int64_t G = w->K / kGroup;
+    *ok = (G % 8) == 0;
+    if (!*ok) { memset(out, 0, sizeof(*out)); return MQ_OK; }
+    struct Slot { const void *p; int64_t N, K; CUtensorMap map; };
+    static thread_local Slot cache[32];
+    static thread_local int next = 0;
+    for (auto &c : cache)
+        if (c.p == w->scales && c.N == w->N && c.K == w->K) { *out = c.map; return MQ_OK; }
+    void *fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn)
+        return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+    auto encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    const cuuint64_t dims[2] = {(cuuint64_t)G, (cuuint64_t)w->N};
+    const cuuint64_t strides[1] = {(cuuint64_t)(G * 2)};
+    const cuuint32_t box[2] = {8u, 16u};
+    const cuuint32_t estr[2] = {1u, 1u};
+    CUtensorMap m;
+    const CUresult res = encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t *>(w->scales),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (res != CUDA_SUCCESS) return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the scales");
+    cache[next] = Slot{w->scales, w->N, w->K, m};
+    next = (next + 1) % 32;
+    *out = m;
+    return MQ_OK;
+}
+
 struct MmaPlan {
     int KS, NT;
     int64_t tiles, ctas_x;
     size_t part_off, bq_off, fac_off, off_off, ws_bytes;
 };
 
-int plan_gpt(int r) { return r >= 6 ? 2 : 16 / r; }
+int plan_gpt(int r) { return r <= 2 ? 8 : r <= 4 ? 4 : 2; }
+
+// Tensor map of the r planes seen as [r][N][K/32] uint32, box (4 GPT words,
+// 16 rows, r planes), swizzled so that a warp's operand reads are
+// conflict-free.  Encoded through the runtime's driver entry point and cached
+// per (buffer, shape, r).
+mq_status plane_map(const mq_weights *w, int gpt, CUtensorMap *out) {
+    struct Slot { const void *p; int64_t N, K; int r; CUtensorMap map; };
+    static thread_local Slot cache[32];
+    static thread_local int next = 0;
+    for (auto &c : cache)
+        if (c.p == w->planes && c.N == w->N && c.K == w->K && c.r == w->r) { *out = c.map; return MQ_OK; }
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (!encode) {
+        cudaDriverEntryPointQueryResult q;
+        void *fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            !fn)
+            return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)(w->K / 32), (cuuint64_t)w->N, (cuuint64_t)w->r};
+    const cuuint64_t strides[2] = {(cuuint64_t)(w->K / 8), (cuuint64_t)(w->N * (w->K / 8))};
+    const cuuint32_t box[3] = {(cuuint32_t)(4 * gpt), 16u, (cuuint32_t)w->r};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUtensorMapSwizzle sw = gpt == 8 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : gpt == 4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+    CUtensorMap m;
+    const CUresult res = encode(&m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint32_t *>(w->planes),
+                                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (res != CUDA_SUCCESS) return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled failed for the planes");
+    cache[next] = Slot{w->planes, w->N, w->K, w->r, m};
+    next = (next + 1) % 32;
+    *out = m;
+    return MQ_OK;
+}
 
 MmaPlan mma_plan(int64_t M, int64_t N, int64_t K, int r) {
     MmaPlan p{};
@@ -443,11 +539,29 @@ mq_status run_i8(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
         if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
         attr_set = true;
     }
-    dim3 grid((unsigned)p.ctas_x, (unsigned)p.KS);
-    gemv_i8_kernel<R, NT><<<grid, kMmaWarps * 32, smem, st>>>(
-        w->planes, reinterpret_cast<const __half *>(w->scales), bq, fac, off, (int)M, w->N, w->K,
-        p.tiles, reinterpret_cast<float *>(ws + p.part_off), reinterpret_cast<unsigned *>(ws),
-        reinterpret_cast<__nv_bfloat16 *>(Y));
+    CUtensorMap tmap, smap;
+    bool stma = false;
+    mq_status ms = plane_map(w, MmaSmem<R, NT>::GPT, &tmap);
+    if (ms == MQ_OK) ms = scale_map(w, &smap, &stma);
+    if (ms != MQ_OK) return ms;
+    // programmatic dependent launch: the kernel starts streaming weights while
+    // the prep kernel finishes, and waits for it before reading its output
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.ctas_x, (unsigned)p.KS);
+    cfg.blockDim = dim3(kMmaWarps * 32);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, gemv_i8_kernel<R, NT>, tmap, smap, stma ? 1 : 0,
+                           reinterpret_cast<const __half *>(w->scales),
+                           (const uint32_t *)bq, (const float *)fac, (const float *)off, (int)M,
+                           w->N, w->K, p.tiles, reinterpret_cast<float *>(ws + p.part_off),
+                           reinterpret_cast<unsigned *>(ws), reinterpret_cast<__nv_bfloat16 *>(Y));
+    if (e != cudaSuccess) return cuda_fail(e, "gemv_i8_kernel launch");
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "gemv_i8_kernel");
     return MQ_OK;
