@@ -156,6 +156,31 @@ MQ_API int mq_get_gemv_variant(void);
  */
 MQ_API mq_status mq_unpack(const mq_weights *w, uint8_t *codes_out, void *stream);
 
+/*
+ * mq_gemv_noalloc: Y = X . W_r^T for 1 <= M <= 8 without a workspace.  For
+ * callers that cannot call cudaMalloc where they run the layer: a plugin
+ * whose host application owns all device memory and offers no allocator, a
+ * server that hands the whole GPU to its own memory pool at start-up, or a
+ * latency-critical loop that must not take cudaMalloc's implicit device
+ * synchronisation.  The paper has no counterpart: this is a calling
+ * convention, not part of the method.
+ *   Arguments and results are those of mq_gemm without the workspace.
+ *   Scratch: a 16 MiB array compiled into the library, resident on every GPU
+ *   that loads it until the process exits.  Problems whose
+ *   mq_gemm_workspace_bytes exceeds 16 MiB return MQ_ERR_WORKSPACE; M > 8
+ *   returns MQ_ERR_INVALID_ARG.  Both checks happen before any launch.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture.  Each call clears the array's arrival tickets (one
+ *   cudaMemsetAsync on `stream`) and overwrites the rest.
+ *   All calls share the one array, which keeps the last call's contents:
+ *   calls that can overlap on the GPU (other streams, other host threads)
+ *   race and must be serialised by the caller.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+MQ_API mq_status mq_gemv_noalloc(const uint16_t *X_dev, const mq_weights *w, int64_t M,
+                                 int64_t N, int64_t K, uint16_t *Y_dev, void *stream);
+
 /* Status of the most recent failing call on this host thread (MQ_OK if none). */
 MQ_API mq_status mq_last_error(void);
 
