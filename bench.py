@@ -142,24 +142,51 @@ def reduce_max(x: float, ws: int) -> float:
 
 
 def cpu_oracle_sample(layers, budget_s: float = 12.0):
-    """The plain-C oracle on whole layers of the same step until ~budget_s."""
+    """The plain-C oracle on whole layers of the same step for about budget_s."""
     import oracle
     done_bytes, t_total, n_layers = 0, 0.0, 0
     order = [(r, i) for r in R_LIST for i in range(len(wl.LLAMA8B))]
-    while n_layers == 0 or (t_total < budget_s and n_layers < 4 * len(order)):
+    xs = [wl.bf16_bits_to_f32(xbits) for (_, _, xbits) in layers]
+    while n_layers == 0 or t_total < budget_s:
         r, i = order[n_layers % len(order)]
         l = wl.LLAMA8B[i]
-        codes, s, xbits = layers[i]
-        X = wl.bf16_bits_to_f32(xbits)
+        codes, s, _ = layers[i]
         t0 = time.perf_counter()
-        oracle.gemm(X, codes, s, r)
+        oracle.gemm(xs[i], codes, s, r)
         t_total += time.perf_counter() - t0
         done_bytes += algo_bytes(l.N, l.K, r)
         n_layers += 1
     return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": f"{n_layers} layer GEMVs of the step (M=1, fp64 C oracle, OpenMP), "
-                      f"{t_total:.1f} s"}
+            "sample": f"{n_layers} layer products of the step (M=1, r in {{4,3,2}}, in step "
+                      f"order), fp64 C oracle with OpenMP, {t_total:.1f} s"}
+
+
+def run_case(args):
+    """One layer, launched eagerly: the small case for ncu captures.
+
+    --case N,K,M,r  runs --warmup + --steps launches of mq_gemm on that shape
+    (seeded weights and X) and prints the CUDA-event time per launch."""
+    import torch
+    import nested_bit_weight_b200 as mq
+    N, K, M, r = (int(v) for v in args.case.split(","))
+    codes, s, _ = wl.gen_weights(N, K, seed=N + K)
+    xbits, _ = wl.gen_x(M, K, seed=N + K)
+    p = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    X = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    for _ in range(args.warmup):
+        mq.gemm(X, p, r, Y=Y)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        mq.gemm(X, p, r, Y=Y)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) / max(args.steps, 1) * 1e3
+    print(json.dumps({"case": [N, K, M, r], "us_per_launch_eager": round(us, 3),
+                      "GBps": round(algo_bytes(N, K, r, M) / (us * 1e-6) / 1e9, 1)}), flush=True)
 
 
 def run_mq(args, ws_n, rank, local):
@@ -316,7 +343,7 @@ def run_mq(args, ws_n, rank, local):
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "mq_gemm M<=8 call: bfrag prep + gemv_mma_kernel, "
+                     "kernel": "nested_gemv_kernel (one launch per mq_gemm call), "
                                "all 21 calls of the step",
                      "frac_of_8TBps": round(achieved / 8000.0, 4)},
         "e2e": {"value": round(ws_n * sb / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
@@ -329,6 +356,88 @@ def run_mq(args, ws_n, rank, local):
     return out, layers
 
 
+def run_sweep(args):
+    """Per-(layer, M, r) isolated timings for one workload table (configs of
+    workloads.CONFIGS), weights rotated over more than twice the L2 so every
+    launch reads its planes from HBM.  Prints one JSON line per point and a
+    markdown table."""
+    import torch
+    import nested_bit_weight_b200 as mq
+    peak, _ = read_peaks()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    cfgs = sorted(wl.CONFIGS) if args.sweep == "all" else [int(c) for c in args.sweep.split(",")]
+    rows = []
+    for ci in cfgs:
+        cfg = wl.CONFIGS[ci]
+        done = {}
+        for li, layer in enumerate(cfg["layers"]):
+            key = (layer.N, layer.K)
+            if key in done:            # same shape as an earlier layer: same numbers
+                for r_ in done[key]:
+                    rows.append(dict(r_, layer=layer.name))
+                continue
+            codes, s, _ = wl.gen_weights(layer.N, layer.K, wl.layer_seed(ci, li))
+            p0 = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+            del codes
+            pbytes = p0.planes.numel() * 4 + p0.scales16.numel() * 2
+            copies = max(1, -(-2 * l2 // pbytes))
+            parents = [p0] + [mq.NestedWeights(p0.planes.clone(), p0.scales16.clone(), p0.N, p0.K)
+                              for _ in range(copies - 1)]
+            rs = cfg["r"] if cfg["r"] is not None else (wl.QWEN3_R[layer.name],)
+            out_rows = []
+            for M in cfg["M"]:
+                xbits, _ = wl.gen_x(M, layer.K, wl.layer_seed(ci, li), outlier_channels=(ci == 3))
+                X = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+                Y = torch.empty((M, layer.N), dtype=torch.bfloat16, device="cuda")
+                for r in rs:
+                    need = mq.mq_gemm_workspace_bytes(M, layer.N, layer.K, r)
+                    ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda")
+                    views = [q.view(r) for q in parents]
+                    n_launch = max(len(views), 24)
+                    stream = torch.cuda.Stream()
+                    with torch.cuda.stream(stream):
+                        for v in views:
+                            mq.mq_gemm(X, v, Y, ws)
+                        torch.cuda.synchronize()
+                        g = torch.cuda.CUDAGraph()
+                        with torch.cuda.graph(g, stream=stream):
+                            for j in range(n_launch):
+                                mq.mq_gemm(X, views[j % len(views)], Y, ws)
+                        for _ in range(3):
+                            g.replay()
+                        torch.cuda.synchronize()
+                        e0 = torch.cuda.Event(enable_timing=True)
+                        e1 = torch.cuda.Event(enable_timing=True)
+                        reps = 5
+                        e0.record()
+                        for _ in range(reps):
+                            g.replay()
+                        e1.record()
+                    torch.cuda.synchronize()
+                    us = e0.elapsed_time(e1) * 1e3 / (reps * n_launch)
+                    del g
+                    b = algo_bytes(layer.N, layer.K, r, M)
+                    fl = 2.0 * M * layer.N * layer.K
+                    row = {"config": ci, "layer": layer.name, "N": layer.N, "K": layer.K, "M": M,
+                           "r": r, "us": round(us, 3), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+                           "TFLOPs": round(fl / (us * 1e-6) / 1e12, 2),
+                           "frac_hbm_measured": round(b / (us * 1e-6) / 1e9 / peak, 3),
+                           "frac_8TBps": round(b / (us * 1e-6) / 8e12, 3),
+                           "path": "gemv" if M <= 8 else "tcgen05 gemm"}
+                    out_rows.append(row)
+                    rows.append(row)
+                    print(json.dumps(row), flush=True)
+            done[key] = out_rows
+            del parents, p0
+            torch.cuda.empty_cache()
+    print("| config | layer | N | K | M | r | µs | GB/s | TFLOP/s | frac of measured HBM | frac of 8 TB/s | path |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|---|")
+    for r_ in rows:
+        print(f"| {r_['config']} | {r_['layer']} | {r_['N']} | {r_['K']} | {r_['M']} | {r_['r']} | "
+              f"{r_['us']} | {r_['GBps']} | {r_['TFLOPs']} | {r_['frac_hbm_measured']} | "
+              f"{r_['frac_8TBps']} | {r_['path']} |")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -336,7 +445,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="mq", choices=["mq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="N,K,M,r: one layer, eager launches (for ncu)")
+    ap.add_argument("--sweep", default=None, help="config indices (e.g. 0,1,2) or 'all': "
+                                                  "per-(layer, M, r) isolated timings")
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
+    if args.sweep:
+        run_sweep(args)
+        return
     ws_n, rank, local = dist_init()
     if args.impl == "reference":
         if rank == 0:

@@ -31,12 +31,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Wait for the phase with the given parity; false if the wait gave up.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
-                                                  uint32_t max_tries = (1u << 24)) {
-    for (uint32_t i = 0; i < max_tries; ++i)
+// Wait for the phase with the given parity; false if the wait gave up after
+// about a second (so that a lost arrival cannot hang the GPU).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0, t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-    return false;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+        if (t - t0 > 1000000000ull) return false;
+    }
 }
 
 // ------------------------------------------------------------------- tcgen05

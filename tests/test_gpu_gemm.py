@@ -138,6 +138,24 @@ def test_deterministic_and_workspace_reusable():
     assert oracle.violation_ratio(outs[0], oracle.gemm(X, codes, s, 3)) <= 1.0
 
 
+@pytest.mark.parametrize("N,K,M,r", [(2048, 14336, 1, 4), (2048, 14336, 8, 8), (2048, 14336, 8, 2),
+                                      (1024, 14336, 4, 3), (2000, 8192, 8, 6), (300, 28672, 3, 5)])
+def test_gemv_stage_ring_and_k_segments(N, K, M, r):
+    # more items per CTA than shared-memory stages (the ring wraps), and X
+    # operands too large for one CTA (K cut into segments, so every tile is
+    # combined across CTAs through the workspace); twice, bit-identical
+    import torch
+    import nested_bit_weight_b200 as mq
+    codes, s, _ = wl.gen_weights(N, K, seed=N + K + M + r)
+    xbits, X = wl.gen_x(M, K, seed=N + K + M + r)
+    parent = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    Xd = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+    Y1 = mq.gemm(Xd, parent, r).float().cpu().numpy()
+    Y2 = mq.gemm(Xd, parent, r).float().cpu().numpy()
+    assert np.array_equal(Y1, Y2)
+    assert oracle.violation_ratio(Y1.astype(np.float64), oracle.gemm(X, codes, s, r)) <= 1.0
+
+
 LLAMA = [(l.name, l.N, l.K) for l in wl.LLAMA8B]
 
 
