@@ -96,11 +96,16 @@ def dequant(codes: np.ndarray, s: np.ndarray, r: int) -> np.ndarray:
 
 # ------------------------------------------------------------- plain-C kernels
 
+def rows128(N: int) -> int:
+    """Rows of the stored planes and scales: N padded to a multiple of 128."""
+    return (N + 127) // 128 * 128
+
+
 def pack(codes: np.ndarray) -> np.ndarray:
-    """8 MSB-first bit planes, uint32 [8, N, K/32]."""
+    """8 MSB-first bit planes in the tiled layout, uint32 [8, rows128(N) * K/32]."""
     codes = np.ascontiguousarray(codes, np.uint8)
     N, K = codes.shape
-    out = np.empty((8, N, K // 32), np.uint32)
+    out = np.empty((8, rows128(N) * (K // 32)), np.uint32)
     _load().oracle_pack(_ptr(codes), N, K, _ptr(out))
     return out
 
@@ -108,10 +113,25 @@ def pack(codes: np.ndarray) -> np.ndarray:
 def unpack(planes: np.ndarray, r: int, N: int, K: int) -> np.ndarray:
     """r-bit codes read from the first r planes, uint8 [N, K]."""
     planes = np.ascontiguousarray(planes, np.uint32)
-    if planes.size < r * N * (K // 32):
+    if planes.size < r * rows128(N) * (K // 32):
         raise ValueError("plane buffer too small")
     out = np.empty((N, K), np.uint8)
     _load().oracle_unpack(_ptr(planes), N, K, r, _ptr(out))
+    return out
+
+
+def scales_stored(s: np.ndarray) -> np.ndarray:
+    """The stored scales: fp16 (RNE) in the tiled order of the planes, the
+    128 rows of block (t, g) contiguous at ((t * G + g) * 128); padding rows 0."""
+    s16 = scales_f16(s)
+    N, G = s16.shape
+    Np = rows128(N)
+    full = np.zeros((Np, G), np.float16)
+    full[:N] = s16
+    out = np.empty(Np * G, np.float16)
+    for t in range(Np // 128):
+        for g in range(G):
+            out[(t * G + g) * 128:(t * G + g + 1) * 128] = full[t * 128:(t + 1) * 128, g]
     return out
 
 

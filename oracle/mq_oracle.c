@@ -17,28 +17,39 @@
  *   weight:  w[n,k] = s16[n, k/128] * v_r[n,k]
  *   output:  Y[m,n] = sum_k X[m,k] * w[n,k]   (fp64, ascending k)
  *
- * Bit-plane layout (the exact-r-bit storage): planes[p][n][K/32] of uint32,
- * p = 0..7; plane p holds bit (7 - p) of the parent code (most significant
- * plane first) and bit j of word w of row n holds the code at k = 32*w + j.
- * An r-bit model is the first r planes.
+ * Bit-plane layout (the exact-r-bit storage, the library's own format: the
+ * pages fix no layout).  Rows are padded with zero rows to N128, a multiple
+ * of 128; G = K / 128.  The buffer is 8 planes of N128*K/32 uint32 words,
+ * plane p holding bit (7 - p) of the parent code (most significant plane
+ * first), so an r-bit model is the first r planes.  Inside a plane the
+ * 128-row x 128-column block (t, g) occupies the 512 words starting at
+ * (t*G + g)*512; row i of the block is words 4i .. 4i+3, and bit j of word w
+ * of that row holds the code at column 128g + 32w + j.
  */
 #include <stdint.h>
 #include <stddef.h>
+#include <string.h>
 
-/* Build the 8 planes bit by bit from the parent codes. */
+static int64_t rows128(int64_t N) { return (N + 127) / 128 * 128; }
+
+/* Word index of (plane p, row n, column k) in the tiled layout. */
+static int64_t word_at(int p, int64_t n, int64_t k, int64_t N, int64_t K)
+{
+    int64_t G = K / 128;
+    int64_t plane = rows128(N) * (K / 32);
+    return p * plane + ((n / 128) * G + k / 128) * 512 + (n % 128) * 4 + (k % 128) / 32;
+}
+
+/* Build the 8 planes bit by bit from the parent codes (padding rows zero). */
 void oracle_pack(const uint8_t *codes, int64_t N, int64_t K, uint32_t *planes)
 {
-    int64_t W = K / 32;
+    memset(planes, 0, (size_t)8 * rows128(N) * (K / 32) * sizeof(uint32_t));
     for (int p = 0; p < 8; ++p) {
         for (int64_t n = 0; n < N; ++n) {
-            for (int64_t w = 0; w < W; ++w) {
-                uint32_t word = 0;
-                for (int j = 0; j < 32; ++j) {
-                    uint8_t q = codes[n * K + 32 * w + j];
-                    uint32_t bit = (q >> (7 - p)) & 1u;
-                    word |= bit << j;
-                }
-                planes[((int64_t)p * N + n) * W + w] = word;
+            for (int64_t k = 0; k < K; ++k) {
+                uint8_t q = codes[n * K + k];
+                uint32_t bit = (q >> (7 - p)) & 1u;
+                planes[word_at(p, n, k, N, K)] |= bit << (k % 32);
             }
         }
     }
@@ -48,12 +59,11 @@ void oracle_pack(const uint8_t *codes, int64_t N, int64_t K, uint32_t *planes)
 void oracle_unpack(const uint32_t *planes, int64_t N, int64_t K, int r,
                    uint8_t *codes_r)
 {
-    int64_t W = K / 32;
     for (int64_t n = 0; n < N; ++n) {
         for (int64_t k = 0; k < K; ++k) {
             unsigned q = 0;
             for (int p = 0; p < r; ++p) {
-                uint32_t word = planes[((int64_t)p * N + n) * W + k / 32];
+                uint32_t word = planes[word_at(p, n, k, N, K)];
                 unsigned bit = (word >> (k % 32)) & 1u;
                 q = (q << 1) | bit;      /* plane 0 is the most significant */
             }

@@ -18,20 +18,27 @@ KINDS = ("zeros", "ones", "alternating", "single_bit", "all_codes", "random")
 
 
 def _packbits_planes(codes):
-    """Plane words via numpy's packbits (an independent route to the layout):
-    bit j of word w of plane p is bit (7 - p) of code k = 32 w + j."""
+    """Plane words via numpy's packbits and reshapes (an independent route to
+    the layout): bit j of row-word w of plane p is bit (7 - p) of code
+    k = 32 w + j; rows are padded with zeros to a multiple of 128 and the
+    128 x 128 blocks (row tile t, group g) are laid out t-major, each block
+    row-major with 4 words per row."""
     N, K = codes.shape
-    out = np.empty((8, N, K // 32), np.uint32)
+    Np, G = (N + 127) // 128 * 128, K // 128
+    rows = np.zeros((8, Np, K // 32), np.uint32)
     for p in range(8):
         bits = ((codes >> (7 - p)) & 1).astype(np.uint8)
         by = np.packbits(bits, axis=1, bitorder="little")          # N x K/8
-        out[p] = by.reshape(N, K // 32, 4).copy().view("<u4")[..., 0]
-    return out
+        rows[p, :N] = by.reshape(N, K // 32, 4).copy().view("<u4")[..., 0]
+    # [p][t][i][g][w] -> [p][t][g][i][w]
+    tiled = rows.reshape(8, Np // 128, 128, G, 4).transpose(0, 1, 3, 2, 4)
+    return np.ascontiguousarray(tiled).reshape(8, -1)
 
 
 @pytest.mark.parametrize("kind", KINDS)
-def test_pack_matches_packbits(kind):
-    codes = wl.adversarial_codes(kind, 24, 256, seed=3)
+@pytest.mark.parametrize("N,K", [(24, 256), (130, 384), (256, 128)])
+def test_pack_matches_packbits(kind, N, K):
+    codes = wl.adversarial_codes(kind, N, K, seed=3)
     assert np.array_equal(oracle.pack(codes), _packbits_planes(codes))
 
 
@@ -48,17 +55,33 @@ def test_pack_unpack_identity_and_prefix(kind):
 
 
 def test_pack_single_code_positions():
-    # brute force: one set code at each position lands in exactly one bit
-    N, K = 2, 64
-    for n in range(N):
-        for k in range(0, K, 7):
-            for b in range(8):
+    # brute force: one set code at each position lands in exactly one bit, at
+    # the word the layout definition gives (written out here independently)
+    N, K = 200, 384
+    G = K // 128
+    for n in (0, 1, 127, 128, 199):
+        for k in (0, 5, 31, 32, 127, 128, 300, 383):
+            for b in (0, 3, 7):
                 codes = np.zeros((N, K), np.uint8)
                 codes[n, k] = 1 << b
                 planes = oracle.pack(codes)
+                word = ((n // 128) * G + k // 128) * 512 + (n % 128) * 4 + (k % 128) // 32
                 nz = np.argwhere(planes)
-                assert nz.tolist() == [[7 - b, n, k // 32]]
-                assert planes[7 - b, n, k // 32] == np.uint32(1 << (k % 32))
+                assert nz.tolist() == [[7 - b, word]]
+                assert planes[7 - b, word] == np.uint32(1 << (k % 32))
+
+
+def test_scales_stored_layout():
+    # the stored scales follow the planes' block order: (t, g) block of 128 rows
+    N, K = 130, 384
+    s = wl.gen_scales(N, K, seed=3)
+    st = oracle.scales_stored(s)
+    s16 = oracle.scales_f16(s)
+    assert st.shape == (256 * 3,)
+    for n in (0, 77, 127, 128, 129):
+        for g in range(3):
+            assert st[((n // 128) * 3 + g) * 128 + n % 128] == s16[n, g]
+    assert np.all(st[(1 * 3 + 0) * 128 + 2:(1 * 3 + 1) * 128] == 0)   # padding rows
 
 
 def test_slicing_is_nested():

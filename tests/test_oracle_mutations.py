@@ -27,7 +27,9 @@ MUTATIONS = {
     "x_transposed": ("acc += X[m * K + k] * w;\n        }\n        out[i]",
                      "acc += X[k * 1 + m] * w;\n        }\n        out[i]"),
     "plane_order": ("(q >> (7 - p)) & 1u", "(q >> p) & 1u"),
-    "bit_order": ("word |= bit << j;", "word |= bit << (31 - j);"),
+    "bit_order": ("|= bit << (k % 32);", "|= bit << (31 - k % 32);"),
+    "block_row": ("(n % 128) * 4 + (k % 128) / 32;", "(n % 128) + (k % 128) / 32 * 128;"),
+    "block_order": ("((n / 128) * G + k / 128) * 512", "((k / 128) * G + n / 128) * 512"),
 }
 
 
@@ -51,9 +53,9 @@ def _pins_pass(lib):
     """Re-run the independent pins against the mutant; True if all hold."""
     ptr = lambda a: a.ctypes.data_as(ctypes.c_void_p)
     # pin 1: layout against numpy packbits
-    codes = wl.adversarial_codes("random", 8, 128, seed=1)
-    planes = np.empty((8, 8, 4), np.uint32)
-    lib.oracle_pack(ptr(codes), 8, 128, ptr(planes))
+    codes = wl.adversarial_codes("random", 130, 256, seed=1)
+    planes = np.empty((8, 256 * 8), np.uint32)
+    lib.oracle_pack(ptr(codes), 130, 256, ptr(planes))
     from tests.test_oracle import _packbits_planes, _exact_gemm
     if not np.array_equal(planes, _packbits_planes(codes)):
         return False
