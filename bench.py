@@ -343,7 +343,7 @@ def run_mq(args, ws_n, rank, local):
                      "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "nested_gemv_kernel (one launch per mq_gemm call), "
+                     "kernel": "nested_gemv_tc_kernel (one launch per mq_gemm call), "
                                "all 21 calls of the step",
                      "frac_of_8TBps": round(achieved / 8000.0, 4)},
         "e2e": {"value": round(ws_n * sb / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",

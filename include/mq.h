@@ -18,12 +18,18 @@
  *   W_r    [n, k] = s[n, k / 128] * v_r[n, k]
  *   Y      = X . W_r^T, X is M x K bf16 row-major, Y is M x N bf16 row-major
  *
- * Storage ("bit planes"): planes[p][n][K/32] of uint32, p = 0..7, plane p
- * holds bit (7 - p) of q (most significant plane first), and bit j of word w
- * of row n holds the code of column k = 32 w + j.  One aligned 16-byte vector
- * is one 128-column group of one plane.  The r-bit model is the prefix made
- * of the first r planes (r * N * K / 8 bytes), so it reads exactly r bits
- * per weight; planes of a weight set are always N * K / 32 words apart.
+ * Storage ("bit planes", the library's own layout; the pages fix none):
+ * rows are padded with zero rows to N128 = 128 * ceil(N / 128).  The buffer
+ * holds 8 planes of N128 * K / 32 uint32 words; plane p holds bit (7 - p) of
+ * q (most significant plane first), so the r-bit model is the prefix made of
+ * the first r planes (r * N128 * K / 8 bytes) and reads exactly r bits per
+ * stored weight.  Inside a plane, the 128-row x 128-column block (row tile
+ * t, column group g) is 512 contiguous words at (t * G + g) * 512, G = K/128;
+ * row i of the block is the 4 words at 4 i, and bit j of word w holds the
+ * code of column 128 g + 32 w + j.  The fp16 scales follow the same block
+ * order: the 128 rows of block (t, g) at (t * G + g) * 128 (padding rows 0).
+ * A run of consecutive (t, g) blocks is therefore one contiguous stream per
+ * plane.
  *
  * Conventions:
  *   - All pointers named *_dev are device pointers; the caller owns every
@@ -64,17 +70,17 @@ typedef enum {
 /* A view of an r-bit weight set inside a bit-plane buffer (no ownership). */
 typedef struct {
     const uint32_t *planes;   /* device: plane 0 of the buffer; first r planes are read */
-    const uint16_t *scales;   /* device: fp16 scales, N x (K / group), row-major */
+    const uint16_t *scales;   /* device: fp16 scales in the tiled block order (see above) */
     int64_t N;                /* output features (rows of W) */
     int64_t K;                /* input features, multiple of 128 */
     int32_t group;            /* columns per scale; must be 128 */
     int32_t r;                /* bits per weight, 1..8 */
 } mq_weights;
 
-/* Bytes of the first r planes: r * N * K / 8 (0 on invalid arguments). */
+/* Bytes of the first r planes: r * N128 * K / 8 (0 on invalid arguments). */
 MQ_API size_t mq_plane_bytes(int64_t N, int64_t K, int r);
 
-/* Bytes of the fp16 scales: 2 * N * (K / group) (0 on invalid arguments). */
+/* Bytes of the stored fp16 scales: 2 * N128 * (K / group) (0 on invalid arguments). */
 MQ_API size_t mq_scale_bytes(int64_t N, int64_t K, int group);
 
 /*
@@ -83,8 +89,9 @@ MQ_API size_t mq_scale_bytes(int64_t N, int64_t K, int group);
  * r-bit loading"; "single multi-precision checkpoint").
  *   codes_dev   uint8 N x K (row-major), the 8-bit parent codes
  *   scales_dev  fp32 N x (K/group), the per-group scales
- *   planes_out  uint32 [8][N][K/32] (mq_plane_bytes(N, K, 8) bytes)
- *   scales_out  fp16 bits N x (K/group), round-to-nearest-even of scales_dev
+ *   planes_out  the 8 tiled planes (mq_plane_bytes(N, K, 8) bytes)
+ *   scales_out  fp16 bits in the tiled block order (mq_scale_bytes(N, K, 128)
+ *               bytes), round-to-nearest-even of scales_dev
  * Preconditions: N >= 1, K >= 128, K % 128 == 0, group == 128, all four
  * pointers 16-byte aligned, buffers do not overlap.
  * Synchronous: returns after the work on `stream` has finished, because it
@@ -112,8 +119,8 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
 /*
  * Y = X . W_r^T (MatGPTQ abstract: kernels for the nested format that serve
- * batch sizes beyond one).  M <= 8 runs a split-K GEMV (see
- * mq_set_gemv_variant); M >= 9 runs the tcgen05 tensor-core GEMM.
+ * batch sizes beyond one).  M <= 8 runs the tcgen05 GEMV (decoded weights in
+ * tensor memory; see mq_set_gemv_variant); M >= 9 runs the tcgen05 GEMM.
  *   X_dev      bf16 M x K row-major
  *   w          r-bit view (from mq_slice, or a parent with r = 8)
  *   Y_dev      bf16 M x N row-major (written, not accumulated)
@@ -134,20 +141,21 @@ MQ_API mq_status mq_gemm(const uint16_t *X_dev, const mq_weights *w,
 
 /* Kernels for M <= 8 (both compute the same Y within the stated tolerance). */
 enum {
-    MQ_GEMV_MMA = 0,   /* default: bf16 operands built in registers, warp MMA m16n8k16 */
-    MQ_GEMV_SIMT = 1   /* CUDA-core fp32 FMA GEMV with warp-shuffle reduction */
+    MQ_GEMV_TC = 0,        /* default: 128 rows per tensor-core MMA, int8 operands,
+                              decoded weights stored in tensor memory */
+    MQ_GEMV_VIA_GEMM = 1   /* the M >= 9 tcgen05 GEMM (bf16 operands), M padded to 16 */
 };
 
 /*
  * Choose the M <= 8 kernel for later mq_gemm calls in this process (host
  * only, no device work).  Returns MQ_ERR_INVALID_ARG for an unknown value.
  * Both variants follow the same definition of Y (MatGPTQ abstract: kernels
- * for slicing and mixed-precision execution); they differ only in which
- * units do the multiply-adds.
+ * for slicing and mixed-precision execution); shapes whose operands do not
+ * fit the GEMV's shared memory always take the GEMM.
  */
 MQ_API mq_status mq_set_gemv_variant(int variant);
 
-/* The M <= 8 kernel in use (MQ_GEMV_MMA or MQ_GEMV_SIMT). */
+/* The M <= 8 kernel in use (MQ_GEMV_TC or MQ_GEMV_VIA_GEMM). */
 MQ_API int mq_get_gemv_variant(void);
 
 /*

@@ -16,7 +16,7 @@ __all__ = [
     "MQError", "MqWeights", "NestedWeights", "lib", "library_path",
     "mq_plane_bytes", "mq_scale_bytes", "mq_pack", "mq_slice", "mq_gemm",
     "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
-    "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_MMA", "GEMV_SIMT",
+    "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -99,7 +99,7 @@ def mq_gemm_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
     return lib.mq_gemm_workspace_bytes(M, N, K, r)
 
 
-GEMV_MMA, GEMV_SIMT = 0, 1
+GEMV_TC, GEMV_VIA_GEMM = 0, 1
 
 
 def mq_set_gemv_variant(variant: int) -> None:
@@ -115,8 +115,9 @@ def mq_version() -> str:
 
 
 def mq_pack(codes, scales, planes_out, scales_out, stream=None) -> None:
-    """codes uint8 [N, K], scales fp32 [N, K/128] -> planes_out (>= 8 planes
-    of uint32 words), scales_out (fp16 or int16 [N, K/128]); all on device."""
+    """codes uint8 [N, K], scales fp32 [N, K/128] -> planes_out (the 8 tiled
+    planes, mq_plane_bytes(N, K, 8) bytes), scales_out (fp16 in the tiled
+    block order, mq_scale_bytes(N, K) bytes); all on device."""
     N, K = codes.shape
     _check(lib.mq_pack(codes.data_ptr(), scales.data_ptr(), N, K, 128,
                        planes_out.data_ptr(), scales_out.data_ptr(), _stream(stream)))
@@ -159,7 +160,7 @@ def pack_parent(codes, scales, stream=None) -> NestedWeights:
     import torch
     N, K = codes.shape
     planes = torch.empty(mq_plane_bytes(N, K, 8) // 4, dtype=torch.int32, device=codes.device)
-    s16 = torch.empty((N, K // 128), dtype=torch.float16, device=codes.device)
+    s16 = torch.empty(mq_scale_bytes(N, K, 128) // 2, dtype=torch.float16, device=codes.device)
     mq_pack(codes, scales, planes, s16, stream)
     return NestedWeights(planes, s16, N, K)
 

@@ -9,7 +9,7 @@
 namespace mq {
 
 static thread_local mq_status g_last = MQ_OK;
-static int g_gemv_variant = MQ_GEMV_MMA;   // process-wide kernel choice for M <= 8
+static int g_gemv_variant = MQ_GEMV_TC;    // process-wide kernel choice for M <= 8
 static thread_local char g_msg[512] = "no error";
 
 void set_error(mq_status s, const char *fmt, ...) {
@@ -81,6 +81,14 @@ mq_status check_weights(const mq_weights *w, int64_t N, int64_t K) {
     return MQ_OK;
 }
 
+mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
+                         void *ws, size_t ws_bytes, cudaStream_t st) {
+    if (__atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) == MQ_GEMV_TC &&
+        gemv_tc_supported(M, w->N, w->K, w->r))
+        return launch_gemv_tc(X, w, M, Y, ws, ws_bytes, st);
+    return launch_gemm_tc(X, w, M, Y, ws, ws_bytes, st);
+}
+
 }  // namespace mq
 
 using namespace mq;
@@ -89,12 +97,12 @@ extern "C" {
 
 size_t mq_plane_bytes(int64_t N, int64_t K, int r) {
     if (N < 1 || K < kGroup || K % kGroup || r < 1 || r > 8) return 0;
-    return (size_t)r * (size_t)N * (size_t)K / 8;
+    return (size_t)r * (size_t)((N + 127) / 128 * 128) * (size_t)K / 8;
 }
 
 size_t mq_scale_bytes(int64_t N, int64_t K, int group) {
     if (N < 1 || K < kGroup || K % kGroup || group != kGroup) return 0;
-    return 2 * (size_t)N * (size_t)(K / group);
+    return 2 * (size_t)((N + 127) / 128 * 128) * (size_t)(K / group);
 }
 
 mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out) {
@@ -112,7 +120,7 @@ mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out) {
 size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
     if (M < 1 || N < 1 || K < kGroup || K % kGroup || r < 1 || r > 8) return 0;
     if (M <= kGemvMaxM) {
-        const size_t a = gemv_workspace_bytes(M, N, K, r), b = gemv_mma_workspace_bytes(M, N, K, r);
+        const size_t a = gemv_tc_workspace_bytes(M, N, K, r), b = gemm_tc_workspace_bytes(M, N, K, r);
         return a > b ? a : b;
     }
     return gemm_tc_workspace_bytes(M, N, K, r);
@@ -133,16 +141,12 @@ mq_status mq_gemm(const uint16_t *X, const mq_weights *w, int64_t M, int64_t N,
         return fail(MQ_ERR_WORKSPACE, "workspace smaller than mq_gemm_workspace_bytes");
     cudaStream_t st = (cudaStream_t)stream;
     if ((s = bind_device(st)) != MQ_OK) return s;
-    if (M <= kGemvMaxM) {
-        if (__atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) == MQ_GEMV_SIMT)
-            return launch_gemv(X, w, M, Y, workspace, workspace_bytes, st);
-        return launch_gemv_mma(X, w, M, Y, workspace, workspace_bytes, st);
-    }
+    if (M <= kGemvMaxM) return launch_small_m(X, w, M, Y, workspace, workspace_bytes, st);
     return launch_gemm_tc(X, w, M, Y, workspace, workspace_bytes, st);
 }
 
 mq_status mq_set_gemv_variant(int variant) {
-    if (variant != MQ_GEMV_MMA && variant != MQ_GEMV_SIMT)
+    if (variant != MQ_GEMV_TC && variant != MQ_GEMV_VIA_GEMM)
         return fail(MQ_ERR_INVALID_ARG, "unknown GEMV variant");
     __atomic_store_n(&g_gemv_variant, variant, __ATOMIC_RELAXED);
     return MQ_OK;

@@ -37,17 +37,18 @@ mq_status bind_device(cudaStream_t st);
 mq_status check_weights(const mq_weights *w, int64_t N, int64_t K);
 
 // Kernel launchers (each returns MQ_OK or MQ_ERR_CUDA after the launch).
-size_t gemv_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
-mq_status launch_gemv(const uint16_t *X, const mq_weights *w, int64_t M,
-                      uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
-size_t gemv_mma_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
-mq_status launch_gemv_mma(const uint16_t *X, const mq_weights *w, int64_t M,
-                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
+bool gemv_tc_supported(int64_t M, int64_t N, int64_t K, int r);
+size_t gemv_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
+mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M,
+                         uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M,
                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
+// The M <= 8 product with the kernel chosen by mq_set_gemv_variant.
+mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M,
+                         uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
 
-// Largest M served by the CUDA-core GEMV; larger M runs the tcgen05 GEMM.
+// Largest M served by the GEMV kernels; larger M runs the tcgen05 GEMM.
 constexpr int kGemvMaxM = 8;
 
 }  // namespace mq

@@ -116,9 +116,8 @@ gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ pla
     constexpr int kCols = BM < 32 ? 32 : BM;                // TMEM columns (power of 2)
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTileN, BM);
     extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // 1024-byte aligned operand tiles: A = 2 x (128 rows x 128 B), B = 2 x (BM x 128 B)
-    uint8_t *base = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    // align the base by an offset so the compiler keeps the shared address space
+    uint8_t *base = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     uint8_t *sA = base;
     uint8_t *sB = base + 2 * kTileN * 128;
     __shared__ uint64_t bar;
@@ -141,7 +140,7 @@ gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ pla
 
     const int64_t n = n0 + t;
     const bool row_ok = n < N;
-    const int64_t plane_words = N * (K / 32);
+    const int64_t plane_words = (N + 127) / 128 * 128 * (K / 32);   // tiled planes
     float y[BM];
 #pragma unroll
     for (int c = 0; c < BM; ++c) y[c] = 0.f;
@@ -153,10 +152,9 @@ gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ pla
         uint4 pv[R];
 #pragma unroll
         for (int p = 0; p < R; ++p)
-            pv[p] = row_ok ? *reinterpret_cast<const uint4 *>(planes + p * plane_words +
-                                                              n * (K / 32) + g * 4)
-                           : make_uint4(0, 0, 0, 0);
-        const float s = row_ok ? __half2float(scales[n * G + g]) : 0.f;
+            pv[p] = *reinterpret_cast<const uint4 *>(planes + p * plane_words +
+                                                     ((int64_t)blockIdx.x * G + g) * 512 + t * 4);
+        const float s = __half2float(scales[((int64_t)blockIdx.x * G + g) * 128 + t]);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             uint32_t P[8], E[8];

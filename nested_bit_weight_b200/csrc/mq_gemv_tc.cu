@@ -1,0 +1,946 @@
+// Batch M <= 8: the nested r-bit product on the tcgen05 tensor cores, with the
+// decoded weights as the MMA's A operand in tensor memory.
+//
+// The r-bit model is the first r bit planes of the parent ("MatGPTQ:
+// Efficient and Accurate Inference over Nested Quantized Models", abstract:
+// an r-bit model reads exactly r bits); its level is
+//     v_r(q) = 2^(8-r) q + 2^(7-r) - 128,   w = s_g v_r(q),
+// so per 128-column group g and batch row m
+//     sum_k x_k w_k = s_g ( 2^(8-r) sum_k x_k q_k + (2^(7-r) - 128) S_g ),
+// with S_g = sum_k x_k.  The tensor core computes sum_k x_k q_k exactly:
+//
+// * A (M = 128 weight rows x K = 128 columns of one group, unsigned 8-bit, in
+//   TMEM).  Each thread of a 4-warp team owns one row: it reads the row's r
+//   plane words of the group (16 bytes per plane), turns every 32-column word
+//   into 8 registers whose bytes are fields q << sh(i) (one AND per register,
+//   sh = the field's bit offset in its byte), and stores the 32 registers to
+//   its TMEM lane with one tcgen05.st.  Byte b of register i of word t is
+//   column 32t + 8b + i; TMEM column 8t + i holds it, so A's k = 32t + 4i + b.
+// * B (N = 16 or 32 columns = 4 slices x M batch rows, signed 8-bit, shared
+//   memory, K-major, 128-byte swizzle).  z_k = x_k 2^(-sh(k)) is cut into
+//   four int8 slices relative to the group exponent Eg = max floor(log2|z|):
+//       z_k = 2^(Eg-27) (a_1 2^21 + a_2 2^14 + a_3 2^7 + a_4),
+//   exact for every x within 2^-14 of the group's largest; column 4m + j at
+//   k = 32t + 4i + b holds slice j of z at column 32t + 8b + i.
+// * D (128 x N, int32, TMEM) = exact per-group integer sums, read back with
+//   tcgen05.ld and folded into fp32: y += s_g 2^(8-r) 2^(Eg-6) sum_j 2^(-7j) D_j
+//   + s_g (2^(7-r) - 128) S_g.
+//
+// Work: the (128-row tile, group) items in tile order are cut into one
+// contiguous range per CTA (stream-K; shapes whose X operands do not fit in
+// shared memory are left to the GEMM).  The packed format stores the
+// 2 KB block of one (tile, group) contiguously per plane, items in this order,
+// so a run of items is one contiguous stream per plane: a producer warp copies
+// batches of items with bulk asynchronous copies into a ring of stages.  Two
+// teams of four warps take items in turn, each double-buffering A and D in
+// TMEM so that decoding the next item overlaps the tensor core and the
+// read-back of the previous one.  Partial sums of a tile are combined in a
+// fixed order; a tile shared with other CTAs goes through the workspace, the
+// last CTA to arrive summing every part in a fixed order.
+#include <string.h>
+
+#include "mq_common.cuh"
+#include "mq_bits.cuh"
+
+namespace mq {
+namespace {
+
+constexpr int kTeams = 3;                    // teams of 4 warps (128 rows)
+constexpr int kCW = 4 * kTeams;              // consumer warps
+constexpr int kProd = kCW, kMma = kCW + 1;   // producer warp, MMA-issuing warp
+constexpr int kThreads = (kCW + 2) * 32;
+constexpr int kBatch = 2 * kTeams;           // items per bulk copy: one pair per team
+constexpr int kSlices = 4;                   // int8 slices per x
+constexpr int kHeadBatches = 2;              // batches streamed before X is requested
+constexpr uint32_t kTmemCols = 512;          // TMEM columns per CTA (one CTA per SM)
+constexpr size_t kSmemMax = 227 * 1024;      // shared memory of one CTA per SM
+constexpr uint64_t kWaitNs = 1000000000ull;  // bound on any wait (1 s)
+
+// ------------------------------------------------------------ operand decode
+// Bit offset of register i's field inside each byte (the byte holds q << sh).
+template <int R> __host__ __device__ constexpr int field_shift(int i) {
+    return R == 1 ? i
+         : R == 2 ? 2 * (i >> 1)
+         : R == 3 ? 4 * (i >> 2) + 1
+         : R == 4 ? 4 * (i >> 2)
+                  : 8 - R;
+}
+
+// P[p] = plane p's word (planes >= R are 0) -> A[i]: byte b = field of column
+// 8b + i, shifted by field_shift<R>(i).
+template <int R>
+__device__ __forceinline__ void field_operands(const uint32_t (&P)[8], uint32_t *A) {
+    if constexpr (R == 1) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) A[i] = P[0] & (0x01010101u << i);
+    } else if constexpr (R == 2) {
+        const uint32_t e = pair_even(P[0], P[1]), o = pair_odd(P[0], P[1]);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+            A[2 * s] = e & (0x03030303u << (2 * s));
+            A[2 * s + 1] = o & (0x03030303u << (2 * s));
+        }
+    } else if constexpr (R <= 4) {
+        uint32_t Nw[4];
+        nibble_words<R>(P, 0, Nw);
+#pragma unroll
+        for (int d = 0; d < 4; ++d) {
+            A[d] = Nw[d] & 0x0F0F0F0Fu;
+            A[4 + d] = Nw[d] & 0xF0F0F0F0u;
+        }
+    } else {
+        uint32_t B8[8];
+        byte_words<R>(P, B8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) A[i] = B8[i];
+    }
+}
+
+// ------------------------------------------------------ barriers and copies
+__device__ unsigned int g_gemv_timeout;     // set when a bounded wait gave up
+
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void bar_init(uint64_t *b, uint32_t n) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(b)), "r"(n));
+}
+__device__ __forceinline__ void bar_expect(uint64_t *b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_addr(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint64_t *b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(b)) : "memory");
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ bool bar_try(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(ok) : "r"(smem_addr(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Wait for the phase of parity `parity` to complete by polling (a suspended
+// try_wait can resume well after the phase completes, which the per-item
+// hand-offs of this kernel cannot afford); gives up after about a second
+// (returns false) so that a lost copy cannot hang the GPU.
+__device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) {
+    if (bar_try(b, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!bar_try(b, parity))
+        if (global_ns() - t0 > kWaitNs) return false;
+    return true;
+}
+__device__ __forceinline__ void st_release(int *p, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+// Bulk copy of `bytes` contiguous bytes (16-byte aligned, multiple of 16).
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *b) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(b)) : "memory");
+}
+// Arrival ticket: acquire-release add at GPU scope, returns the old value.
+__device__ __forceinline__ unsigned ticket_add(unsigned *p) {
+    unsigned old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+    return old;
+}
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// ------------------------------------------------------------------ tcgen05
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// 32 lanes (this warp's quarter) x 32 columns of 32 bits from registers.
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t *v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+          "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+          "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]),
+          "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+          "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 32 lanes x 4 / 8 / 16 / 32 columns of 32 bits into registers.
+__device__ __forceinline__ void tmem_ld4(uint32_t taddr, int *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]) : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, int *v) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+                   "=r"(v[7])
+                 : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, int *v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, int *v) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] (128 x 32, u8) * B[smem]^T (N x 32, s8), int32 D; one thread.
+__device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+// Arrive on `bar` once the MMAs this thread issued before have completed.
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_addr(bar)) : "memory");
+}
+// Shared-memory descriptor of a K-major operand in the 128-byte swizzle
+// layout: 128-byte rows, 8-row atoms of 1024 bytes (stride 1024), atoms
+// 1024-byte aligned; the start address may step by 32 bytes inside a row.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);           // start address
+    d |= (uint64_t)1 << 16;                             // leading byte offset (unused)
+    d |= (uint64_t)(1024 >> 4) << 32;                   // stride byte offset
+    d |= (uint64_t)1 << 46;                             // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;                             // 128-byte swizzle
+    return d;
+}
+// Instruction descriptor: unsigned 8-bit A, signed 8-bit B (both K-major),
+// int32 D, shape 128 x N.
+__host__ __device__ constexpr uint32_t idesc_u8s8(int N) {
+    return (2u << 4)                      // D format: s32
+         | (0u << 7)                      // A format: unsigned 8-bit
+         | (1u << 10)                     // B format: signed 8-bit
+         | ((uint32_t)(N >> 3) << 17)     // N / 8
+         | ((uint32_t)(128 >> 4) << 24);  // M / 16
+}
+
+// ------------------------------------------------------------ decomposition
+// Items u = 0 .. W-1, W = T * KC (T 128-row tiles, KC = K / 128 groups), in
+// (tile, group) order; CTA b owns the contiguous items [first(b), first(b+1)).
+struct Work {
+    int64_t T, KC, W, C;
+    __host__ __device__ int64_t first(int64_t b) const { return b * W / C; }
+    __host__ __device__ int64_t cta_of(int64_t u) const { return ((u + 1) * C - 1) / W; }
+};
+
+struct Range { int u0, u1, L; };
+__host__ __device__ inline Range make_range(const Work &w, int64_t b) {
+    Range r;
+    r.u0 = (int)w.first(b);
+    r.u1 = (int)w.first(b + 1);
+    r.L = r.u1 - r.u0;
+    return r;
+}
+// Group held by X slot `slot` of the CTA (slots count groups from the group
+// of the CTA's first item, modulo KC).
+__host__ __device__ inline int slot_chunk(const Work &w, const Range &r, int slot) {
+    const int KC = (int)w.KC;
+    const int c = r.u0 % KC + slot;
+    return c >= KC ? c - KC : c;
+}
+
+// Kernel arguments (one struct, passed as a grid constant).
+struct Args {
+    const __nv_bfloat16 *X;
+    const uint8_t *planes;  // tiled planes (2 KB per (tile, group) block per plane)
+    const uint8_t *scales;  // tiled fp16 scales (256 B per block)
+    __nv_bfloat16 *Y;
+    float *part;            // [T][G][M][128] partial sums of shared tiles
+    unsigned *tickets;      // [T] arrivals at shared tiles (zero between calls)
+    Work w;
+    int64_t N, K, G;
+    int64_t plane_bytes;    // bytes of one plane
+    int M, NB, S;           // batch rows, MMA N (16 or 32), ring stages (multiple of kBatch)
+    // shared-memory offsets from the 1024-byte aligned base
+    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_run, o_coff, o_misc;
+};
+
+// ------------------------------------------------------------- X operand
+// Fixed-point value F = z 2^(27 - Ez), z = x 2^(-sh), truncated toward zero;
+// x is given by its bf16 bits (zero and subnormal inputs give 0).
+__device__ __forceinline__ int fixed_point(uint32_t h, int sh, int Ez) {
+    const int e8 = (int)((h >> 7) & 0xFFu);
+    const int mant = (int)((h & 0x7Fu) | 0x80u);
+    const int sft = e8 - 107 - sh - Ez;                  // <= 20 for finite x
+    int mag = sft >= 0 ? (mant << sft) : (sft > -9 ? (mant >> -sft) : 0);
+    if (e8 == 0) mag = 0;
+    return (h & 0x8000u) ? -mag : mag;
+}
+
+// Low bytes of four values -> one word (byte b from v_b).
+__device__ __forceinline__ uint32_t pack_bytes(int v0, int v1, int v2, int v3) {
+    const uint32_t lo = __byte_perm((uint32_t)v0, (uint32_t)v1, 0x0040);
+    const uint32_t hi = __byte_perm((uint32_t)v2, (uint32_t)v3, 0x0040);
+    return __byte_perm(lo, hi, 0x5410);
+}
+
+// X operand of the CTA's groups, built by the team warps.  Slot sl (the
+// sl-th distinct group of the range) lives in B tile sl / gpb at position
+// pos = sl % gpb (gpb = groups per tile): MMA column 4 (pos M + m) + j holds
+// slice j of batch row m, K-major with the 128-byte swizzle; the pair
+// {2^(8-r) 2^(Eg-6), S_g} of (slot, m) at pairs[sl * 8 + m].  X is staged
+// first with one round of 16-byte copies (staging[sl][m][128 values]).
+template <int R>
+__device__ void build_x_operand(const Args &a, uint8_t *smem, const Work &w, const Range &rg,
+                                int nslot, int *flags) {
+    constexpr int kPrep = kCW * 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int M = a.M, gpb = a.NB == 16 ? (M == 1 ? 4 : M == 2 ? 2 : 1) : 1;
+    const int t = lane >> 3, wi = lane & 7;
+    const int sh = field_shift<R>(wi);
+    float2 *pairs = reinterpret_cast<float2 *>(smem + a.o_pair);
+    // the warp's tasks (slot, m) in chunks of 4: all loads of a chunk first
+    const uint16_t *X = reinterpret_cast<const uint16_t *>(a.X);
+    for (int t0 = warp; t0 < nslot * M; t0 += 4 * kCW) {
+        uint32_t hv[4][4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int task = t0 + c * kCW;
+            if (task < nslot * M) {
+                const int sl = task / M, m = task - sl * M;
+                const uint16_t *xr = X + (int64_t)m * a.K + (int64_t)slot_chunk(w, rg, sl) * kGroup + 32 * t + wi;
+#pragma unroll
+                for (int b = 0; b < 4; ++b) hv[c][b] = xr[8 * b];
+            }
+        }
+        if (t0 == 0 && lane == 0) st_release(&flags[2], (int)(hv[0][0] | 1u));   // X fetched: stream the rest
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int task = t0 + c * kCW;
+            if (task >= nslot * M) break;
+            const int sl = task / M, m = task - sl * M;
+            uint32_t h[4];
+            int emax = -1000;
+            float sum = 0.f;
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                h[b] = hv[c][b];
+                const int e8 = (int)((h[b] >> 7) & 0xFFu);
+                const int v = e8 ? e8 - sh : -1000;
+                emax = v > emax ? v : emax;
+                sum += __uint_as_float(h[b] << 16);
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) {
+                const int other = __shfl_xor_sync(0xffffffffu, emax, o);
+                emax = other > emax ? other : emax;
+                sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            }
+            const int Eg = emax > -1000 ? emax - 127 : 0;
+            int F[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) F[b] = fixed_point(h[b], sh, Eg);
+            uint32_t wd[kSlices];
+            wd[0] = pack_bytes(F[0] >> 21, F[1] >> 21, F[2] >> 21, F[3] >> 21);
+            wd[1] = pack_bytes(F[0] >> 14, F[1] >> 14, F[2] >> 14, F[3] >> 14) & 0x7F7F7F7Fu;
+            wd[2] = pack_bytes(F[0] >> 7, F[1] >> 7, F[2] >> 7, F[3] >> 7) & 0x7F7F7F7Fu;
+            wd[3] = pack_bytes(F[0], F[1], F[2], F[3]) & 0x7F7F7F7Fu;
+            uint8_t *tile = smem + a.o_b + (size_t)(sl / gpb) * a.NB * 128;
+            const int chunk = 2 * t + (wi >> 2);               // 16-byte chunk of k = 32t + 4wi
+#pragma unroll
+            for (int j = 0; j < kSlices; ++j) {
+                const int row = 4 * ((sl % gpb) * M + m) + j;
+                *reinterpret_cast<uint32_t *>(tile + (row >> 3) * 1024 + (row & 7) * 128 +
+                                              ((chunk ^ (row & 7)) << 4) + 4 * (wi & 3)) = wd[j];
+            }
+            if (lane == 0) {
+                // 2^(8-r) 2^(Eg-6), clamped to the normal fp32 range
+                int ex = 2 - R + Eg;
+                ex = ex < -126 ? -126 : (ex > 127 ? 127 : ex);
+                pairs[sl * 8 + m] = make_float2(__int_as_float((ex + 127) << 23), sum);
+            }
+        }
+    }
+    // the tensor core reads B through the async proxy
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    named_sync(1, kPrep);
+}
+
+// ------------------------------------------------------------------ kernel
+// D columns of one item (4 slices per batch row, 4 MT registers) into registers.
+template <int MT>
+__device__ __forceinline__ void read_d(uint32_t taddr, int *d) {
+    if constexpr (MT == 1) tmem_ld4(taddr, d);
+    else if constexpr (MT == 2) tmem_ld8(taddr, d);
+    else if constexpr (MT == 4) tmem_ld16(taddr, d);
+    else tmem_ld32(taddr, d);
+}
+
+// Fold one item's D into y (row `row` of the team's current tile); on a tile
+// change the finished tile's sums go to res first.
+#define FOLD_ITEM(D, SC, SLOT, LTILE)                                                      \
+    do {                                                                                   \
+        if ((LTILE) != cur) {                                                              \
+            if (cur >= 0) {                                                                \
+                _Pragma("unroll") for (int m = 0; m < MT; ++m) if (m < M)                  \
+                    res[((team * ntile + cur) * M + m) * 128 + row] = y[m];                \
+            }                                                                              \
+            _Pragma("unroll") for (int m = 0; m < MT; ++m) y[m] = 0.f;                     \
+            cur = (LTILE);                                                                 \
+        }                                                                                  \
+        _Pragma("unroll") for (int m = 0; m < MT; ++m) {                                   \
+            if (m < M) {                                                                   \
+                const float v = (float)(D)[4 * m] + 0x1p-7f * (float)(D)[4 * m + 1] +      \
+                                0x1p-14f * (float)(D)[4 * m + 2] +                         \
+                                0x1p-21f * (float)(D)[4 * m + 3];                          \
+                const float2 ge = pairs[(SLOT) * 8 + m];                                   \
+                y[m] = fmaf((SC) * ge.x, v, fmaf((SC) * kOffset, ge.y, y[m]));             \
+            }                                                                              \
+        }                                                                                  \
+    } while (0)
+
+// MT: batch class (M = 1, M = 2, M <= 4, M <= 8), fixing the MMA N (16 or 32)
+// and the D columns read back per item.
+template <int R, int MT>
+__global__ void __launch_bounds__(kThreads, 1)
+nested_gemv_tc_kernel(const __grid_constant__ Args a) {
+    constexpr uint32_t kPlaneBlk = 2048;                // one (tile, group) block of one plane
+    extern __shared__ uint8_t smem_raw[];
+    // align the base by an offset so the compiler keeps the shared address space
+    uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
+    const Work &w = a.w;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const Range rg = make_range(w, blockIdx.x);
+    const int L = rg.L, S = a.S, M = a.M, G = (int)a.G;
+    const int nbs = S / kBatch;                          // batch slots in the ring
+    const int nbatch = (L + kBatch - 1) / kBatch;
+    const int64_t tf = rg.u0 / G;                        // first tile of the range
+    const int ntile = (int)((rg.u1 - 1) / G - tf + 1);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.o_bar);
+    uint64_t *empty = full + nbs;
+    uint64_t *aready = empty + nbs;                      // [team]: the pair's A stored (4 warps)
+    uint64_t *dfull = aready + kTeams;                   // [team]: the pair's MMAs done
+    uint64_t *mdone = dfull + kTeams;                    // every MMA of the CTA done
+    int2 *runinfo = reinterpret_cast<int2 *>(smem + a.o_run);   // [tile]: (tile, last arrival)
+    int *coff = reinterpret_cast<int *>(smem + a.o_coff);        // first group of each contributor
+    int *flags = reinterpret_cast<int *>(smem + a.o_misc);   // [0] error [1] batches issued [2] X asked
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + a.o_misc + 16);
+    float *res = reinterpret_cast<float *>(smem + a.o_res);  // [team][tile][m][128]
+    const int nslot = (int)(L < G ? L : G);
+
+    // a batch of 4 items = one pair per team; each team warp frees it once
+    if (threadIdx.x < 2 * nbs) bar_init(full + threadIdx.x, threadIdx.x < nbs ? 1u : 4u * kTeams);
+    if (threadIdx.x < 2 * kTeams + 1) bar_init(aready + threadIdx.x, threadIdx.x < kTeams ? 4u : 1u);
+    if (threadIdx.x == 0) { flags[0] = 0; flags[1] = 0; flags[2] = 0; }
+    for (int i = threadIdx.x; i < kTeams * ntile * M * 128; i += kThreads) res[i] = 0.f;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+
+    if (warp == kProd) {
+        // ---------------------------------------------------------- producer
+        // batch b = items [4b, 4b + 4): one bulk copy per plane and one for the
+        // scales (consecutive items are consecutive blocks), into ring slot b % nbs
+        if (lane == 0) {
+            bool ok = true;
+            for (int b = 0; b < nbatch && ok; ++b) {
+                if (b == kHeadBatches) {
+                    // the next call may start; and X should not queue behind the rest
+                    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire(&flags[2]) == 0 && ok) {
+                        if (global_ns() - t0 > kWaitNs) ok = false;
+                        __nanosleep(128);
+                    }
+                    if (!ok) break;
+                }
+                const int bs = b % nbs;
+                if (b >= nbs && !bar_wait(empty + bs, (uint32_t)((b / nbs) - 1) & 1u)) { ok = false; break; }
+                const int i0 = b * kBatch, n = (L - i0) < kBatch ? (L - i0) : kBatch;
+                const int64_t u = rg.u0 + i0;
+                bar_expect(full + bs, (uint32_t)n * (kPlaneBlk * R + 256));
+#pragma unroll
+                for (int p = 0; p < R; ++p)
+                    bulk_g2s(smem + a.o_ring + ((size_t)p * S + (size_t)bs * kBatch) * kPlaneBlk,
+                             a.planes + p * a.plane_bytes + u * kPlaneBlk, (uint32_t)n * kPlaneBlk, full + bs);
+                bulk_g2s(smem + a.o_sring + (size_t)bs * kBatch * 256, a.scales + u * 256,
+                         (uint32_t)n * 256, full + bs);
+                st_release(&flags[1], b + 1);
+            }
+            if (nbatch <= kHeadBatches) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+            if (!ok) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
+        }
+    } else if (warp == kMma) {
+        // ------------------------------------------------------- MMA issue
+        // Pair jj of team t = items kBatch jj + 2 t and kBatch jj + 2 t + 1 (one ring
+        // batch).  Once the team has stored the pair's A, for each item e:
+        // D[t][e] = A[t][e] . B(X slot of the item)^T, K = 128 in 4 steps.
+        if (lane == 0) {
+            const uint32_t idesc = idesc_u8s8(a.NB);
+            constexpr int gsh = MT == 1 ? 2 : MT == 2 ? 1 : 0;   // log2 groups per B tile
+            const uint32_t b0 = smem_addr(smem + a.o_b);
+            bool ok = true;
+            uint32_t tmem = 0;
+            int nxt[kTeams], np[kTeams], xs[kTeams];   // next pair, pairs, X slot of its item 0
+#pragma unroll
+            for (int t = 0; t < kTeams; ++t) {
+                nxt[t] = 0;
+                np[t] = 2 * t < L ? (L - 2 * t + kBatch - 1) / kBatch : 0;
+                xs[t] = 2 * t;
+                while (xs[t] >= G) xs[t] -= G;
+            }
+            // serve whichever team has stored its next pair (teams run independently)
+            uint64_t last = global_ns();
+            while (ok) {
+                bool pending = false, progress = false;
+#pragma unroll
+                for (int t = 0; t < kTeams; ++t) {
+                    if (nxt[t] >= np[t]) continue;
+                    pending = true;
+                    if (!bar_try(aready + t, (uint32_t)(nxt[t] & 1))) continue;
+                    tc_fence_after();
+                    if (!tmem) tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+                    const int i0 = kBatch * nxt[t] + 2 * t;
+                    const uint32_t col0 = tmem + (uint32_t)t * 128;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        if (i0 + e >= L) break;
+                        const int sl = xs[t] + e >= G ? xs[t] + e - G : xs[t] + e;
+                        const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_i8_ts(col0 + 64 + (uint32_t)(e * a.NB), col0 + 32 * e + 8 * kk,
+                                      smem_desc_sw128(baddr + 32 * kk), idesc, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(dfull + t);
+                    ++nxt[t];
+                    xs[t] += kBatch;
+                    while (xs[t] >= G) xs[t] -= G;
+                    progress = true;
+                }
+                if (!pending) break;
+                const uint64_t now = global_ns();
+                if (progress) last = now;
+                else if (now - last > kWaitNs) ok = false;
+            }
+            // TMEM may be freed only after every issued MMA has completed
+            mma_commit(mdone);
+            if (!bar_wait(mdone, 0u)) ok = false;
+            if (!ok) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
+        }
+    } else if (warp < kCW) {
+        // ------------------------------------------------------------- teams
+        // TMEM is taken here, off the producer's path; the MMA warp reads its
+        // address after the first A hand-off
+        if (warp == 0) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_addr(tmem_slot)), "r"(kTmemCols) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
+        tc_fence_before();
+        asm volatile("griddepcontrol.wait;" ::: "memory");      // X comes from the previous kernel
+        build_x_operand<R>(a, smem, w, rg, nslot, flags);       // ends with a team barrier
+        tc_fence_after();
+        const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+        const int team = warp >> 2, q = warp & 3, row = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const uint32_t col0 = tmem + (uint32_t)team * 128;       // A0 A1 at +0 +32, D0 D1 at +64 +64+NB
+        constexpr int gpb = MT <= 4 ? 4 / MT : 1;      // groups per B tile
+        const float2 *pairs = reinterpret_cast<const float2 *>(smem + a.o_pair);
+        constexpr float kOffset = (float)(128 >> (R - 1)) * 0.5f - 128.0f;   // 2^(7-r) - 128
+        float y[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) y[m] = 0.f;
+        int cur = -1;                                    // local tile of y
+        // Iteration jj decodes the team's pair jj (items i0 = kBatch jj + 2 team and
+        // i0 + 1) into registers, waits for the MMAs of pair jj - 1, stores
+        // the new A, reads the old D, and folds pair jj - 1.  Indices advance
+        // by kBatch items without divisions: ring stage, X slot, group and tile.
+        const int Jp = (L - 2 * team + kBatch - 1) / kBatch;   // pairs of this team
+        float sp[2] = {0.f, 0.f};                        // previous pair: scales, X slots, tiles
+        int slp[2] = {0, 0}, ltp[2] = {0, 0}, np = 0;
+        int st = 2 * team, fpar = 0;                     // ring stage of i0, parity of its fill
+        int xslot = 2 * team, g = rg.u0 % G + 2 * team, lt = 0;
+        while (xslot >= G) xslot -= G;
+        while (g >= G) { g -= G; ++lt; }
+        bool ok = true;
+        constexpr int ND = 4 * MT;                       // D columns read per item
+        for (int jj = 0; jj <= Jp; ++jj) {
+            const bool have = jj < Jp, back = jj > 0;
+            const int i0 = kBatch * jj + 2 * team;
+            const int n = have ? (i0 + 1 < L ? 2 : 1) : 0;   // items in this pair
+            uint32_t A0[32], A1[32];
+            float sc[2] = {0.f, 0.f};
+            if (have) {
+                const int bs = st / kBatch;              // ring slot of the batch
+                if (!__all_sync(0xffffffffu, bar_wait(full + bs, (uint32_t)fpar))) { ok = false; break; }
+                uint4 pw[R];
+#pragma unroll
+                for (int p = 0; p < R; ++p)
+                    pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st) * kPlaneBlk + row * 16);
+                sc[0] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)st * 256 + row * 2));
+#pragma unroll
+                for (int t4 = 0; t4 < 4; ++t4) {
+                    uint32_t P[8];
+#pragma unroll
+                    for (int p = 0; p < 8; ++p) {
+                        const uint4 &v = pw[p < R ? p : 0];
+                        P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
+                    }
+                    field_operands<R>(P, A0 + 8 * t4);
+                }
+                if (n == 2) {
+#pragma unroll
+                    for (int p = 0; p < R; ++p)
+                        pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st + 1) * kPlaneBlk + row * 16);
+                    sc[1] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)(st + 1) * 256 + row * 2));
+#pragma unroll
+                    for (int t4 = 0; t4 < 4; ++t4) {
+                        uint32_t P[8];
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            const uint4 &v = pw[p < R ? p : 0];
+                            P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
+                        }
+                        field_operands<R>(P, A1 + 8 * t4);
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) bar_arrive(empty + bs);
+            }
+            if (back) {
+                // the MMAs of pair jj - 1 are done: A is free and D holds their sums
+                if (!__all_sync(0xffffffffu, bar_wait(dfull + team, (uint32_t)((jj - 1) & 1)))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (have) {
+                tmem_st32(lane_base + col0, A0);
+                if (n == 2) tmem_st32(lane_base + col0 + 32, A1);
+            }
+            int d0[ND], d1[ND];
+            if (back) {
+                read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
+                if constexpr (MT <= 4) {
+                    if (np == 2) read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
+                    tmem_ld_wait();
+                } else {
+                    tmem_ld_wait();
+                    FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
+                    if (np == 2) {
+                        read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
+                        tmem_ld_wait();
+                    }
+                }
+            }
+            if (have) {
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(aready + team);
+            }
+            if (back) {
+                if constexpr (MT <= 4) FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
+                if (np == 2) FOLD_ITEM(d1, sp[1], slp[1], ltp[1]);
+            }
+            // this pair becomes the previous one; advance by kBatch items
+            np = n;
+            sp[0] = sc[0]; sp[1] = sc[1];
+            slp[0] = xslot; ltp[0] = lt;
+            slp[1] = xslot + 1 == G ? 0 : xslot + 1;
+            ltp[1] = g + 1 == G ? lt + 1 : lt;
+            st += kBatch;
+            if (st >= S) { st -= S; fpar ^= 1; }
+            xslot += kBatch;
+            while (xslot >= G) xslot -= G;
+            g += kBatch;
+            while (g >= G) { g -= G; ++lt; }
+        }
+        if (cur >= 0) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m)
+                if (m < M) res[((team * ntile + cur) * M + m) * 128 + row] = y[m];
+        }
+        if (!ok && lane == 0) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
+        named_sync(1, kCW * 32);
+        // ---- combine the teams per tile (fixed order) and write Y or the part
+        for (int idx = threadIdx.x; idx < ntile * M * 128; idx += kCW * 32) {
+            const int lt = idx / (M * 128), rem = idx - lt * M * 128, m = rem >> 7, rr = rem & 127;
+            float v = 0.f;
+#pragma unroll
+            for (int tm = 0; tm < kTeams; ++tm) v += res[((tm * ntile + lt) * M + m) * 128 + rr];
+            const int64_t t = tf + lt;
+            const int64_t ra = t * G, rb = ra + G;
+            const int64_t n = t * 128 + rr;
+            if (ra >= rg.u0 && rb <= rg.u1) {
+                if (n < a.N) a.Y[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
+            } else {
+                const int64_t kcf = (ra > rg.u0 ? ra : rg.u0) - ra;
+                a.part[((t * G + kcf) * M + m) * 128 + rr] = v;
+            }
+        }
+        named_sync(1, kCW * 32);
+        // ---- shared tiles: one arrival ticket per tile; the last CTA to
+        // arrive sums every part in a fixed order (contributing CTAs in
+        // increasing order) and writes Y.  The CTA barrier before the
+        // acquire-release ticket makes all of this CTA's parts visible with
+        // it; the barrier after it orders the last arriver's reads.
+        for (int lt = threadIdx.x; lt < ntile; lt += kCW * 32) {
+            const int64_t t = tf + lt, ra = t * G, rb = ra + G;
+            int last = 0;
+            if (ra < rg.u0 || rb > rg.u1) {
+                const unsigned nct = (unsigned)(w.cta_of(rb - 1) - w.cta_of(ra) + 1);
+                last = ticket_add(&a.tickets[t]) == nct - 1u;
+            }
+            runinfo[lt] = make_int2((int)t, last);
+        }
+        named_sync(1, kCW * 32);
+        for (int lt = 0; lt < ntile; ++lt) {
+            if (!runinfo[lt].y) continue;
+            const int64_t t = runinfo[lt].x, ra = t * G;
+            const int64_t c0 = w.cta_of(ra);
+            const int nc = (int)(w.cta_of(ra + G - 1) - c0 + 1);
+            for (int c = threadIdx.x; c < nc; c += kCW * 32) {
+                const int64_t f = w.first(c0 + c);
+                coff[c] = (int)((f > ra ? f : ra) - ra);
+            }
+            named_sync(1, kCW * 32);
+            const float *pt = a.part + t * G * M * 128;
+            for (int idx = threadIdx.x; idx < M * 128; idx += kCW * 32) {
+                float v = 0.f;
+                int c = 0;
+                for (; c + 4 <= nc; c += 4) {
+                    const float p0 = __ldcg(pt + (int64_t)coff[c] * M * 128 + idx);
+                    const float p1 = __ldcg(pt + (int64_t)coff[c + 1] * M * 128 + idx);
+                    const float p2 = __ldcg(pt + (int64_t)coff[c + 2] * M * 128 + idx);
+                    const float p3 = __ldcg(pt + (int64_t)coff[c + 3] * M * 128 + idx);
+                    v += p0;
+                    v += p1;
+                    v += p2;
+                    v += p3;
+                }
+                for (; c < nc; ++c) v += __ldcg(pt + (int64_t)coff[c] * M * 128 + idx);
+                const int64_t n = t * 128 + (idx & 127);
+                if (n < a.N) a.Y[(int64_t)(idx >> 7) * a.N + n] = __float2bfloat16_rn(v);
+            }
+            named_sync(1, kCW * 32);
+            if (threadIdx.x == 0) a.tickets[t] = 0u;
+        }
+    }
+
+    // after a timed-out wait, let the copies already issued land; then free TMEM
+    tc_fence_before();
+    __syncthreads();
+    if (flags[0] && threadIdx.x == 0) {
+        const int issued = flags[1];
+        for (int bs = 0; bs < nbs && bs < issued; ++bs) {
+            const int last = bs + ((issued - 1 - bs) / nbs) * nbs;
+            bar_wait(full + bs, (uint32_t)(last / nbs) & 1u);
+        }
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- host side
+struct Plan {
+    Work w;
+    int NB, S, nslot, L, ntile;
+    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_run, o_coff, o_misc;
+    size_t smem, part_off, ws_bytes;
+    bool ok;
+};
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+inline uint32_t align_up(size_t x, size_t a) { return (uint32_t)((x + a - 1) / a * a); }
+
+// Shared-memory layout for S stages; returns its size without slack.
+size_t layout(Plan &p, int r, int M, int S) {
+    const int gpb = p.NB == 16 ? (M == 1 ? 4 : M == 2 ? 2 : 1) : 1;
+    size_t o = 0;
+    p.o_ring = 0;
+    o = (size_t)r * S * 2048;
+    p.o_sring = align_up(o, 128);
+    o = p.o_sring + (size_t)S * 256;
+    p.o_b = align_up(o, 1024);
+    o = p.o_b + (size_t)((p.nslot + gpb - 1) / gpb) * p.NB * 128;
+    p.o_pair = align_up(o, 16);
+    o = p.o_pair + (size_t)p.nslot * 8 * 8;
+    p.o_res = align_up(o, 16);
+    o = p.o_res + (size_t)kTeams * p.ntile * M * 128 * 4;
+    p.o_bar = align_up(o, 16);
+    o = p.o_bar + (size_t)(2 * (S / kBatch) + 2 * kTeams + 1) * 8;
+    p.o_run = align_up(o, 16);
+    o = p.o_run + (size_t)p.ntile * 8;
+    p.o_coff = align_up(o, 16);
+    o = p.o_coff + (size_t)(p.w.C + 1) * 4;
+    p.o_misc = align_up(o, 16);
+    o = p.o_misc + 64;                                     // flags, TMEM address
+    return o;
+}
+
+Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
+    Plan p{};
+    const int64_t T = (N + 127) / 128, G = K / kGroup;
+    const int64_t W = T * G;
+    p.NB = M <= 4 ? 16 : 32;
+    const int64_t C = W < sm_count() ? W : sm_count();
+    const Work w{T, G, W, C};
+    int64_t L = 0, nt = 0;
+    for (int64_t b = 0; b < C; ++b) {
+        const int64_t u0 = w.first(b), u1 = w.first(b + 1);
+        if (u1 <= u0) continue;
+        L = u1 - u0 > L ? u1 - u0 : L;
+        const int64_t tt = (u1 - 1) / G - u0 / G + 1;
+        nt = tt > nt ? tt : nt;
+    }
+    p.w = w;
+    p.L = (int)L;
+    p.ntile = (int)nt;
+    p.nslot = (int)(L < G ? L : G);
+    const size_t stage = (size_t)2048 * r + 256;
+    const size_t fixed = layout(p, r, (int)M, 0);
+    const int need = (int)((L + kBatch - 1) / kBatch) * kBatch;   // stages for the whole range
+    const int want = need < 2 * kBatch ? need : 2 * kBatch;        // fewest stages accepted
+    p.part_off = kTicketBytes;
+    p.ws_bytes = p.part_off + (size_t)W * M * 128 * sizeof(float);
+    p.ok = false;
+    if (T > (int64_t)(kTicketBytes / sizeof(unsigned))) return p;
+    if (fixed + (size_t)want * stage + 1024 > kSmemMax) return p;
+    int S = (int)((kSmemMax - 1024 - fixed) / stage) / kBatch * kBatch;
+    if (S > need) S = need;
+    p.S = S;
+    p.smem = layout(p, r, (int)M, S) + 1024;
+    p.ok = true;
+    return p;
+}
+
+template <int R, int MT>
+mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, char *ws,
+              const Plan &p, cudaStream_t st) {
+    static bool attr_set = false;          // per instantiation
+    cudaError_t e;
+    if (!attr_set) {
+        e = cudaFuncSetAttribute(nested_gemv_tc_kernel<R, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemMax);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+        attr_set = true;
+    }
+    Args a{};
+    a.X = reinterpret_cast<const __nv_bfloat16 *>(X);
+    a.planes = reinterpret_cast<const uint8_t *>(wt->planes);
+    a.scales = reinterpret_cast<const uint8_t *>(wt->scales);
+    a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+    a.part = reinterpret_cast<float *>(ws + p.part_off);
+    a.tickets = reinterpret_cast<unsigned *>(ws);
+    a.w = p.w;
+    a.N = wt->N;
+    a.K = wt->K;
+    a.G = wt->K / kGroup;
+    a.plane_bytes = (int64_t)mq_plane_bytes(wt->N, wt->K, 1);
+    a.M = (int)M;
+    a.NB = p.NB;
+    a.S = p.S;
+    a.o_ring = p.o_ring; a.o_sring = p.o_sring; a.o_b = p.o_b; a.o_pair = p.o_pair;
+    a.o_res = p.o_res; a.o_bar = p.o_bar; a.o_run = p.o_run; a.o_coff = p.o_coff; a.o_misc = p.o_misc;
+    // programmatic dependent launch: this grid may start while the previous
+    // kernel of the stream finishes; it waits for it before reading X
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.w.C);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = p.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, nested_gemv_tc_kernel<R, MT>, a);
+    if (e != cudaSuccess) return cuda_fail(e, "nested_gemv_tc_kernel launch");
+    return MQ_OK;
+}
+
+template <int R>
+mq_status run_r(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, char *ws,
+                const Plan &p, cudaStream_t st) {
+    if (M == 1) return run<R, 1>(X, wt, M, Y, ws, p, st);
+    if (M == 2) return run<R, 2>(X, wt, M, Y, ws, p, st);
+    if (M <= 4) return run<R, 4>(X, wt, M, Y, ws, p, st);
+    return run<R, 8>(X, wt, M, Y, ws, p, st);
+}
+
+}  // namespace
+
+bool gemv_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
+    return M >= 1 && M <= kGemvMaxM && make_plan(M, N, K, r).ok;
+}
+
+size_t gemv_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
+    const Plan p = make_plan(M, N, K, r);
+    return p.ok ? p.ws_bytes : 0;
+}
+
+mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
+                         void *ws, size_t ws_bytes, cudaStream_t st) {
+    const Plan p = make_plan(M, w->N, w->K, w->r);
+    if (!p.ok) return fail(MQ_ERR_UNSUPPORTED, "no tensor-core GEMV plan fits this shape");
+    if (p.ws_bytes > ws_bytes) return fail(MQ_ERR_WORKSPACE, "GEMV workspace too small");
+    char *b = static_cast<char *>(ws);
+    switch (w->r) {
+        case 1: return run_r<1>(X, w, M, Y, b, p, st);
+        case 2: return run_r<2>(X, w, M, Y, b, p, st);
+        case 3: return run_r<3>(X, w, M, Y, b, p, st);
+        case 4: return run_r<4>(X, w, M, Y, b, p, st);
+        case 5: return run_r<5>(X, w, M, Y, b, p, st);
+        case 6: return run_r<6>(X, w, M, Y, b, p, st);
+        case 7: return run_r<7>(X, w, M, Y, b, p, st);
+        default: return run_r<8>(X, w, M, Y, b, p, st);
+    }
+}
+
+}  // namespace mq

@@ -57,7 +57,5 @@ extern "C" mq_status mq_gemv_noalloc(const uint16_t *X, const mq_weights *w, int
     // the arrival tickets must start at zero whatever an earlier call left
     e = cudaMemsetAsync(scratch, 0, kTicketBytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-    if (mq_get_gemv_variant() == MQ_GEMV_SIMT)
-        return launch_gemv(X, w, M, Y, scratch, kNoAllocBytes, st);
-    return launch_gemv_mma(X, w, M, Y, scratch, kNoAllocBytes, st);
+    return launch_small_m(X, w, M, Y, scratch, kNoAllocBytes, st);
 }

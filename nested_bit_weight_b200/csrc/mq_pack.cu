@@ -1,6 +1,12 @@
 // Bit-plane packer and its inverse (exact-r-bit storage of the MatGPTQ
 // abstract and Table 1, "Exact r-bit loading").
 //
+// Layout (include/mq.h): rows padded to a multiple of 128; each plane is a
+// sequence of 2 KB blocks, one per (128-row tile t, 128-column group g) in
+// t-major order; row i of a block is 4 words (16 bytes), bit j of word w
+// holding column 128g + 32w + j.  Scales use the same block order, 128
+// fp16 values per block.
+//
 // pack: a warp turns 32 consecutive codes of a row into one word of each of
 // the 8 planes with warp ballots (lane j votes bit j of its code).
 #include "mq_common.cuh"
@@ -18,7 +24,7 @@ pack_kernel(const uint8_t *__restrict__ codes, int64_t N, int64_t K,
     const int64_t W = K / 32;                        // words per plane row
     const int64_t blocks_per_row = (W + 31) / 32;
     const int64_t total = N * blocks_per_row;
-    const int64_t plane_words = N * W;
+    const int64_t plane_words = (N + 127) / 128 * 128 * W;
     int64_t warp = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     for (int64_t i = warp; i < total; i += nwarps) {
@@ -33,21 +39,23 @@ pack_kernel(const uint8_t *__restrict__ codes, int64_t N, int64_t K,
             }
         }
         if (w0 + lane < W) {
+            const int64_t w = w0 + lane;
+            const int64_t at = ((n / 128) * (W / 4) + w / 4) * 512 + (n % 128) * 4 + (w % 4);
 #pragma unroll
-            for (int p = 0; p < kPlanes; ++p)
-                planes[(int64_t)p * plane_words + n * W + w0 + lane] = mine[p];
+            for (int p = 0; p < kPlanes; ++p) planes[(int64_t)p * plane_words + at] = mine[p];
         }
     }
 }
 
 __global__ void __launch_bounds__(256)
-scales_kernel(const float *__restrict__ s, int64_t count, __half *__restrict__ out) {
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count;
+scales_kernel(const float *__restrict__ s, int64_t N, int64_t G, __half *__restrict__ out) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N * G;
          i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i / G, g = i - n * G;
         const float v = s[i];
         const __half h = __float2half_rn(v);
         if (!(v >= 0.0f) || __hisinf(h)) atomicOr(&g_pack_bad, 1u);
-        out[i] = h;
+        out[((n / 128) * G + g) * 128 + n % 128] = h;
     }
 }
 
@@ -56,11 +64,13 @@ __global__ void __launch_bounds__(256)
 unpack_kernel(const uint32_t *__restrict__ planes, int64_t N, int64_t K, int r,
               uint8_t *__restrict__ out) {
     const int64_t W = K / 32;
-    const int64_t plane_words = N * W;
+    const int64_t plane_words = (N + 127) / 128 * 128 * W;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N * W;
          i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t n = i / W, w = i - n * W;
+        const int64_t at = ((n / 128) * (W / 4) + w / 4) * 512 + (n % 128) * 4 + (w % 4);
         uint32_t P[kPlanes];
-        for (int p = 0; p < r; ++p) P[p] = planes[(int64_t)p * plane_words + i];
+        for (int p = 0; p < r; ++p) P[p] = planes[(int64_t)p * plane_words + at];
         uint32_t packed[8];
 #pragma unroll
         for (int b = 0; b < 8; ++b) {
@@ -108,10 +118,16 @@ extern "C" mq_status mq_pack(const uint8_t *codes, const float *scales, int64_t 
     cudaError_t e = cudaMemcpyToSymbolAsync(g_pack_bad, &zero, sizeof(zero), 0,
                                             cudaMemcpyHostToDevice, st);
     if (e != cudaSuccess) return cuda_fail(e, "mq_pack reset");
+    if (N % 128) {
+        // padding rows of the last tile: zero bits and zero scales
+        e = cudaMemsetAsync(planes_out, 0, mq_plane_bytes(N, K, 8), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(scales_out, 0, mq_scale_bytes(N, K, kGroup), st);
+        if (e != cudaSuccess) return cuda_fail(e, "mq_pack padding");
+    }
     pack_kernel<<<grid_for(N * ((K / 32 + 31) / 32) * 32, 256), 256, 0, st>>>(codes, N, K, planes_out);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pack_kernel");
     const int64_t ns = N * (K / kGroup);
-    scales_kernel<<<grid_for(ns, 256), 256, 0, st>>>(scales, ns,
+    scales_kernel<<<grid_for(ns, 256), 256, 0, st>>>(scales, N, K / kGroup,
                                                      reinterpret_cast<__half *>(scales_out));
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "scales_kernel");
     unsigned bad = 0;

@@ -52,11 +52,11 @@ def test_golden_samples_config0():
         assert oracle.violation_ratio(Y[0, g["columns"]], ref, rms) <= 1.0
 
 
-@pytest.fixture(params=["mma", "simt"])
+@pytest.fixture(params=["tc", "via_gemm"])
 def gemv_variant(request):
     import nested_bit_weight_b200 as mq
     old = mq.mq_get_gemv_variant()
-    mq.mq_set_gemv_variant(mq.GEMV_MMA if request.param == "mma" else mq.GEMV_SIMT)
+    mq.mq_set_gemv_variant(mq.GEMV_TC if request.param == "tc" else mq.GEMV_VIA_GEMM)
     yield request.param
     mq.mq_set_gemv_variant(old)
 

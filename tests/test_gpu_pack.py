@@ -23,15 +23,17 @@ KINDS = ("zeros", "ones", "alternating", "single_bit", "all_codes", "random")
 
 
 @pytest.mark.parametrize("kind", KINDS)
-@pytest.mark.parametrize("N,K", [(1, 128), (7, 384), (64, 512), (33, 1280)])
+@pytest.mark.parametrize("N,K", [(1, 128), (7, 384), (64, 512), (33, 1280), (130, 256),
+                                 (256, 384)])
 def test_pack_bit_exact(kind, N, K):
+    # whole buffers, padding rows included (they must be zero on both sides)
     codes = wl.adversarial_codes(kind, N, K, seed=N + K)
     s = wl.gen_scales(N, K, seed=N)
     w = _pack(codes, s)
-    got = w.planes.cpu().numpy().view(np.uint32).reshape(8, N, K // 32)
+    got = w.planes.cpu().numpy().view(np.uint32).reshape(8, -1)
     assert np.array_equal(got, oracle.pack(codes))
     s16 = w.scales16.cpu().numpy()
-    assert np.array_equal(s16.view(np.uint16), oracle.scales_f16(s).view(np.uint16))
+    assert np.array_equal(s16.view(np.uint16), oracle.scales_stored(s).view(np.uint16))
 
 
 @pytest.mark.parametrize("r", range(1, 9))
@@ -48,17 +50,15 @@ def test_unpack_bit_exact(r):
     assert np.array_equal(out.cpu().numpy(), oracle.slice_codes(codes, r))
 
 
-def test_pack_large_layer_sampled():
-    # full Llama gate/up size: compare a sample of plane rows with the oracle
+def test_pack_large_layer():
+    # full Llama gate/up size (14336 x 4096): every word against the C oracle
     N, K = 14336, 4096
     codes, s, _ = wl.gen_weights(N, K, seed=4)
     w = _pack(codes, s)
-    rows = np.random.default_rng(0).choice(N, 64, replace=False)
-    rows.sort()
-    got = w.planes.view(8, N, K // 32)[:, rows.tolist()].cpu().numpy().view(np.uint32)
-    assert np.array_equal(got, oracle.pack(codes[rows]))
+    got = w.planes.cpu().numpy().view(np.uint32).reshape(8, -1)
+    assert np.array_equal(got, oracle.pack(codes))
     assert np.array_equal(w.scales16.cpu().numpy().view(np.uint16),
-                          oracle.scales_f16(s).view(np.uint16))
+                          oracle.scales_stored(s).view(np.uint16))
 
 
 @pytest.mark.parametrize("bad", [-1.0, float("nan"), 1e6])
@@ -77,4 +77,4 @@ def test_pack_zero_scale_is_kept():
     s = wl.gen_scales(8, 256, seed=2, zero_groups=5)
     w = _pack(codes, s)
     assert np.array_equal(w.scales16.cpu().numpy().view(np.uint16),
-                          oracle.scales_f16(s).view(np.uint16))
+                          oracle.scales_stored(s).view(np.uint16))
