@@ -47,8 +47,8 @@ namespace {
 
 constexpr int kTeams = 3;                    // teams of 4 warps (128 rows)
 constexpr int kCW = 4 * kTeams;              // consumer warps
-constexpr int kProd = kCW, kMma = kCW + 1;   // producer warp, MMA-issuing warp
-constexpr int kThreads = (kCW + 2) * 32;
+constexpr int kProd = kCW;                   // producer warp
+constexpr int kThreads = (kCW + 1) * 32;
 constexpr int kBatch = 2 * kTeams;           // items per bulk copy: one pair per team
 constexpr int kSlices = 4;                   // int8 slices per x
 constexpr int kHeadBatches = 2;              // batches streamed before X is requested
@@ -129,6 +129,23 @@ __device__ __forceinline__ bool bar_try(uint64_t *b, uint32_t parity) {
 // try_wait can resume well after the phase completes, which the per-item
 // hand-offs of this kernel cannot afford); gives up after about a second
 // (returns false) so that a lost copy cannot hang the GPU.
+// Suspending variant for the producer, which waits long and is not on the
+// per-item critical path: the thread sleeps in try_wait instead of spinning
+// (spinning would take issue slots from the decoding warps).
+__device__ __forceinline__ bool bar_try_sleep(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 2000;\n"
+                 " selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(ok) : "r"(smem_addr(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool bar_wait_sleep(uint64_t *b, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!bar_try_sleep(b, parity))
+        if (global_ns() - t0 > kWaitNs) return false;
+    return true;
+}
 __device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) {
     if (bar_try(b, parity)) return true;
     const uint64_t t0 = global_ns();
@@ -158,6 +175,15 @@ __device__ __forceinline__ unsigned ticket_add(unsigned *p) {
 }
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Named barrier that also returns the AND of `v` over its threads, so that a
+// whole team takes the same branch after a wait that may have timed out.
+__device__ __forceinline__ bool named_sync_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 q, %2, 0;\n"
+                 " bar.red.and.pred p, %1, %3, q;\n selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(r) : "r"(id), "r"((uint32_t)v), "r"(n) : "memory");
+    return r != 0;
 }
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tc_fence_before() {
@@ -446,9 +472,7 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
     const int ntile = (int)((rg.u1 - 1) / G - tf + 1);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.o_bar);
     uint64_t *empty = full + nbs;
-    uint64_t *aready = empty + nbs;                      // [team]: the pair's A stored (4 warps)
-    uint64_t *dfull = aready + kTeams;                   // [team]: the pair's MMAs done
-    uint64_t *mdone = dfull + kTeams;                    // every MMA of the CTA done
+    uint64_t *dfull = empty + nbs;                       // [team]: the pair's MMAs done
     int2 *runinfo = reinterpret_cast<int2 *>(smem + a.o_run);   // [tile]: (tile, last arrival)
     int *coff = reinterpret_cast<int *>(smem + a.o_coff);        // first group of each contributor
     int *flags = reinterpret_cast<int *>(smem + a.o_misc);   // [0] error [1] batches issued [2] X asked
@@ -458,7 +482,7 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
 
     // a batch of 4 items = one pair per team; each team warp frees it once
     if (threadIdx.x < 2 * nbs) bar_init(full + threadIdx.x, threadIdx.x < nbs ? 1u : 4u * kTeams);
-    if (threadIdx.x < 2 * kTeams + 1) bar_init(aready + threadIdx.x, threadIdx.x < kTeams ? 4u : 1u);
+    if (threadIdx.x < kTeams) bar_init(dfull + threadIdx.x, 1u);
     if (threadIdx.x == 0) { flags[0] = 0; flags[1] = 0; flags[2] = 0; }
     for (int i = threadIdx.x; i < kTeams * ntile * M * 128; i += kThreads) res[i] = 0.f;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -482,7 +506,7 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
                     if (!ok) break;
                 }
                 const int bs = b % nbs;
-                if (b >= nbs && !bar_wait(empty + bs, (uint32_t)((b / nbs) - 1) & 1u)) { ok = false; break; }
+                if (b >= nbs && !bar_wait_sleep(empty + bs, (uint32_t)((b / nbs) - 1) & 1u)) { ok = false; break; }
                 const int i0 = b * kBatch, n = (L - i0) < kBatch ? (L - i0) : kBatch;
                 const int64_t u = rg.u0 + i0;
                 bar_expect(full + bs, (uint32_t)n * (kPlaneBlk * R + 256));
@@ -497,68 +521,9 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
             if (nbatch <= kHeadBatches) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
             if (!ok) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
         }
-    } else if (warp == kMma) {
-        // ------------------------------------------------------- MMA issue
-        // Pair jj of team t = items kBatch jj + 2 t and kBatch jj + 2 t + 1 (one ring
-        // batch).  Once the team has stored the pair's A, for each item e:
-        // D[t][e] = A[t][e] . B(X slot of the item)^T, K = 128 in 4 steps.
-        if (lane == 0) {
-            const uint32_t idesc = idesc_u8s8(a.NB);
-            constexpr int gsh = MT == 1 ? 2 : MT == 2 ? 1 : 0;   // log2 groups per B tile
-            const uint32_t b0 = smem_addr(smem + a.o_b);
-            bool ok = true;
-            uint32_t tmem = 0;
-            int nxt[kTeams], np[kTeams], xs[kTeams];   // next pair, pairs, X slot of its item 0
-#pragma unroll
-            for (int t = 0; t < kTeams; ++t) {
-                nxt[t] = 0;
-                np[t] = 2 * t < L ? (L - 2 * t + kBatch - 1) / kBatch : 0;
-                xs[t] = 2 * t;
-                while (xs[t] >= G) xs[t] -= G;
-            }
-            // serve whichever team has stored its next pair (teams run independently)
-            uint64_t last = global_ns();
-            while (ok) {
-                bool pending = false, progress = false;
-#pragma unroll
-                for (int t = 0; t < kTeams; ++t) {
-                    if (nxt[t] >= np[t]) continue;
-                    pending = true;
-                    if (!bar_try(aready + t, (uint32_t)(nxt[t] & 1))) continue;
-                    tc_fence_after();
-                    if (!tmem) tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
-                    const int i0 = kBatch * nxt[t] + 2 * t;
-                    const uint32_t col0 = tmem + (uint32_t)t * 128;
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        if (i0 + e >= L) break;
-                        const int sl = xs[t] + e >= G ? xs[t] + e - G : xs[t] + e;
-                        const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma_i8_ts(col0 + 64 + (uint32_t)(e * a.NB), col0 + 32 * e + 8 * kk,
-                                      smem_desc_sw128(baddr + 32 * kk), idesc, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(dfull + t);
-                    ++nxt[t];
-                    xs[t] += kBatch;
-                    while (xs[t] >= G) xs[t] -= G;
-                    progress = true;
-                }
-                if (!pending) break;
-                const uint64_t now = global_ns();
-                if (progress) last = now;
-                else if (now - last > kWaitNs) ok = false;
-            }
-            // TMEM may be freed only after every issued MMA has completed
-            mma_commit(mdone);
-            if (!bar_wait(mdone, 0u)) ok = false;
-            if (!ok) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
-        }
     } else if (warp < kCW) {
         // ------------------------------------------------------------- teams
-        // TMEM is taken here, off the producer's path; the MMA warp reads its
-        // address after the first A hand-off
+        // TMEM is taken here, off the producer's path
         if (warp == 0) {
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                          ::"r"(smem_addr(tmem_slot)), "r"(kTmemCols) : "memory");
@@ -592,35 +557,27 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
         while (g >= G) { g -= G; ++lt; }
         bool ok = true;
         constexpr int ND = 4 * MT;                       // D columns read per item
+        const uint32_t idesc = idesc_u8s8(a.NB);
+        constexpr int gsh = MT == 1 ? 2 : MT == 2 ? 1 : 0;   // log2 groups per B tile
+        const uint32_t b0 = smem_addr(smem + a.o_b);
+        const bool issuer = q == 0 && lane == 0;        // issues the team's MMAs
+        int issued = 0;                                  // pairs whose MMAs were issued
         for (int jj = 0; jj <= Jp; ++jj) {
             const bool have = jj < Jp, back = jj > 0;
             const int i0 = kBatch * jj + 2 * team;
             const int n = have ? (i0 + 1 < L ? 2 : 1) : 0;   // items in this pair
             uint32_t A0[32], A1[32];
             float sc[2] = {0.f, 0.f};
-            if (have) {
+            bool good = ok;
+            if (have && good) {
                 const int bs = st / kBatch;              // ring slot of the batch
-                if (!__all_sync(0xffffffffu, bar_wait(full + bs, (uint32_t)fpar))) { ok = false; break; }
-                uint4 pw[R];
-#pragma unroll
-                for (int p = 0; p < R; ++p)
-                    pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st) * kPlaneBlk + row * 16);
-                sc[0] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)st * 256 + row * 2));
-#pragma unroll
-                for (int t4 = 0; t4 < 4; ++t4) {
-                    uint32_t P[8];
-#pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const uint4 &v = pw[p < R ? p : 0];
-                        P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
-                    }
-                    field_operands<R>(P, A0 + 8 * t4);
-                }
-                if (n == 2) {
+                good = __all_sync(0xffffffffu, bar_wait(full + bs, (uint32_t)fpar));
+                if (good) {
+                    uint4 pw[R];
 #pragma unroll
                     for (int p = 0; p < R; ++p)
-                        pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st + 1) * kPlaneBlk + row * 16);
-                    sc[1] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)(st + 1) * 256 + row * 2));
+                        pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st) * kPlaneBlk + row * 16);
+                    sc[0] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)st * 256 + row * 2));
 #pragma unroll
                     for (int t4 = 0; t4 < 4; ++t4) {
                         uint32_t P[8];
@@ -629,45 +586,75 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
                             const uint4 &v = pw[p < R ? p : 0];
                             P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
                         }
-                        field_operands<R>(P, A1 + 8 * t4);
+                        field_operands<R>(P, A0 + 8 * t4);
                     }
+                    if (n == 2) {
+#pragma unroll
+                        for (int p = 0; p < R; ++p)
+                            pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st + 1) * kPlaneBlk + row * 16);
+                        sc[1] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)(st + 1) * 256 + row * 2));
+#pragma unroll
+                        for (int t4 = 0; t4 < 4; ++t4) {
+                            uint32_t P[8];
+#pragma unroll
+                            for (int p = 0; p < 8; ++p) {
+                                const uint4 &v = pw[p < R ? p : 0];
+                                P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
+                            }
+                            field_operands<R>(P, A1 + 8 * t4);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(empty + bs);
                 }
-                __syncwarp();
-                if (lane == 0) bar_arrive(empty + bs);
             }
-            if (back) {
+            if (back && good) {
                 // the MMAs of pair jj - 1 are done: A is free and D holds their sums
-                if (!__all_sync(0xffffffffu, bar_wait(dfull + team, (uint32_t)((jj - 1) & 1)))) {
-                    ok = false;
-                    break;
-                }
+                good = __all_sync(0xffffffffu, bar_wait(dfull + team, (uint32_t)((jj - 1) & 1)));
                 tc_fence_after();
             }
-            if (have) {
-                tmem_st32(lane_base + col0, A0);
-                if (n == 2) tmem_st32(lane_base + col0 + 32, A1);
-            }
             int d0[ND], d1[ND];
-            if (back) {
-                read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
-                if constexpr (MT <= 4) {
-                    if (np == 2) read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
-                    tmem_ld_wait();
-                } else {
-                    tmem_ld_wait();
-                    FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
-                    if (np == 2) {
-                        read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
+            if (good) {
+                if (have) {
+                    tmem_st32(lane_base + col0, A0);
+                    if (n == 2) tmem_st32(lane_base + col0 + 32, A1);
+                }
+                if (back) {
+                    read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
+                    if constexpr (MT <= 4) {
+                        if (np == 2) read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
                         tmem_ld_wait();
+                    } else {
+                        tmem_ld_wait();
+                        FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
+                        if (np == 2) {
+                            read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
+                            tmem_ld_wait();
+                        }
                     }
                 }
+                if (have) tmem_st_wait();
             }
-            if (have) {
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) bar_arrive(aready + team);
+            tc_fence_before();
+            // the whole team has stored A and read D (or a wait timed out)
+            if (!named_sync_and(2 + team, 128, good)) { ok = false; break; }
+            if (have && issuer) {
+                // D[team][e] = A[team][e] . B(X slot of item e)^T, K = 128 in 4 steps
+                tc_fence_after();
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    if (e < n) {
+                        const int sl = xslot + e >= G ? xslot + e - G : xslot + e;
+                        const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_i8_ts(col0 + 64 + (uint32_t)(e * a.NB), col0 + 32 * e + 8 * kk,
+                                      smem_desc_sw128(baddr + 32 * kk), idesc, kk > 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(dfull + team);
             }
+            if (have) ++issued;
             if (back) {
                 if constexpr (MT <= 4) FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
                 if (np == 2) FOLD_ITEM(d1, sp[1], slp[1], ltp[1]);
@@ -689,6 +676,10 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
 #pragma unroll
             for (int m = 0; m < MT; ++m)
                 if (m < M) res[((team * ntile + cur) * M + m) * 128 + row] = y[m];
+        }
+        if (!ok && issued > 0) {
+            // the team's last MMAs may still run: let them finish before TMEM is freed
+            bar_wait(dfull + team, (uint32_t)((issued - 1) & 1));
         }
         if (!ok && lane == 0) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
         named_sync(1, kCW * 32);
@@ -814,7 +805,7 @@ size_t layout(Plan &p, int r, int M, int S) {
     p.o_res = align_up(o, 16);
     o = p.o_res + (size_t)kTeams * p.ntile * M * 128 * 4;
     p.o_bar = align_up(o, 16);
-    o = p.o_bar + (size_t)(2 * (S / kBatch) + 2 * kTeams + 1) * 8;
+    o = p.o_bar + (size_t)(2 * (S / kBatch) + kTeams) * 8;
     p.o_run = align_up(o, 16);
     o = p.o_run + (size_t)p.ntile * 8;
     p.o_coff = align_up(o, 16);
