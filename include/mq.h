@@ -192,6 +192,18 @@ MQ_API mq_status mq_gemv_noalloc(const uint16_t *X_dev, const mq_weights *w, int
 /* Status of the most recent failing call on this host thread (MQ_OK if none). */
 MQ_API mq_status mq_last_error(void);
 
+/*
+ * Device-side failures of earlier launches on the current device: every wait
+ * inside the kernels gives up after about one second of GPU time (a copy or
+ * an MMA that never completes), records the fact in a device flag and returns
+ * instead of hanging.  This call synchronises the current device, reads and
+ * clears the flags, and returns MQ_ERR_TIMEOUT if any was set (MQ_OK
+ * otherwise; MQ_ERR_CUDA if the device cannot be read).  The Y of a launch
+ * that timed out is unspecified.  No counterpart in the paper (a robustness
+ * hook of this library).
+ */
+MQ_API mq_status mq_device_status(void);
+
 /* Text of the most recent failure on this host thread (never NULL). */
 MQ_API const char *mq_last_error_string(void);
 

@@ -17,6 +17,7 @@ __all__ = [
     "mq_plane_bytes", "mq_scale_bytes", "mq_pack", "mq_slice", "mq_gemm",
     "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
     "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
+    "mq_device_status",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -45,7 +46,7 @@ def _load() -> ctypes.CDLL:
     if not os.path.exists(library_path):
         raise ImportError(
             f"{library_path} is missing: build it with "
-            "`python -m nested_bit_weight_b200._build` (nvcc, sm_100a)")
+            "`python nested_bit_weight_b200/_build.py` (nvcc, sm_100a)")
     L = ctypes.CDLL(library_path)
     P, I64, I, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     W = ctypes.POINTER(MqWeights)
@@ -58,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "mq_gemm": (I, [P, W, I64, I64, I64, P, P, SZ, P]),
         "mq_unpack": (I, [W, P, P]),
         "mq_last_error": (I, []),
+        "mq_device_status": (I, []),
         "mq_last_error_string": (ctypes.c_char_p, []),
         "mq_status_string": (ctypes.c_char_p, [I]),
         "mq_version": (ctypes.c_char_p, []),
@@ -108,6 +110,11 @@ def mq_set_gemv_variant(variant: int) -> None:
 
 def mq_get_gemv_variant() -> int:
     return lib.mq_get_gemv_variant()
+
+
+def mq_device_status() -> None:
+    """Synchronise the device; raise if a bounded wait in an earlier launch gave up."""
+    _check(lib.mq_device_status())
 
 
 def mq_version() -> str:

@@ -155,6 +155,16 @@ mq_status mq_set_gemv_variant(int variant) {
 int mq_get_gemv_variant(void) { return __atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED); }
 
 mq_status mq_last_error(void) { return g_last; }
+
+mq_status mq_device_status(void) {
+    const cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    bool a = false, b = false;
+    if (!gemv_tc_take_timeout(&a) || !gemm_tc_take_timeout(&b))
+        return fail(MQ_ERR_CUDA, "device timeout flags not readable");
+    if (a || b) return fail(MQ_ERR_TIMEOUT, "a bounded device-side wait expired in an earlier launch");
+    return MQ_OK;
+}
 const char *mq_last_error_string(void) { return g_msg; }
 
 const char *mq_status_string(mq_status s) {

@@ -38,6 +38,9 @@ mq_status check_weights(const mq_weights *w, int64_t N, int64_t K);
 
 // Kernel launchers (each returns MQ_OK or MQ_ERR_CUDA after the launch).
 bool gemv_tc_supported(int64_t M, int64_t N, int64_t K, int r);
+// Read and clear the device flag of a timed-out wait (false: device not readable).
+bool gemv_tc_take_timeout(bool *set);
+bool gemm_tc_take_timeout(bool *set);
 size_t gemv_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M,
                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);

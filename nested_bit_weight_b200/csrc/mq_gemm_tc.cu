@@ -337,4 +337,12 @@ mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint
     return MQ_OK;
 }
 
+bool gemm_tc_take_timeout(bool *set) {
+    unsigned v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_timeout, sizeof(v)) != cudaSuccess) return false;
+    if (v && cudaMemcpyToSymbol(g_tc_timeout, &z, sizeof(z)) != cudaSuccess) return false;
+    *set = v != 0;
+    return true;
+}
+
 }  // namespace mq

@@ -837,7 +837,7 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     const size_t stage = (size_t)2048 * r + 256;
     const size_t fixed = layout(p, r, (int)M, 0);
     const int need = (int)((L + kBatch - 1) / kBatch) * kBatch;   // stages for the whole range
-    const int want = need < 2 * kBatch ? need : 2 * kBatch;        // fewest stages accepted
+    const int want = need < kBatch ? need : kBatch;                // fewest stages accepted (one batch)
     p.part_off = kTicketBytes;
     p.ws_bytes = p.part_off + (size_t)W * M * 128 * sizeof(float);
     p.ok = false;
@@ -906,6 +906,14 @@ mq_status run_r(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y,
 }
 
 }  // namespace
+
+bool gemv_tc_take_timeout(bool *set) {
+    unsigned v = 0, z = 0;
+    if (cudaMemcpyFromSymbol(&v, g_gemv_timeout, sizeof(v)) != cudaSuccess) return false;
+    if (v && cudaMemcpyToSymbol(g_gemv_timeout, &z, sizeof(z)) != cudaSuccess) return false;
+    *set = v != 0;
+    return true;
+}
 
 bool gemv_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
     return M >= 1 && M <= kGemvMaxM && make_plan(M, N, K, r).ok;

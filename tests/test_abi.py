@@ -32,6 +32,10 @@ def test_sizes():
     assert mq.mq_plane_bytes(4096, 4096, 2) == 2 * 4096 * 4096 // 8
     assert mq.mq_plane_bytes(4096, 4096, 8) == 4096 * 4096
     assert mq.mq_scale_bytes(4096, 4096) == 2 * 4096 * 32
+    # rows are padded to a multiple of 128 in the stored planes and scales
+    assert mq.mq_plane_bytes(130, 256, 2) == 2 * 256 * 256 // 8
+    assert mq.mq_scale_bytes(130, 256) == 2 * 256 * 2
+    assert mq.mq_plane_bytes(1, 128, 8) == 128 * 128
     assert mq.mq_plane_bytes(4, 100, 2) == 0          # K not a multiple of 128
     assert mq.mq_plane_bytes(4, 128, 9) == 0
     assert mq.mq_scale_bytes(4, 256, 64) == 0

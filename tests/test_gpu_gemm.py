@@ -183,3 +183,16 @@ def test_workspace_shared_across_shapes():
         mq.mq_gemm(Xd, parent.view(r), Y, ws)
         Yh = Y.float().cpu().numpy()
         assert oracle.violation_ratio(Yh, oracle.gemm(X, codes, s, r)) <= 1.0
+
+
+def test_no_device_wait_timed_out():
+    # every launch above and these ones completed without a bounded wait giving up
+    import torch
+    import nested_bit_weight_b200 as mq
+    for (N, K, M, r) in ((4096, 4096, 1, 4), (1024, 4096, 2, 2), (640, 1280, 5, 3), (512, 512, 32, 8)):
+        codes, s, _ = wl.gen_weights(N, K, seed=N + M)
+        xb, _ = wl.gen_x(M, K, seed=K + M)
+        p = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+        X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+        mq.gemm(X, p, r)
+    mq.mq_device_status()
