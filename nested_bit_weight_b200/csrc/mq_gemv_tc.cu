@@ -39,6 +39,8 @@
 // last CTA to arrive summing every part in a fixed order.
 #include <string.h>
 
+#include <mutex>
+
 #include "mq_common.cuh"
 #include "mq_bits.cuh"
 
@@ -167,14 +169,36 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
         ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(b)) : "memory");
 }
-// Arrival ticket: acquire-release add at GPU scope, returns the old value.
-__device__ __forceinline__ unsigned ticket_add(unsigned *p) {
-    unsigned old;
-    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
-    return old;
-}
 __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// Distributed shared memory: the address of `local` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+// Arrive on an mbarrier of another CTA of the cluster, releasing this CTA's
+// earlier writes (cumulative over the CTA barrier that precedes it).
+__device__ __forceinline__ void bar_arrive_remote(uint32_t addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(addr) : "memory");
+}
+__device__ __forceinline__ bool bar_try_cluster(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(ok) : "r"(smem_addr(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
 }
 // Named barrier that also returns the AND of `v` over its threads, so that a
 // whole team takes the same branch after a wait that may have timed out.
@@ -281,10 +305,33 @@ __host__ __device__ constexpr uint32_t idesc_u8s8(int N) {
 // ------------------------------------------------------------ decomposition
 // Items u = 0 .. W-1, W = T * KC (T 128-row tiles, KC = K / 128 groups), in
 // (tile, group) order; CTA b owns the contiguous items [first(b), first(b+1)).
+// Clusters: the row tiles are cut into NC contiguous runs, one per cluster of
+// CS CTAs; the items of a cluster's run are cut into CS contiguous ranges.  A
+// row tile is therefore shared only by CTAs of one cluster, which sum it
+// through distributed shared memory (CS = 1: every CTA owns whole tiles).
 struct Work {
-    int64_t T, KC, W, C;
-    __host__ __device__ int64_t first(int64_t b) const { return b * W / C; }
-    __host__ __device__ int64_t cta_of(int64_t u) const { return ((u + 1) * C - 1) / W; }
+    int64_t T, KC;          // row tiles, groups per tile
+    int NC, CS;             // clusters, CTAs per cluster
+    // 32-bit arithmetic (T * KC < 2^31 and the products below stay under 2^32):
+    // a 64-bit division costs hundreds of cycles on the GPU
+    __host__ __device__ uint32_t tile_begin(uint32_t c) const {
+        return (uint32_t)(c * (uint32_t)T) / (uint32_t)NC;
+    }
+    __host__ __device__ int64_t first(int64_t bb) const {
+        const uint32_t b = (uint32_t)bb, c = b / (uint32_t)CS, k = b - c * (uint32_t)CS;
+        const uint32_t t0 = tile_begin(c), t1 = tile_begin(c + 1);
+        const uint32_t a = t0 * (uint32_t)KC, wc = (t1 - t0) * (uint32_t)KC;
+        return (int64_t)(a + k * wc / (uint32_t)CS);
+    }
+    // CTA that holds item u
+    __host__ __device__ int64_t cta_of(int64_t uu) const {
+        const uint32_t u = (uint32_t)uu, t = u / (uint32_t)KC;
+        const uint32_t c = ((t + 1) * (uint32_t)NC - 1) / (uint32_t)T;
+        const uint32_t t0 = tile_begin(c), t1 = tile_begin(c + 1);
+        const uint32_t a = t0 * (uint32_t)KC, wc = (t1 - t0) * (uint32_t)KC;
+        return (int64_t)(c * (uint32_t)CS + ((u - a + 1) * (uint32_t)CS - 1) / wc);
+    }
+    __host__ __device__ int64_t ctas() const { return (int64_t)NC * CS; }
 };
 
 struct Range { int u0, u1, L; };
@@ -309,14 +356,13 @@ struct Args {
     const uint8_t *planes;  // tiled planes (2 KB per (tile, group) block per plane)
     const uint8_t *scales;  // tiled fp16 scales (256 B per block)
     __nv_bfloat16 *Y;
-    float *part;            // [T][G][M][128] partial sums of shared tiles
-    unsigned *tickets;      // [T] arrivals at shared tiles (zero between calls)
     Work w;
     int64_t N, K, G;
     int64_t plane_bytes;    // bytes of one plane
     int M, NB, S;           // batch rows, MMA N (16 or 32), ring stages (multiple of kBatch)
     // shared-memory offsets from the 1024-byte aligned base
-    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_run, o_coff, o_misc;
+    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_red, o_misc;
+    int ntile_max;          // largest number of row tiles a CTA touches
 };
 
 // ------------------------------------------------------------- X operand
@@ -473,8 +519,9 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.o_bar);
     uint64_t *empty = full + nbs;
     uint64_t *dfull = empty + nbs;                       // [team]: the pair's MMAs done
-    int2 *runinfo = reinterpret_cast<int2 *>(smem + a.o_run);   // [tile]: (tile, last arrival)
-    int *coff = reinterpret_cast<int *>(smem + a.o_coff);        // first group of each contributor
+    uint64_t *rbar = dfull + kTeams;                     // [tile]: parts of the tile received
+    // parts of the split tiles this CTA owns: [tile][contributor][m][128]
+    float *red = reinterpret_cast<float *>(smem + a.o_red);
     int *flags = reinterpret_cast<int *>(smem + a.o_misc);   // [0] error [1] batches issued [2] X asked
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + a.o_misc + 16);
     float *res = reinterpret_cast<float *>(smem + a.o_res);  // [team][tile][m][128]
@@ -483,10 +530,18 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
     // a batch of 4 items = one pair per team; each team warp frees it once
     if (threadIdx.x < 2 * nbs) bar_init(full + threadIdx.x, threadIdx.x < nbs ? 1u : 4u * kTeams);
     if (threadIdx.x < kTeams) bar_init(dfull + threadIdx.x, 1u);
+    // The CTA holding a tile's first item owns it; if the tile continues in
+    // later CTAs (of the same cluster), it waits for their parts.
+    const int64_t tl = (rg.u1 - 1) / G;                  // last tile of the range
+    const int64_t own_last = (tl * G >= rg.u0 && tl * G + G > rg.u1) ? tl : -1;
+    const int own_nc = own_last >= 0 ? (int)(w.cta_of(own_last * G + G - 1) - blockIdx.x + 1) : 0;
+    if (threadIdx.x == 0 && own_nc > 1) bar_init(rbar + (own_last - tf), (uint32_t)(own_nc - 1));
     if (threadIdx.x == 0) { flags[0] = 0; flags[1] = 0; flags[2] = 0; }
     for (int i = threadIdx.x; i < kTeams * ntile * M * 128; i += kThreads) res[i] = 0.f;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
+    // every CTA of the cluster has initialised its barriers before any part is sent
+    if (w.CS > 1) cluster_arrive();
 
     if (warp == kProd) {
         // ---------------------------------------------------------- producer
@@ -683,68 +738,54 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
         }
         if (!ok && lane == 0) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
         named_sync(1, kCW * 32);
-        // ---- combine the teams per tile (fixed order) and write Y or the part
+        // ---- combine the teams per tile (fixed order).  A tile inside this
+        // CTA goes to Y; a tile this CTA owns but shares keeps its part in
+        // slot 0 of `red`; the first tile, if it started in an earlier CTA of
+        // the cluster, is sent to slot j of its owner (j = distance in CTAs).
+        const int64_t ra0 = tf * G;
+        const bool sends = ra0 < rg.u0;                  // the first tile started earlier
+        const int64_t owner = sends ? w.cta_of(ra0) : -1;
+        const int owner_rank = (int)owner % w.CS;
+        const int owner_lt = sends ? (int)tf - (int)w.first(owner) / G : 0;
+        const int jsend = (int)(blockIdx.x - owner);
+        if (sends) cluster_wait();                       // the owner's barrier is initialised
+        const uint32_t red_base = smem_addr(red);
         for (int idx = threadIdx.x; idx < ntile * M * 128; idx += kCW * 32) {
             const int lt = idx / (M * 128), rem = idx - lt * M * 128, m = rem >> 7, rr = rem & 127;
             float v = 0.f;
 #pragma unroll
             for (int tm = 0; tm < kTeams; ++tm) v += res[((tm * ntile + lt) * M + m) * 128 + rr];
-            const int64_t t = tf + lt;
-            const int64_t ra = t * G, rb = ra + G;
-            const int64_t n = t * 128 + rr;
-            if (ra >= rg.u0 && rb <= rg.u1) {
-                if (n < a.N) a.Y[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
-            } else {
-                const int64_t kcf = (ra > rg.u0 ? ra : rg.u0) - ra;
-                a.part[((t * G + kcf) * M + m) * 128 + rr] = v;
-            }
-        }
-        named_sync(1, kCW * 32);
-        // ---- shared tiles: one arrival ticket per tile; the last CTA to
-        // arrive sums every part in a fixed order (contributing CTAs in
-        // increasing order) and writes Y.  The CTA barrier before the
-        // acquire-release ticket makes all of this CTA's parts visible with
-        // it; the barrier after it orders the last arriver's reads.
-        for (int lt = threadIdx.x; lt < ntile; lt += kCW * 32) {
             const int64_t t = tf + lt, ra = t * G, rb = ra + G;
-            int last = 0;
-            if (ra < rg.u0 || rb > rg.u1) {
-                const unsigned nct = (unsigned)(w.cta_of(rb - 1) - w.cta_of(ra) + 1);
-                last = ticket_add(&a.tickets[t]) == nct - 1u;
+            if (ra >= rg.u0 && rb <= rg.u1) {
+                const int64_t n = t * 128 + rr;
+                if (n < a.N) a.Y[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
+            } else if (ra >= rg.u0) {
+                red[((size_t)lt * w.CS) * M * 128 + rem] = v;
+            } else {
+                const uint32_t off = (uint32_t)((((size_t)owner_lt * w.CS + jsend) * M * 128 + rem) * 4);
+                st_cluster_f32(cluster_map(red_base + off, (uint32_t)owner_rank), v);
             }
-            runinfo[lt] = make_int2((int)t, last);
         }
         named_sync(1, kCW * 32);
-        for (int lt = 0; lt < ntile; ++lt) {
-            if (!runinfo[lt].y) continue;
-            const int64_t t = runinfo[lt].x, ra = t * G;
-            const int64_t c0 = w.cta_of(ra);
-            const int nc = (int)(w.cta_of(ra + G - 1) - c0 + 1);
-            for (int c = threadIdx.x; c < nc; c += kCW * 32) {
-                const int64_t f = w.first(c0 + c);
-                coff[c] = (int)((f > ra ? f : ra) - ra);
+        if (sends && threadIdx.x == 0)
+            bar_arrive_remote(cluster_map(smem_addr(rbar + owner_lt), (uint32_t)owner_rank));
+        if (own_nc > 1) {
+            // the owned last tile: wait for the other parts, sum in CTA order
+            const int lt = (int)(own_last - tf);
+            bool got = true;
+            if (threadIdx.x == 0) {
+                const uint64_t t0 = global_ns();
+                while (!bar_try_cluster(rbar + lt, 0u))
+                    if (global_ns() - t0 > kWaitNs) { got = false; break; }
+                if (!got) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
             }
             named_sync(1, kCW * 32);
-            const float *pt = a.part + t * G * M * 128;
             for (int idx = threadIdx.x; idx < M * 128; idx += kCW * 32) {
                 float v = 0.f;
-                int c = 0;
-                for (; c + 4 <= nc; c += 4) {
-                    const float p0 = __ldcg(pt + (int64_t)coff[c] * M * 128 + idx);
-                    const float p1 = __ldcg(pt + (int64_t)coff[c + 1] * M * 128 + idx);
-                    const float p2 = __ldcg(pt + (int64_t)coff[c + 2] * M * 128 + idx);
-                    const float p3 = __ldcg(pt + (int64_t)coff[c + 3] * M * 128 + idx);
-                    v += p0;
-                    v += p1;
-                    v += p2;
-                    v += p3;
-                }
-                for (; c < nc; ++c) v += __ldcg(pt + (int64_t)coff[c] * M * 128 + idx);
-                const int64_t n = t * 128 + (idx & 127);
+                for (int j = 0; j < own_nc; ++j) v += red[((size_t)lt * w.CS + j) * M * 128 + idx];
+                const int64_t n = own_last * 128 + (idx & 127);
                 if (n < a.N) a.Y[(int64_t)(idx >> 7) * a.N + n] = __float2bfloat16_rn(v);
             }
-            named_sync(1, kCW * 32);
-            if (threadIdx.x == 0) a.tickets[t] = 0u;
         }
     }
 
@@ -770,8 +811,8 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
 struct Plan {
     Work w;
     int NB, S, nslot, L, ntile;
-    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_run, o_coff, o_misc;
-    size_t smem, part_off, ws_bytes;
+    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_red, o_misc;
+    size_t smem;
     bool ok;
 };
 
@@ -805,32 +846,28 @@ size_t layout(Plan &p, int r, int M, int S) {
     p.o_res = align_up(o, 16);
     o = p.o_res + (size_t)kTeams * p.ntile * M * 128 * 4;
     p.o_bar = align_up(o, 16);
-    o = p.o_bar + (size_t)(2 * (S / kBatch) + kTeams) * 8;
-    p.o_run = align_up(o, 16);
-    o = p.o_run + (size_t)p.ntile * 8;
-    p.o_coff = align_up(o, 16);
-    o = p.o_coff + (size_t)(p.w.C + 1) * 4;
+    o = p.o_bar + (size_t)(2 * (S / kBatch) + kTeams + p.ntile) * 8;
+    p.o_red = align_up(o, 16);
+    o = p.o_red + (p.w.CS > 1 ? (size_t)p.ntile * p.w.CS * M * 128 * 4 : 0);
     p.o_misc = align_up(o, 16);
     o = p.o_misc + 64;                                     // flags, TMEM address
     return o;
 }
 
-Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
+// Ranges, ring and shared memory for one (clusters, CTAs per cluster) split.
+Plan plan_for(const Work &w, int64_t M, int r) {
     Plan p{};
-    const int64_t T = (N + 127) / 128, G = K / kGroup;
-    const int64_t W = T * G;
+    p.w = w;
     p.NB = M <= 4 ? 16 : 32;
-    const int64_t C = W < sm_count() ? W : sm_count();
-    const Work w{T, G, W, C};
+    const int64_t G = w.KC;
     int64_t L = 0, nt = 0;
-    for (int64_t b = 0; b < C; ++b) {
+    for (int64_t b = 0; b < w.ctas(); ++b) {
         const int64_t u0 = w.first(b), u1 = w.first(b + 1);
-        if (u1 <= u0) continue;
+        if (u1 <= u0) return p;                            // an empty CTA: not a valid split
         L = u1 - u0 > L ? u1 - u0 : L;
         const int64_t tt = (u1 - 1) / G - u0 / G + 1;
         nt = tt > nt ? tt : nt;
     }
-    p.w = w;
     p.L = (int)L;
     p.ntile = (int)nt;
     p.nslot = (int)(L < G ? L : G);
@@ -838,17 +875,46 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     const size_t fixed = layout(p, r, (int)M, 0);
     const int need = (int)((L + kBatch - 1) / kBatch) * kBatch;   // stages for the whole range
     const int want = need < kBatch ? need : kBatch;                // fewest stages accepted (one batch)
-    p.part_off = kTicketBytes;
-    p.ws_bytes = p.part_off + (size_t)W * M * 128 * sizeof(float);
-    p.ok = false;
-    if (T > (int64_t)(kTicketBytes / sizeof(unsigned))) return p;
     if (fixed + (size_t)want * stage + 1024 > kSmemMax) return p;
     int S = (int)((kSmemMax - 1024 - fixed) / stage) / kBatch * kBatch;
     if (S > need) S = need;
+    // the ring's barriers and alignment come on top of `fixed`
+    while (S > want && layout(p, r, (int)M, S) + 1024 > kSmemMax) S -= kBatch;
     p.S = S;
     p.smem = layout(p, r, (int)M, S) + 1024;
-    p.ok = true;
+    p.ok = p.smem <= kSmemMax;
     return p;
+}
+
+int max_clusters(int r, int64_t M, size_t smem, int cs);   // below, per instantiation
+
+// Choose the split: whole tiles per CTA (CS = 1) or clusters of CS CTAs that
+// share tiles, taking the one with the fewest items on the busiest CTA (a
+// shared tile costs about one extra item of latency for its exchange).
+Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
+    const int64_t T = (N + 127) / 128, G = K / kGroup;
+    const int sms = sm_count();
+    Plan best{};
+    double best_cost = 1e30;
+    if (T * G * 8 >= ((int64_t)1 << 32) || T * (int64_t)sms >= ((int64_t)1 << 32)) return best;
+    for (int cs = 1; cs <= 8; ++cs) {
+        int64_t nc = sms / cs;
+        if (nc > T) nc = T;
+        if (nc < 1 || T / nc * G < cs) continue;
+        Plan p{};
+        for (int it = 0; it < 3; ++it) {
+            p = plan_for(Work{T, G, (int)nc, cs}, M, r);
+            if (!p.ok) break;
+            const int mc = cs > 1 ? max_clusters(r, M, p.smem, cs) : sms;
+            if (mc >= nc) break;
+            if (mc < 1) { p.ok = false; break; }
+            nc = mc;
+        }
+        if (!p.ok) continue;
+        const double cost = p.L + (cs > 1 ? 1.0 : 0.0);
+        if (cost < best_cost) { best_cost = cost; best = p; }
+    }
+    return best;
 }
 
 template <int R, int MT>
@@ -867,8 +933,6 @@ mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, c
     a.planes = reinterpret_cast<const uint8_t *>(wt->planes);
     a.scales = reinterpret_cast<const uint8_t *>(wt->scales);
     a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
-    a.part = reinterpret_cast<float *>(ws + p.part_off);
-    a.tickets = reinterpret_cast<unsigned *>(ws);
     a.w = p.w;
     a.N = wt->N;
     a.K = wt->K;
@@ -878,22 +942,59 @@ mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, c
     a.NB = p.NB;
     a.S = p.S;
     a.o_ring = p.o_ring; a.o_sring = p.o_sring; a.o_b = p.o_b; a.o_pair = p.o_pair;
-    a.o_res = p.o_res; a.o_bar = p.o_bar; a.o_run = p.o_run; a.o_coff = p.o_coff; a.o_misc = p.o_misc;
+    a.o_res = p.o_res; a.o_bar = p.o_bar; a.o_red = p.o_red; a.o_misc = p.o_misc;
+    a.ntile_max = p.ntile;
     // programmatic dependent launch: this grid may start while the previous
     // kernel of the stream finishes; it waits for it before reading X
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)p.w.C);
+    cfg.gridDim = dim3((unsigned)p.w.ctas());
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)p.w.CS;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = p.w.CS > 1 ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, nested_gemv_tc_kernel<R, MT>, a);
     if (e != cudaSuccess) return cuda_fail(e, "nested_gemv_tc_kernel launch");
     return MQ_OK;
+}
+
+// Clusters of cs CTAs (with `smem` bytes each) that can be resident at once.
+template <int R, int MT>
+int occ_clusters(size_t smem, int cs) {
+    if (cudaFuncSetAttribute(nested_gemv_tc_kernel<R, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kSmemMax) != cudaSuccess)
+        return 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)cs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute at;
+    at.id = cudaLaunchAttributeClusterDimension;
+    at.val.clusterDim.x = (unsigned)cs;
+    at.val.clusterDim.y = 1;
+    at.val.clusterDim.z = 1;
+    cfg.attrs = &at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, nested_gemv_tc_kernel<R, MT>, &cfg) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return n;
+}
+template <int R>
+int occ_clusters_r(int64_t M, size_t smem, int cs) {
+    if (M == 1) return occ_clusters<R, 1>(smem, cs);
+    if (M == 2) return occ_clusters<R, 2>(smem, cs);
+    if (M <= 4) return occ_clusters<R, 4>(smem, cs);
+    return occ_clusters<R, 8>(smem, cs);
 }
 
 template <int R>
@@ -903,6 +1004,41 @@ mq_status run_r(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y,
     if (M == 2) return run<R, 2>(X, wt, M, Y, ws, p, st);
     if (M <= 4) return run<R, 4>(X, wt, M, Y, ws, p, st);
     return run<R, 8>(X, wt, M, Y, ws, p, st);
+}
+
+int max_clusters(int r, int64_t M, size_t smem, int cs) {
+    switch (r) {
+        case 1: return occ_clusters_r<1>(M, smem, cs);
+        case 2: return occ_clusters_r<2>(M, smem, cs);
+        case 3: return occ_clusters_r<3>(M, smem, cs);
+        case 4: return occ_clusters_r<4>(M, smem, cs);
+        case 5: return occ_clusters_r<5>(M, smem, cs);
+        case 6: return occ_clusters_r<6>(M, smem, cs);
+        case 7: return occ_clusters_r<7>(M, smem, cs);
+        default: return occ_clusters_r<8>(M, smem, cs);
+    }
+}
+
+// make_plan runs a search (and occupancy queries): keep the last plans.
+Plan cached_plan(int64_t M, int64_t N, int64_t K, int r) {
+    struct Entry { int64_t M, N, K; int r, dev; Plan p; };
+    static std::mutex mu;
+    static Entry tab[64];
+    static int used = 0, next = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        for (int i = 0; i < used; ++i)
+            if (tab[i].M == M && tab[i].N == N && tab[i].K == K && tab[i].r == r && tab[i].dev == dev)
+                return tab[i].p;
+    }
+    const Plan p = make_plan(M, N, K, r);
+    std::lock_guard<std::mutex> lk(mu);
+    tab[next] = Entry{M, N, K, r, dev, p};
+    next = (next + 1) % 64;
+    if (used < 64) ++used;
+    return p;
 }
 
 }  // namespace
@@ -916,19 +1052,17 @@ bool gemv_tc_take_timeout(bool *set) {
 }
 
 bool gemv_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
-    return M >= 1 && M <= kGemvMaxM && make_plan(M, N, K, r).ok;
+    return M >= 1 && M <= kGemvMaxM && cached_plan(M, N, K, r).ok;
 }
 
-size_t gemv_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
-    const Plan p = make_plan(M, N, K, r);
-    return p.ok ? p.ws_bytes : 0;
-}
+// The GEMV sums shared tiles inside clusters: it needs no workspace.
+size_t gemv_tc_workspace_bytes(int64_t, int64_t, int64_t, int) { return 0; }
 
 mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
                          void *ws, size_t ws_bytes, cudaStream_t st) {
-    const Plan p = make_plan(M, w->N, w->K, w->r);
+    (void)ws_bytes;
+    const Plan p = cached_plan(M, w->N, w->K, w->r);
     if (!p.ok) return fail(MQ_ERR_UNSUPPORTED, "no tensor-core GEMV plan fits this shape");
-    if (p.ws_bytes > ws_bytes) return fail(MQ_ERR_WORKSPACE, "GEMV workspace too small");
     char *b = static_cast<char *>(ws);
     switch (w->r) {
         case 1: return run_r<1>(X, w, M, Y, b, p, st);

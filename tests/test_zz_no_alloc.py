@@ -60,7 +60,7 @@ def test_noalloc_rejects_oversized_and_large_m():
     Y = torch.zeros((9, N), dtype=torch.bfloat16, device="cuda")
     assert fn(X.data_ptr(), ctypes.byref(w), 9, N, K, Y.data_ptr(), None) == 1
     # a workspace need above 16 MiB is refused before any launch
-    # (M = 1, N = 2^17, K = 4096, r = 2: 32768 items of 512 B of partial sums)
-    big = mq.MqWeights(w.planes, w.scales, 1 << 17, 4096, 128, 2)
-    assert mq.mq_gemm_workspace_bytes(1, 1 << 17, 4096, 2) > (16 << 20)
-    assert fn(X.data_ptr(), ctypes.byref(big), 1, 1 << 17, 4096, Y.data_ptr(), None) == 6
+    # (M = 1, N = 128, K = 2^20: the GEMM fallback's operand copy of X alone is 32 MiB)
+    big = mq.MqWeights(w.planes, w.scales, 128, 1 << 20, 128, 2)
+    assert mq.mq_gemm_workspace_bytes(1, 128, 1 << 20, 2) > (16 << 20)
+    assert fn(X.data_ptr(), ctypes.byref(big), 1, 128, 1 << 20, Y.data_ptr(), None) == 6
