@@ -414,39 +414,51 @@ __device__ void build_x_operand(const Args &a, uint8_t *smem, const Work &w, con
             }
         }
         if (t0 == 0 && lane == 0) st_release(&flags[2], (int)(hv[0][0] | 1u));   // X fetched: stream the rest
+        // the four tasks side by side (independent chains; absent tasks are
+        // computed on zeros and not stored)
+        int emax[4];
+        float sum[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            emax[c] = -1000;
+            sum[c] = 0.f;
+            if (t0 + c * kCW >= nslot * M) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) hv[c][b] = 0u;
+            }
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int e8 = (int)((hv[c][b] >> 7) & 0xFFu);
+                const int v = e8 ? e8 - sh : -1000;
+                emax[c] = v > emax[c] ? v : emax[c];
+                sum[c] += __uint_as_float(hv[c][b] << 16);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int other = __shfl_xor_sync(0xffffffffu, emax[c], o);
+                emax[c] = other > emax[c] ? other : emax[c];
+                sum[c] += __shfl_xor_sync(0xffffffffu, sum[c], o);
+            }
+        }
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             const int task = t0 + c * kCW;
             if (task >= nslot * M) break;
             const int sl = task / M, m = task - sl * M;
-            uint32_t h[4];
-            int emax = -1000;
-            float sum = 0.f;
-#pragma unroll
-            for (int b = 0; b < 4; ++b) {
-                h[b] = hv[c][b];
-                const int e8 = (int)((h[b] >> 7) & 0xFFu);
-                const int v = e8 ? e8 - sh : -1000;
-                emax = v > emax ? v : emax;
-                sum += __uint_as_float(h[b] << 16);
-            }
-#pragma unroll
-            for (int o = 16; o >= 1; o >>= 1) {
-                const int other = __shfl_xor_sync(0xffffffffu, emax, o);
-                emax = other > emax ? other : emax;
-                sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            }
-            const int Eg = emax > -1000 ? emax - 127 : 0;
+            const int Eg = emax[c] > -1000 ? emax[c] - 127 : 0;
             int F[4];
 #pragma unroll
-            for (int b = 0; b < 4; ++b) F[b] = fixed_point(h[b], sh, Eg);
+            for (int b = 0; b < 4; ++b) F[b] = fixed_point(hv[c][b], sh, Eg);
             uint32_t wd[kSlices];
             wd[0] = pack_bytes(F[0] >> 21, F[1] >> 21, F[2] >> 21, F[3] >> 21);
             wd[1] = pack_bytes(F[0] >> 14, F[1] >> 14, F[2] >> 14, F[3] >> 14) & 0x7F7F7F7Fu;
             wd[2] = pack_bytes(F[0] >> 7, F[1] >> 7, F[2] >> 7, F[3] >> 7) & 0x7F7F7F7Fu;
             wd[3] = pack_bytes(F[0], F[1], F[2], F[3]) & 0x7F7F7F7Fu;
             uint8_t *tile = smem + a.o_b + (size_t)(sl / gpb) * a.NB * 128;
-            const int chunk = 2 * t + (wi >> 2);               // 16-byte chunk of k = 32t + 4wi
+            const int chunk = 2 * t + (wi >> 2);           // 16-byte chunk of k = 32t + 4wi
 #pragma unroll
             for (int j = 0; j < kSlices; ++j) {
                 const int row = 4 * ((sl % gpb) * M + m) + j;
@@ -457,7 +469,7 @@ __device__ void build_x_operand(const Args &a, uint8_t *smem, const Work &w, con
                 // 2^(8-r) 2^(Eg-6), clamped to the normal fp32 range
                 int ex = 2 - R + Eg;
                 ex = ex < -126 ? -126 : (ex > 127 ? 127 : ex);
-                pairs[sl * 8 + m] = make_float2(__int_as_float((ex + 127) << 23), sum);
+                pairs[sl * 8 + m] = make_float2(__int_as_float((ex + 127) << 23), sum[c]);
             }
         }
     }
@@ -529,7 +541,8 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
 
     // a batch of 4 items = one pair per team; each team warp frees it once
     if (threadIdx.x < 2 * nbs) bar_init(full + threadIdx.x, threadIdx.x < nbs ? 1u : 4u * kTeams);
-    if (threadIdx.x < kTeams) bar_init(dfull + threadIdx.x, 1u);
+    // one commit per MMA issuer of a pair (kIssuers threads per team)
+    if (threadIdx.x < kTeams) bar_init(dfull + threadIdx.x, (uint32_t)(MT <= 2 ? 4 : 2));
     // The CTA holding a tile's first item owns it; if the tile continues in
     // later CTAs (of the same cluster), it waits for their parts.
     const int64_t tl = (rg.u1 - 1) / G;                  // last tile of the range
@@ -615,7 +628,10 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
         const uint32_t idesc = idesc_u8s8(a.NB);
         constexpr int gsh = MT == 1 ? 2 : MT == 2 ? 1 : 0;   // log2 groups per B tile
         const uint32_t b0 = smem_addr(smem + a.o_b);
-        const bool issuer = q == 0 && lane == 0;        // issues the team's MMAs
+        // MMA issuers: for M <= 2 the first thread of each warp q issues K steps
+        // 2(q&1), 2(q&1)+1 of item q>>1 into its own half of D; otherwise the
+        // first thread of warp e < 2 issues all four steps of item e
+        const bool issuer = lane == 0 && (MT <= 2 || q < 2);
         int issued = 0;                                  // pairs whose MMAs were issued
         for (int jj = 0; jj <= Jp; ++jj) {
             const bool have = jj < Jp, back = jj > 0;
@@ -675,11 +691,28 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
                     if (n == 2) tmem_st32(lane_base + col0 + 32, A1);
                 }
                 if (back) {
-                    read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
-                    if constexpr (MT <= 4) {
+                    if constexpr (MT <= 2) {
+                        // each item's D is two halves (K steps 0-1 and 2-3): add them
+                        int h0[ND], h1[ND];
+                        const uint32_t o0 = 4 * M * (slp[0] & (gpb - 1)), o1 = 4 * M * (slp[1] & (gpb - 1));
+                        read_d<MT>(lane_base + col0 + 64 + o0, d0);
+                        read_d<MT>(lane_base + col0 + 64 + 16 + o0, h0);
+                        if (np == 2) {
+                            read_d<MT>(lane_base + col0 + 96 + o1, d1);
+                            read_d<MT>(lane_base + col0 + 112 + o1, h1);
+                        }
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < ND; ++i) {
+                            d0[i] += h0[i];
+                            d1[i] += h1[i];
+                        }
+                    } else if constexpr (MT <= 4) {
+                        read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
                         if (np == 2) read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
                         tmem_ld_wait();
                     } else {
+                        read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
                         tmem_ld_wait();
                         FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
                         if (np == 2) {
@@ -694,10 +727,23 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
             // the whole team has stored A and read D (or a wait timed out)
             if (!named_sync_and(2 + team, 128, good)) { ok = false; break; }
             if (have && issuer) {
-                // D[team][e] = A[team][e] . B(X slot of item e)^T, K = 128 in 4 steps
+                // D[team][e] = A[team][e] . B(X slot of item e)^T, K = 128 in 4 steps;
+                // every issuer commits (an empty commit arrives at once)
                 tc_fence_after();
+                if constexpr (MT <= 2) {
+                    const int e = q >> 1, h = q & 1;
+                    if (e < n) {
+                        const int sl = xslot + e >= G ? xslot + e - G : xslot + e;
+                        const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
+                        for (int k2 = 0; k2 < 2; ++k2) {
+                            const int kk = 2 * h + k2;
+                            mma_i8_ts(col0 + 64 + (uint32_t)(32 * e + 16 * h), col0 + 32 * e + 8 * kk,
+                                      smem_desc_sw128(baddr + 32 * kk), idesc, k2 > 0 ? 1u : 0u);
+                        }
+                    }
+                } else {
+                    const int e = q;
                     if (e < n) {
                         const int sl = xslot + e >= G ? xslot + e - G : xslot + e;
                         const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
