@@ -113,7 +113,11 @@ MQ_API mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out);
 
 /*
  * Bytes of device workspace mq_gemm needs for this problem (0 if none).
- * The workspace holds split-K partial sums and arrival counters.
+ * The workspace holds the M >= 9 GEMM's split-K partial sums, its X operand
+ * and arrival counters.  The M <= 8 kernel uses none (tiles shared between
+ * CTAs are summed inside thread-block clusters), but for M <= 8 the size
+ * still covers the GEMM, which serves shapes the GEMV cannot take and the
+ * MQ_GEMV_VIA_GEMM variant.
  */
 MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
