@@ -20,23 +20,25 @@
 //   memory, K-major, 128-byte swizzle).  z_k = x_k 2^(-sh(k)) is cut into
 //   four int8 slices relative to the group exponent Eg = max floor(log2|z|):
 //       z_k = 2^(Eg-27) (a_1 2^21 + a_2 2^14 + a_3 2^7 + a_4),
-//   exact for every x within 2^-14 of the group's largest; column 4m + j at
+//   exact for every x within 2^-20 of the group's largest; column 4m + j at
 //   k = 32t + 4i + b holds slice j of z at column 32t + 8b + i.
 // * D (128 x N, int32, TMEM) = exact per-group integer sums, read back with
 //   tcgen05.ld and folded into fp32: y += s_g 2^(8-r) 2^(Eg-6) sum_j 2^(-7j) D_j
 //   + s_g (2^(7-r) - 128) S_g.
 //
 // Work: the (128-row tile, group) items in tile order are cut into one
-// contiguous range per CTA (stream-K; shapes whose X operands do not fit in
-// shared memory are left to the GEMM).  The packed format stores the
-// 2 KB block of one (tile, group) contiguously per plane, items in this order,
-// so a run of items is one contiguous stream per plane: a producer warp copies
-// batches of items with bulk asynchronous copies into a ring of stages.  Two
-// teams of four warps take items in turn, each double-buffering A and D in
-// TMEM so that decoding the next item overlaps the tensor core and the
-// read-back of the previous one.  Partial sums of a tile are combined in a
-// fixed order; a tile shared with other CTAs goes through the workspace, the
-// last CTA to arrive summing every part in a fixed order.
+// contiguous range per CTA, row tiles being shared only by the CTAs of one
+// thread-block cluster (shapes whose X operand does not fit in shared memory
+// are left to the GEMM).  The packed format stores the 2 KB block of one
+// (tile, group) contiguously per plane, items in this order, so a run of
+// items is one contiguous stream per plane: a producer warp copies batches of
+// items with bulk asynchronous copies into a ring of stages.  Three teams of
+// four warps each take a pair of items per iteration: decode into registers,
+// wait for the MMAs of their previous pair, store the new A to TMEM, read the
+// previous D, meet at a team barrier, issue the MMAs and fold the previous
+// pair.  Partial sums of a tile are combined in a fixed order; a tile shared
+// by several CTAs of a cluster is summed by its owner from the parts the
+// others write into its shared memory.
 #include <string.h>
 
 #include <mutex>
@@ -362,7 +364,6 @@ struct Args {
     int M, NB, S;           // batch rows, MMA N (16 or 32), ring stages (multiple of kBatch)
     // shared-memory offsets from the 1024-byte aligned base
     uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_red, o_misc;
-    int ntile_max;          // largest number of row tiles a CTA touches
 };
 
 // ------------------------------------------------------------- X operand
@@ -964,8 +965,8 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
 }
 
 template <int R, int MT>
-mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, char *ws,
-              const Plan &p, cudaStream_t st) {
+mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, const Plan &p,
+              cudaStream_t st) {
     static bool attr_set = false;          // per instantiation
     cudaError_t e;
     if (!attr_set) {
@@ -989,7 +990,6 @@ mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, c
     a.S = p.S;
     a.o_ring = p.o_ring; a.o_sring = p.o_sring; a.o_b = p.o_b; a.o_pair = p.o_pair;
     a.o_res = p.o_res; a.o_bar = p.o_bar; a.o_red = p.o_red; a.o_misc = p.o_misc;
-    a.ntile_max = p.ntile;
     // programmatic dependent launch: this grid may start while the previous
     // kernel of the stream finishes; it waits for it before reading X
     cudaLaunchConfig_t cfg = {};
@@ -1044,12 +1044,12 @@ int occ_clusters_r(int64_t M, size_t smem, int cs) {
 }
 
 template <int R>
-mq_status run_r(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, char *ws,
-                const Plan &p, cudaStream_t st) {
-    if (M == 1) return run<R, 1>(X, wt, M, Y, ws, p, st);
-    if (M == 2) return run<R, 2>(X, wt, M, Y, ws, p, st);
-    if (M <= 4) return run<R, 4>(X, wt, M, Y, ws, p, st);
-    return run<R, 8>(X, wt, M, Y, ws, p, st);
+mq_status run_r(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, const Plan &p,
+                cudaStream_t st) {
+    if (M == 1) return run<R, 1>(X, wt, M, Y, p, st);
+    if (M == 2) return run<R, 2>(X, wt, M, Y, p, st);
+    if (M <= 4) return run<R, 4>(X, wt, M, Y, p, st);
+    return run<R, 8>(X, wt, M, Y, p, st);
 }
 
 int max_clusters(int r, int64_t M, size_t smem, int cs) {
@@ -1109,16 +1109,16 @@ mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint
     (void)ws_bytes;
     const Plan p = cached_plan(M, w->N, w->K, w->r);
     if (!p.ok) return fail(MQ_ERR_UNSUPPORTED, "no tensor-core GEMV plan fits this shape");
-    char *b = static_cast<char *>(ws);
+    (void)ws;
     switch (w->r) {
-        case 1: return run_r<1>(X, w, M, Y, b, p, st);
-        case 2: return run_r<2>(X, w, M, Y, b, p, st);
-        case 3: return run_r<3>(X, w, M, Y, b, p, st);
-        case 4: return run_r<4>(X, w, M, Y, b, p, st);
-        case 5: return run_r<5>(X, w, M, Y, b, p, st);
-        case 6: return run_r<6>(X, w, M, Y, b, p, st);
-        case 7: return run_r<7>(X, w, M, Y, b, p, st);
-        default: return run_r<8>(X, w, M, Y, b, p, st);
+        case 1: return run_r<1>(X, w, M, Y, p, st);
+        case 2: return run_r<2>(X, w, M, Y, p, st);
+        case 3: return run_r<3>(X, w, M, Y, p, st);
+        case 4: return run_r<4>(X, w, M, Y, p, st);
+        case 5: return run_r<5>(X, w, M, Y, p, st);
+        case 6: return run_r<6>(X, w, M, Y, p, st);
+        case 7: return run_r<7>(X, w, M, Y, p, st);
+        default: return run_r<8>(X, w, M, Y, p, st);
     }
 }
 

@@ -167,6 +167,16 @@ def test_llama_layers_full_m1(name, N, K, r, gemv_variant):
     assert _case(N, K, 1, r, seed) <= 1.0
 
 
+@pytest.mark.parametrize("r", [4, 2])
+@pytest.mark.parametrize("M", [2, 4, 8])
+@pytest.mark.parametrize("name,N,K", [l for l in LLAMA if l[0] in ("gate_proj", "down_proj", "k_proj")])
+def test_llama_layers_full_small_batch(name, N, K, M, r):
+    # full-size layers at M = 2..8 (GEMV batch classes 2, 4 and 8; clusters
+    # and whole-tile splits): every output against the oracle
+    seed = wl.layer_seed(2, [l[0] for l in LLAMA].index(name))
+    assert _case(N, K, M, r, seed) <= 1.0
+
+
 def test_workspace_shared_across_shapes():
     # a larger split-K call followed by a smaller one on the same workspace
     import torch
