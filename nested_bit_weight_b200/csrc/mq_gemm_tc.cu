@@ -147,14 +147,51 @@ gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ pla
     uint32_t phase = 0;
     bool ok = true;
 
+    // The next group's plane words, scale and X chunks are loaded into
+    // registers while the current group is decoded and multiplied (the loop
+    // is otherwise bound by the global-load latency of every group).
+    constexpr bool kPrefetch = R * 8 + BM <= 96;
+    constexpr int kXv = BM * 16 / kTcThreads;            // X chunks per thread (BM <= 32)
+    uint4 pvn[R];
+    float sn = 0.f;
+    uint4 xvn[kXv > 0 && BM <= 32 ? kXv : 1];
+    auto load_group = [&](int64_t g) {
+#pragma unroll
+        for (int p = 0; p < R; ++p)
+            pvn[p] = *reinterpret_cast<const uint4 *>(planes + p * plane_words +
+                                                      ((int64_t)blockIdx.x * G + g) * 512 + t * 4);
+        sn = __half2float(scales[((int64_t)blockIdx.x * G + g) * 128 + t]);
+        if constexpr (BM <= 32) {
+#pragma unroll
+            for (int i = 0; i < kXv; ++i) {
+                const int idx = t + i * kTcThreads, row = idx >> 4, c = idx & 15;
+                xvn[i] = *reinterpret_cast<const uint4 *>(Xp + (int64_t)(m0 + row) * K + g * kGroup + c * 8);
+            }
+        }
+    };
+    if (kPrefetch && gbeg < gend) load_group(gbeg);
+
     for (int64_t g = gbeg; g < gend; ++g) {
         // ---- decode this thread's row of the A tile
         uint4 pv[R];
+        float s;
+        uint4 xv[kXv > 0 && BM <= 32 ? kXv : 1];
+        if constexpr (kPrefetch) {
 #pragma unroll
-        for (int p = 0; p < R; ++p)
-            pv[p] = *reinterpret_cast<const uint4 *>(planes + p * plane_words +
-                                                     ((int64_t)blockIdx.x * G + g) * 512 + t * 4);
-        const float s = __half2float(scales[((int64_t)blockIdx.x * G + g) * 128 + t]);
+            for (int p = 0; p < R; ++p) pv[p] = pvn[p];
+            s = sn;
+            if constexpr (BM <= 32) {
+#pragma unroll
+                for (int i = 0; i < kXv; ++i) xv[i] = xvn[i];
+            }
+            if (g + 1 < gend) load_group(g + 1);
+        } else {
+#pragma unroll
+            for (int p = 0; p < R; ++p)
+                pv[p] = *reinterpret_cast<const uint4 *>(planes + p * plane_words +
+                                                         ((int64_t)blockIdx.x * G + g) * 512 + t * 4);
+            s = __half2float(scales[((int64_t)blockIdx.x * G + g) * 128 + t]);
+        }
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
             uint32_t P[8], E[8];
@@ -177,11 +214,19 @@ gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ pla
             }
         }
         // ---- stage the X tile (already in decode order)
-        for (int idx = t; idx < BM * 16; idx += kTcThreads) {
-            const int row = idx >> 4, c = idx & 15;
-            const uint4 v = *reinterpret_cast<const uint4 *>(
-                Xp + (int64_t)(m0 + row) * K + g * kGroup + c * 8);
-            *reinterpret_cast<uint4 *>(sB + (c >> 3) * (BM * 128) + sw128_offset(row, c & 7)) = v;
+        if constexpr (kPrefetch && BM <= 32) {
+#pragma unroll
+            for (int i = 0; i < kXv; ++i) {
+                const int idx = t + i * kTcThreads, row = idx >> 4, c = idx & 15;
+                *reinterpret_cast<uint4 *>(sB + (c >> 3) * (BM * 128) + sw128_offset(row, c & 7)) = xv[i];
+            }
+        } else {
+            for (int idx = t; idx < BM * 16; idx += kTcThreads) {
+                const int row = idx >> 4, c = idx & 15;
+                const uint4 v = *reinterpret_cast<const uint4 *>(
+                    Xp + (int64_t)(m0 + row) * K + g * kGroup + c * 8);
+                *reinterpret_cast<uint4 *>(sB + (c >> 3) * (BM * 128) + sw128_offset(row, c & 7)) = v;
+            }
         }
         fence_proxy_async_smem();
         __syncthreads();
