@@ -206,3 +206,29 @@ def test_no_device_wait_timed_out():
         X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
         mq.gemm(X, p, r)
     mq.mq_device_status()
+
+
+@pytest.mark.parametrize("name,N,K", [("gate_proj", 28672, 8192), ("down_proj", 8192, 28672)])
+def test_70b_layers_full(name, N, K):
+    # 70B-class shapes at M = 1, 8, 32 and r = 4, 2 (GEMV with clusters or
+    # whole tiles, the GEMM fallback where the X operand does not fit, and
+    # the GEMM): every output against the oracle
+    codes, s, _ = wl.gen_weights(N, K, wl.layer_seed(4, 4 if name == "gate_proj" else 6))
+    parent = None
+    for M in (1, 8, 32):
+        xbits, X = wl.gen_x(M, K, wl.layer_seed(4, 0) + M)
+        for r in (4, 2):
+            Y, parent = _run(codes, s, xbits, r, parent)
+            ratio = oracle.violation_ratio(Y, oracle.gemm(X, codes, s, r))
+            assert ratio <= 1.0, (M, r, ratio)
+
+
+@pytest.mark.parametrize("name,N,K,M", [("gate_proj", 12288, 4096, 64), ("q_proj", 4096, 4096, 128),
+                                        ("down_proj", 4096, 12288, 16)])
+def test_qwen_chain_outlier_x(name, N, K, M):
+    # Qwen3-8B chain: attention at r = 4, FFN at r = 3, X with x20 outlier channels
+    r = wl.QWEN3_R[name]
+    codes, s, _ = wl.gen_weights(N, K, wl.layer_seed(3, 0))
+    xbits, X = wl.gen_x(M, K, wl.layer_seed(3, 0) + M, outlier_channels=True)
+    Y, _ = _run(codes, s, xbits, r)
+    assert oracle.violation_ratio(Y, oracle.gemm(X, codes, s, r)) <= 1.0
