@@ -178,12 +178,16 @@ MQ_API mq_status mq_unpack(const mq_weights *w, uint8_t *codes_out, void *stream
  * convention, not part of the method.
  *   Arguments and results are those of mq_gemm without the workspace.
  *   Scratch: a 16 MiB array compiled into the library, resident on every GPU
- *   that loads it until the process exits.  Problems whose
- *   mq_gemm_workspace_bytes exceeds 16 MiB return MQ_ERR_WORKSPACE; M > 8
- *   returns MQ_ERR_INVALID_ARG.  Both checks happen before any launch.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture.  Each call clears the array's arrival tickets (one
+ *   that loads it until the process exits.  The call runs the kernel
+ *   mq_gemm would run for M <= 8: the tensor-core GEMV needs no scratch; the
+ *   GEMM (shapes the GEMV does not take, or the MQ_GEMV_VIA_GEMM variant)
+ *   keeps its split-K partial sums, its X operand and its arrival tickets in
+ *   the array.  A problem whose kernel needs more than 16 MiB of scratch
+ *   returns MQ_ERR_WORKSPACE; M > 8 returns MQ_ERR_INVALID_ARG.  Both checks
+ *   happen before any launch.  The first call on a device that takes the
+ *   GEMM looks up the array's device address (once per device, with that
+ *   device current); make that first call before any stream capture.  Each
+ *   call that takes the GEMM clears the array's arrival tickets (one
  *   cudaMemsetAsync on `stream`) and overwrites the rest.
  *   All calls share the one array, which keeps the last call's contents:
  *   calls that can overlap on the GPU (other streams, other host threads)

@@ -81,10 +81,14 @@ mq_status check_weights(const mq_weights *w, int64_t N, int64_t K) {
     return MQ_OK;
 }
 
+bool small_m_uses_gemv(int64_t M, int64_t N, int64_t K, int r) {
+    return __atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) == MQ_GEMV_TC &&
+           gemv_tc_supported(M, N, K, r);
+}
+
 mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
                          void *ws, size_t ws_bytes, cudaStream_t st) {
-    if (__atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) == MQ_GEMV_TC &&
-        gemv_tc_supported(M, w->N, w->K, w->r))
+    if (small_m_uses_gemv(M, w->N, w->K, w->r))
         return launch_gemv_tc(X, w, M, Y, ws, ws_bytes, st);
     return launch_gemm_tc(X, w, M, Y, ws, ws_bytes, st);
 }

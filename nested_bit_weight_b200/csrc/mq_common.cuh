@@ -47,6 +47,8 @@ mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M,
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M,
                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);
+// Whether an M <= 8 call takes the tensor-core GEMV (variant and shape).
+bool small_m_uses_gemv(int64_t M, int64_t N, int64_t K, int r);
 // The M <= 8 product with the kernel chosen by mq_set_gemv_variant.
 mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M,
                          uint16_t *Y, void *ws, size_t ws_bytes, cudaStream_t st);

@@ -252,7 +252,7 @@ gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ pla
 #pragma unroll
         for (int cb = 0; cb < BM / 16; ++cb) {
             float v[16];
-            tmem_ld16(taddr + ((uint32_t)(32 * warp) << 16) + cb * 16, v);
+            { uint32_t u[16]; tmem_ld16(taddr + ((uint32_t)(32 * warp) << 16) + cb * 16, u); for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(u[q]); }
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 16; ++i) y[cb * 16 + i] = fmaf(s, v[i], y[cb * 16 + i]);

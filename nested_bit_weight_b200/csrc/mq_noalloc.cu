@@ -5,9 +5,10 @@
 // and exposes no allocator, serving processes that hand the whole GPU to
 // their own pool at start-up, and latency-critical loops that cannot take
 // cudaMalloc's implicit device synchronisation.  They can still call this
-// entry point: its scratch (split-K partial sums, the X operand fragments and
-// the arrival tickets) lives in a fixed array compiled into the library
-// instead of a workspace they would have to provide.
+// entry point: its scratch (the X operand of the call, and for the GEMM route
+// the split-K partial sums and arrival tickets) lives in a fixed array
+// compiled into the library instead of a workspace they would have to
+// provide.
 #include "mq_common.cuh"
 
 namespace mq {
@@ -36,13 +37,18 @@ extern "C" mq_status mq_gemv_noalloc(const uint16_t *X, const mq_weights *w, int
     if (!X || !Y) return fail(MQ_ERR_INVALID_ARG, "X or Y is NULL");
     if (!aligned16(X) || !aligned16(Y))
         return fail(MQ_ERR_MISALIGNED, "X and Y must be 16-byte aligned");
-    const size_t need = mq_gemm_workspace_bytes(M, N, K, w->r);
+    // the kernel this call will run, and the scratch that kernel needs (the
+    // tensor-core GEMV: its X operand; the GEMM: its split-K partial sums,
+    // its X operand and its arrival tickets)
+    cudaStream_t st = (cudaStream_t)stream;
+    if ((s = bind_device(st)) != MQ_OK) return s;
+    const bool gemv = small_m_uses_gemv(M, N, K, w->r);
+    const size_t need = gemv ? gemv_tc_workspace_bytes(M, N, K, w->r)
+                             : gemm_tc_workspace_bytes(M, N, K, w->r);
     if (need > kNoAllocBytes)
         return fail(MQ_ERR_WORKSPACE,
                     "problem needs more scratch than the 16 MiB built into mq_gemv_noalloc; "
                     "use mq_gemm with a workspace");
-    cudaStream_t st = (cudaStream_t)stream;
-    if ((s = bind_device(st)) != MQ_OK) return s;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
@@ -54,8 +60,11 @@ extern "C" mq_status mq_gemv_noalloc(const uint16_t *X, const mq_weights *w, int
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
         __atomic_store_n(&g_scratch_addr[dev], scratch, __ATOMIC_RELEASE);
     }
-    // the arrival tickets must start at zero whatever an earlier call left
+    // the tensor-core GEMV keeps the X operand of the call in the scratch
+    if (gemv) return launch_gemv_tc(X, w, M, Y, scratch, kNoAllocBytes, st);
+    // the GEMM's arrival tickets must start at zero whatever an earlier call
+    // (or one that gave up on a wait) left there
     e = cudaMemsetAsync(scratch, 0, kTicketBytes, st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
-    return launch_small_m(X, w, M, Y, scratch, kNoAllocBytes, st);
+    return launch_gemm_tc(X, w, M, Y, scratch, kNoAllocBytes, st);
 }
