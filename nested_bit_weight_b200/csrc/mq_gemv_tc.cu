@@ -10,7 +10,7 @@
 // with S_g = sum_k x_k.  The tensor core computes sum_k x_k q_k exactly:
 //
 // * A (M = 128 weight rows x K = 128 columns of one group, unsigned 8-bit, in
-//   TMEM).  A thread of a decode warp owns one row: it reads the row's r
+//   TMEM).  Each thread of a 4-warp team owns one row: it reads the row's r
 //   plane words of the group (16 bytes per plane), turns every 32-column word
 //   into 8 registers whose bytes are fields q << sh(i) (one AND per register,
 //   sh = the field's bit offset in its byte), and stores the 32 registers to
@@ -21,42 +21,24 @@
 //   four int8 slices relative to the group exponent Eg = max floor(log2|z|):
 //       z_k = 2^(Eg-27) (a_1 2^21 + a_2 2^14 + a_3 2^7 + a_4),
 //   exact for every x within 2^-20 of the group's largest; column 4m + j at
-//   k = 32t + 4i + b holds slice j of z at column 32t + 8b + i.  A small
-//   kernel builds the slices of every group once per call (x_prep_kernel);
-//   each CTA then copies the tiles of its groups into shared memory.
+//   k = 32t + 4i + b holds slice j of z at column 32t + 8b + i.
 // * D (128 x N, int32, TMEM) = exact per-group integer sums, read back with
 //   tcgen05.ld and folded into fp32: y += s_g 2^(8-r) 2^(Eg-6) sum_j 2^(-7j) D_j
 //   + s_g (2^(7-r) - 128) S_g.
 //
 // Work: the (128-row tile, group) items in tile order are cut into one
 // contiguous range per CTA, row tiles being shared only by the CTAs of one
-// thread-block cluster (shapes whose operands do not fit in shared memory
+// thread-block cluster (shapes whose X operand does not fit in shared memory
 // are left to the GEMM).  The packed format stores the 2 KB block of one
 // (tile, group) contiguously per plane, items in this order, so a run of
-// items is one contiguous stream per plane.
-//
-// Roles (warp-specialised, every hand-off an mbarrier or a shared atomic,
-// no CTA-wide barrier in the steady state):
-//   producer warp   bulk copies of the planes and scales of batches of
-//                   items into two rings of shared-memory stages;
-//   8 decode warps  two quads; quad e decodes items e, e + 2, ...: warp q of
-//                   a quad owns rows 32q .. 32q + 31 (its TMEM lane quarter)
-//                   and stores the item's A into one of eight TMEM A slots;
-//                   the last of the four warps to finish an item (a counter
-//                   per A slot) issues the item's four K = 32 MMAs into one
-//                   of the TMEM D slots and commits to the D slot's barrier
-//                   (D full; the A slot is free again once it lands);
-//   4 fold warps    one copies the X tiles of the CTA's groups (after the
-//                   kernels before it in the stream have completed:
-//                   programmatic dependent launch); all four then fold the D
-//                   slots, several items per round, into fp32 rows and
-//                   write Y (or send a shared tile's part to its owner).
-// The producer and decode warps read only the weights, so with programmatic
-// dependent launch they stream and decode while the kernels before it are
-// still finishing.  Waiting warps back off between polls, leaving the issue
-// slots to the warps doing the work.  Every wait is bounded (about a second);
-// a wait that gives up sets a CTA abort flag that ends every other wait at
-// once, and a device flag the host reads with mq_device_status.
+// items is one contiguous stream per plane: a producer warp copies batches of
+// items with bulk asynchronous copies into a ring of stages.  Three teams of
+// four warps each take a pair of items per iteration: decode into registers,
+// wait for the MMAs of their previous pair, store the new A to TMEM, read the
+// previous D, meet at a team barrier, issue the MMAs and fold the previous
+// pair.  Partial sums of a tile are combined in a fixed order; a tile shared
+// by several CTAs of a cluster is summed by its owner from the parts the
+// others write into its shared memory.
 #include <string.h>
 
 #include <atomic>
@@ -71,19 +53,15 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kDecWarps = 8;                 // two quads of decode warps
-constexpr int kFoldW0 = kDecWarps;           // fold warps kFoldW0 .. kFoldW0 + 3
-constexpr int kProdWarp = kFoldW0 + 4;
-constexpr int kThreads = (kProdWarp + 1) * 32;
-constexpr int kB = 2;                        // items per ring batch (one per quad)
-constexpr int kNA = 8;                       // A slots in TMEM (32 columns each)
-constexpr uint32_t kTmemCols = 512;          // A slots in [0, 256), D slots in [256, 512)
-constexpr uint32_t kDCol0 = 256;
+constexpr int kTeams = 3;                    // teams of 4 warps (128 rows)
+constexpr int kCW = 4 * kTeams;              // consumer warps
+constexpr int kProd = kCW;                   // producer warp
+constexpr int kThreads = (kCW + 1) * 32;
+constexpr int kBatch = 2 * kTeams;           // items per bulk copy: one pair per team
 constexpr int kSlices = 4;                   // int8 slices per x
+constexpr int kHeadBatches = 2;              // batches streamed before X is requested
+constexpr uint32_t kTmemCols = 512;          // TMEM columns per CTA (one CTA per SM)
 constexpr size_t kSmemMax = 227 * 1024;      // shared memory of one CTA per SM
-constexpr size_t kRingBytes = 144 * 1024;    // plane ring budget
-constexpr uint32_t kPlaneBlk = 2048;         // one (tile, group) block of one plane
-constexpr size_t kXOff = kTicketBytes;       // prepared X in the workspace (after the GEMM's tickets)
 
 // ------------------------------------------------------------ operand decode
 // Bit offset of register i's field inside each byte (the byte holds q << sh).
@@ -125,9 +103,60 @@ __device__ __forceinline__ void field_operands(const uint32_t (&P)[8], uint32_t 
     }
 }
 
+// ------------------------------------------------------ barriers and copies
+// (mbarrier, bulk-copy, cluster and tcgen05 wrappers shared by every kernel
+// of the library are in mq_sm100.cuh)
 __device__ unsigned int g_gemv_timeout;     // set when a bounded wait gave up
 
-// ------------------------------------------------------------- decomposition
+// Suspending variant for the producer, which waits long and is not on the
+// per-item critical path: the thread sleeps in try_wait instead of spinning
+// (spinning would take issue slots from the decoding warps).
+__device__ __forceinline__ bool bar_try_sleep(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 2000;\n"
+                 " selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool bar_wait_sleep(uint64_t *b, uint32_t parity) {
+    const uint64_t t0 = global_ns();
+    while (!bar_try_sleep(b, parity))
+        if (global_ns() - t0 > kWaitNs) return false;
+    return true;
+}
+// Wait for the phase of parity `parity` to complete by polling (a suspended
+// try_wait can resume well after the phase completes, which the per-item
+// hand-offs of this kernel cannot afford); gives up after about a second.
+__device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) { return mbar_wait_bounded(b, parity); }
+__device__ __forceinline__ void st_release(int *p, int v) {
+    asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+// test_wait with cluster-scope acquire (parts written by other CTAs).
+__device__ __forceinline__ bool bar_try_cluster(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n .reg .pred p;\n"
+                 " mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+                 " selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
+    return ok != 0;
+}
+// Named barrier that also returns the AND of `v` over its threads, so that a
+// whole team takes the same branch after a wait that may have timed out.
+__device__ __forceinline__ bool named_sync_and(int id, int n, bool v) {
+    uint32_t r;
+    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 q, %2, 0;\n"
+                 " bar.red.and.pred p, %1, %3, q;\n selp.u32 %0, 1, 0, p;\n}"
+                 : "=r"(r) : "r"(id), "r"((uint32_t)v), "r"(n) : "memory");
+    return r != 0;
+}
+
+// ------------------------------------------------------------ decomposition
 // Items u = 0 .. W-1, W = T * KC (T 128-row tiles, KC = K / 128 groups), in
 // (tile, group) order; CTA b owns the contiguous items [first(b), first(b+1)).
 // Clusters: the row tiles are cut into NC contiguous runs, one per cluster of
@@ -167,58 +196,27 @@ __host__ __device__ inline Range make_range(const Work &w, int64_t b) {
     r.L = r.u1 - r.u0;
     return r;
 }
-
-// Batch class MT (M = 1, 2, <= 4, <= 8): MMA N and groups per B tile.  The
-// slices of group g sit in B tile g / gpb at position g % gpb (rows
-// 4 (pos M + m) + j), and fill D columns 4 (pos M + m) + j.
-__host__ __device__ constexpr int class_nb(int MT) { return MT <= 4 ? 16 : 32; }
-__host__ __device__ constexpr int class_gpb(int MT) { return MT == 1 ? 4 : MT == 2 ? 2 : 1; }
-__host__ __device__ inline int batch_class(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 4 ? 4 : 8; }
-// Items folded per round by a fold warp (D registers: 4 MT per item).
-__host__ __device__ constexpr int fold_chunk(int MT) { return MT <= 2 ? 4 : MT == 4 ? 2 : 1; }
-
-// The CTA's groups g0 .. g0 + nslot - 1 (mod G) as B tiles: the tiles of
-// groups g0 .. min(gend, G - 1) first (na of them), then, when the range
-// wraps past the last group, the tiles of groups 0 .. gend - G.
-struct XSpan {
-    int g0, nslot, ta0, na, nb;
-    __host__ __device__ XSpan(int g0_, int nslot_, int G, int gpb) : g0(g0_), nslot(nslot_) {
-        const int gend = g0 + nslot - 1;
-        ta0 = g0 / gpb;
-        na = (gend < G ? gend : G - 1) / gpb - ta0 + 1;
-        nb = gend >= G ? (gend - G) / gpb + 1 : 0;
-    }
-    // shared-memory tile of group g (one of the CTA's groups)
-    __host__ __device__ int tile_of(int g, int gpb) const { return g >= g0 ? g / gpb - ta0 : na + g / gpb; }
-};
+// Group held by X slot `slot` of the CTA (slots count groups from the group
+// of the CTA's first item, modulo KC).
+__host__ __device__ inline int slot_chunk(const Work &w, const Range &r, int slot) {
+    const int KC = (int)w.KC;
+    const int c = r.u0 % KC + slot;
+    return c >= KC ? c - KC : c;
+}
 
 // Kernel arguments (one struct, passed as a grid constant).
 struct Args {
+    const __nv_bfloat16 *X;
     const uint8_t *planes;  // tiled planes (2 KB per (tile, group) block per plane)
     const uint8_t *scales;  // tiled fp16 scales (256 B per block)
-    const uint8_t *xtiles;  // prepared X: B tiles of all groups (workspace)
-    const float2 *xpairs;   // prepared X: {2^(8-r) 2^(Eg-6), S_g} per (group, m), 8 per group
     __nv_bfloat16 *Y;
     Work w;
     int64_t N, K, G;
     int64_t plane_bytes;    // bytes of one plane
-    int M;                  // batch rows
-    int nring, nss;         // batches in the plane ring / the scale ring
+    int M, NB, S;           // batch rows, MMA N (16 or 32), ring stages (multiple of kBatch)
     // shared-memory offsets from the 1024-byte aligned base
-    uint32_t o_ring, o_sring, o_b, o_pair, o_bar, o_red, o_misc;
+    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_red, o_misc;
 };
-
-// Shared-memory barriers of one CTA, in the order they are laid out.
-struct Bars {
-    uint64_t *full, *empty;     // [nring] plane ring
-    uint64_t *sfull, *sempty;   // [nss] scale ring
-    uint64_t *dfull, *dempty;   // [kND] TMEM D slots
-    uint64_t *rbar;             // parts of the owned shared tile received
-    uint64_t *xbar;             // the CTA's X tiles and pairs landed
-};
-__host__ __device__ inline int bar_count(int nring, int nss, int nd) {
-    return 2 * nring + 2 * nss + 2 * nd + 2;
-}
 
 // ------------------------------------------------------------- X operand
 // Fixed-point value F = z 2^(27 - Ez), z = x 2^(-sh), truncated toward zero;
@@ -239,426 +237,473 @@ __device__ __forceinline__ uint32_t pack_bytes(int v0, int v1, int v2, int v3) {
     return __byte_perm(lo, hi, 0x5410);
 }
 
-constexpr int kPrepWarps = 8;
-
-// The B operand of every group, once per call: one warp per (group, batch
-// row) task.  Writes B tile g / gpb (row 4 (pos M + m) + j, K-major with the
-// 128-byte swizzle, ready to be copied into shared memory as is) and the
-// pair {2^(8-r) 2^(Eg-6), S_g} at pairs[g * 8 + m].
-template <int R, int MT>
-__global__ void __launch_bounds__(kPrepWarps * 32)
-x_prep_kernel(const uint16_t *__restrict__ X, int M, int64_t K, int G, uint8_t *__restrict__ tiles,
-              float2 *__restrict__ pairs) {
-    constexpr int NB = class_nb(MT), gpb = class_gpb(MT);
-    pdl_launch_dependents();            // the GEMV may start streaming its weights
-    pdl_wait();                         // X comes from the kernels before this one
-    const int lane = threadIdx.x & 31;
-    const int task = blockIdx.x * kPrepWarps + (threadIdx.x >> 5);
-    if (task >= G * M) return;
-    const int g = task / M, m = task - g * M;
+// X operand of the CTA's groups, built by the team warps.  Slot sl (the
+// sl-th distinct group of the range) lives in B tile sl / gpb at position
+// pos = sl % gpb (gpb = groups per tile): MMA column 4 (pos M + m) + j holds
+// slice j of batch row m, K-major with the 128-byte swizzle; the pair
+// {2^(8-r) 2^(Eg-6), S_g} of (slot, m) at pairs[sl * 8 + m].  X is staged
+// first with one round of 16-byte copies (staging[sl][m][128 values]).
+template <int R>
+__device__ void build_x_operand(const Args &a, uint8_t *smem, const Work &w, const Range &rg,
+                                int nslot, int *flags) {
+    constexpr int kPrep = kCW * 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int M = a.M, gpb = a.NB == 16 ? (M == 1 ? 4 : M == 2 ? 2 : 1) : 1;
     const int t = lane >> 3, wi = lane & 7;
     const int sh = field_shift<R>(wi);
-    const uint16_t *xr = X + (int64_t)m * K + (int64_t)g * kGroup + 32 * t + wi;
-    uint32_t hv[4];
+    float2 *pairs = reinterpret_cast<float2 *>(smem + a.o_pair);
+    // the warp's tasks (slot, m) in chunks of 4: all loads of a chunk first
+    const uint16_t *X = reinterpret_cast<const uint16_t *>(a.X);
+    for (int t0 = warp; t0 < nslot * M; t0 += 4 * kCW) {
+        uint32_t hv[4][4];
 #pragma unroll
-    for (int b = 0; b < 4; ++b) hv[b] = xr[8 * b];
-    int emax = -1000;
-    float sum = 0.f;
+        for (int c = 0; c < 4; ++c) {
+            const int task = t0 + c * kCW;
+            if (task < nslot * M) {
+                const int sl = task / M, m = task - sl * M;
+                const uint16_t *xr = X + (int64_t)m * a.K + (int64_t)slot_chunk(w, rg, sl) * kGroup + 32 * t + wi;
 #pragma unroll
-    for (int b = 0; b < 4; ++b) {
-        const int e8 = (int)((hv[b] >> 7) & 0xFFu);
-        const int v = e8 ? e8 - sh : -1000;
-        emax = v > emax ? v : emax;
-        sum += __uint_as_float(hv[b] << 16);
+                for (int b = 0; b < 4; ++b) hv[c][b] = xr[8 * b];
+            }
+        }
+        if (t0 == 0 && lane == 0) st_release(&flags[2], (int)(hv[0][0] | 1u));   // X fetched: stream the rest
+        // the four tasks side by side (independent chains; absent tasks are
+        // computed on zeros and not stored)
+        int emax[4];
+        float sum[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            emax[c] = -1000;
+            sum[c] = 0.f;
+            if (t0 + c * kCW >= nslot * M) {
+#pragma unroll
+                for (int b = 0; b < 4; ++b) hv[c][b] = 0u;
+            }
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+                const int e8 = (int)((hv[c][b] >> 7) & 0xFFu);
+                const int v = e8 ? e8 - sh : -1000;
+                emax[c] = v > emax[c] ? v : emax[c];
+                sum[c] += __uint_as_float(hv[c][b] << 16);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int other = __shfl_xor_sync(0xffffffffu, emax[c], o);
+                emax[c] = other > emax[c] ? other : emax[c];
+                sum[c] += __shfl_xor_sync(0xffffffffu, sum[c], o);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int task = t0 + c * kCW;
+            if (task >= nslot * M) break;
+            const int sl = task / M, m = task - sl * M;
+            const int Eg = emax[c] > -1000 ? emax[c] - 127 : 0;
+            int F[4];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) F[b] = fixed_point(hv[c][b], sh, Eg);
+            uint32_t wd[kSlices];
+            wd[0] = pack_bytes(F[0] >> 21, F[1] >> 21, F[2] >> 21, F[3] >> 21);
+            wd[1] = pack_bytes(F[0] >> 14, F[1] >> 14, F[2] >> 14, F[3] >> 14) & 0x7F7F7F7Fu;
+            wd[2] = pack_bytes(F[0] >> 7, F[1] >> 7, F[2] >> 7, F[3] >> 7) & 0x7F7F7F7Fu;
+            wd[3] = pack_bytes(F[0], F[1], F[2], F[3]) & 0x7F7F7F7Fu;
+            uint8_t *tile = smem + a.o_b + (size_t)(sl / gpb) * a.NB * 128;
+            const int chunk = 2 * t + (wi >> 2);           // 16-byte chunk of k = 32t + 4wi
+#pragma unroll
+            for (int j = 0; j < kSlices; ++j) {
+                const int row = 4 * ((sl % gpb) * M + m) + j;
+                *reinterpret_cast<uint32_t *>(tile + (row >> 3) * 1024 + (row & 7) * 128 +
+                                              ((chunk ^ (row & 7)) << 4) + 4 * (wi & 3)) = wd[j];
+            }
+            if (lane == 0) {
+                // 2^(8-r) 2^(Eg-6), clamped to the normal fp32 range
+                int ex = 2 - R + Eg;
+                ex = ex < -126 ? -126 : (ex > 127 ? 127 : ex);
+                pairs[sl * 8 + m] = make_float2(__int_as_float((ex + 127) << 23), sum[c]);
+            }
+        }
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        const int other = __shfl_xor_sync(0xffffffffu, emax, o);
-        emax = other > emax ? other : emax;
-        sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    }
-    const int Eg = emax > -1000 ? emax - 127 : 0;
-    int F[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) F[b] = fixed_point(hv[b], sh, Eg);
-    uint32_t wd[kSlices];
-    wd[0] = pack_bytes(F[0] >> 21, F[1] >> 21, F[2] >> 21, F[3] >> 21);
-    wd[1] = pack_bytes(F[0] >> 14, F[1] >> 14, F[2] >> 14, F[3] >> 14) & 0x7F7F7F7Fu;
-    wd[2] = pack_bytes(F[0] >> 7, F[1] >> 7, F[2] >> 7, F[3] >> 7) & 0x7F7F7F7Fu;
-    wd[3] = pack_bytes(F[0], F[1], F[2], F[3]) & 0x7F7F7F7Fu;
-    uint8_t *tile = tiles + (size_t)(g / gpb) * NB * 128;
-    const int chunk = 2 * t + (wi >> 2);                 // 16-byte chunk of k = 32t + 4wi
-#pragma unroll
-    for (int j = 0; j < kSlices; ++j) {
-        const int row = 4 * ((g % gpb) * M + m) + j;
-        *reinterpret_cast<uint32_t *>(tile + sw128_offset(row, chunk) + 4 * (wi & 3)) = wd[j];
-    }
-    if (lane == 0) {
-        // 2^(8-r) 2^(Eg-6), clamped to the normal fp32 range
-        int ex = 2 - R + Eg;
-        ex = ex < -126 ? -126 : (ex > 127 ? 127 : ex);
-        pairs[(size_t)g * 8 + m] = make_float2(__int_as_float((ex + 127) << 23), sum);
-    }
+    // the tensor core reads B through the async proxy
+    fence_proxy_async_smem();
+    named_sync(1, kPrep);
 }
 
 // ------------------------------------------------------------------ kernel
-// D columns of one item (4 slices per batch row) into registers.
+// D columns of one item (4 slices per batch row, 4 MT registers) into registers.
 template <int MT>
-__device__ __forceinline__ void read_d(uint32_t taddr, uint32_t *d) {
-    if constexpr (MT == 1) tmem_ld4(taddr, d);
-    else if constexpr (MT == 2) tmem_ld8(taddr, d);
-    else if constexpr (MT == 4) tmem_ld16(taddr, d);
-    else tmem_ld32(taddr, d);
+__device__ __forceinline__ void read_d(uint32_t taddr, int *d) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(d);
+    if constexpr (MT == 1) tmem_ld4(taddr, u);
+    else if constexpr (MT == 2) tmem_ld8(taddr, u);
+    else if constexpr (MT == 4) tmem_ld16(taddr, u);
+    else tmem_ld32(taddr, u);
 }
 
-// Shared-memory atomic add with acquire-release order (a counter that also
-// hands over the tensor-memory stores of the warps that counted before).
-__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t *p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;"
-                 : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
-    return old;
-}
+// Fold one item's D into y (row `row` of the team's current tile); on a tile
+// change the finished tile's sums go to res first.
+#define FOLD_ITEM(D, SC, SLOT, LTILE)                                                      \
+    do {                                                                                   \
+        if ((LTILE) != cur) {                                                              \
+            if (cur >= 0) {                                                                \
+                _Pragma("unroll") for (int m = 0; m < MT; ++m) if (m < M)                  \
+                    res[((team * ntile + cur) * M + m) * 128 + row] = y[m];                \
+            }                                                                              \
+            _Pragma("unroll") for (int m = 0; m < MT; ++m) y[m] = 0.f;                     \
+            cur = (LTILE);                                                                 \
+        }                                                                                  \
+        _Pragma("unroll") for (int m = 0; m < MT; ++m) {                                   \
+            if (m < M) {                                                                   \
+                const float v = (float)(D)[4 * m] + 0x1p-7f * (float)(D)[4 * m + 1] +      \
+                                0x1p-14f * (float)(D)[4 * m + 2] +                         \
+                                0x1p-21f * (float)(D)[4 * m + 3];                          \
+                const float2 ge = pairs[(SLOT) * 8 + m];                                   \
+                y[m] = fmaf((SC) * ge.x, v, fmaf((SC) * kOffset, ge.y, y[m]));             \
+            }                                                                              \
+        }                                                                                  \
+    } while (0)
 
-// MT: batch class (M = 1, M = 2, M <= 4, M <= 8), fixing the MMA N (16 or 32),
-// the groups per B tile and the D columns read back per item.
+// MT: batch class (M = 1, M = 2, M <= 4, M <= 8), fixing the MMA N (16 or 32)
+// and the D columns read back per item.
 template <int R, int MT>
 __global__ void __launch_bounds__(kThreads, 1)
 nested_gemv_tc_kernel(const __grid_constant__ Args a) {
-    constexpr int NB = class_nb(MT), gpb = class_gpb(MT), CH = fold_chunk(MT);
-    constexpr int kND = 256 / NB;                        // D slots in TMEM
-    static_assert(kND >= kNA, "a decode warp waits on the D slot of the item kNA earlier");
+    constexpr uint32_t kPlaneBlk = 2048;                // one (tile, group) block of one plane
     extern __shared__ uint8_t smem_raw[];
     // align the base by an offset so the compiler keeps the shared address space
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *smem = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
     const Work &w = a.w;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const Range rg = make_range(w, blockIdx.x);
-    const int L = rg.L, M = a.M, G = (int)a.G;
-    const int nring = a.nring, nss = a.nss;
-    const int g0 = rg.u0 % G;
-    const int nslot = L < G ? L : G;                     // distinct groups of the range
-    const XSpan xs(g0, nslot, G, gpb);
-    const int tf = rg.u0 / G, tl = (rg.u1 - 1) / G;      // first and last row tile
+    const int L = rg.L, S = a.S, M = a.M, G = (int)a.G;
+    const int nbs = S / kBatch;                          // batch slots in the ring
+    const int nbatch = (L + kBatch - 1) / kBatch;
+    const int64_t tf = rg.u0 / G;                        // first tile of the range
+    const int ntile = (int)((rg.u1 - 1) / G - tf + 1);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + a.o_bar);
+    uint64_t *empty = full + nbs;
+    uint64_t *dfull = empty + nbs;                       // [team]: the pair's MMAs done
+    uint64_t *rbar = dfull + kTeams;                     // [tile]: parts of the tile received
+    // parts of the split tiles this CTA owns: [tile][contributor][m][128]
+    float *red = reinterpret_cast<float *>(smem + a.o_red);
+    int *flags = reinterpret_cast<int *>(smem + a.o_misc);   // [0] error [1] batches issued [2] X asked
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + a.o_misc + 16);
+    float *res = reinterpret_cast<float *>(smem + a.o_res);  // [team][tile][m][128]
+    const int nslot = (int)(L < G ? L : G);
 
-    Bars bar;
-    bar.full = reinterpret_cast<uint64_t *>(smem + a.o_bar);
-    bar.empty = bar.full + nring;
-    bar.sfull = bar.empty + nring;
-    bar.sempty = bar.sfull + nss;
-    bar.dfull = bar.sempty + nss;
-    bar.dempty = bar.dfull + kND;
-    bar.rbar = bar.dempty + kND;
-    bar.xbar = bar.rbar + 1;
-    volatile int *flags = reinterpret_cast<volatile int *>(smem + a.o_misc);   // [0] abort [1] batches issued
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + a.o_misc + 8);
-    uint32_t *acnt = reinterpret_cast<uint32_t *>(smem + a.o_misc + 16);      // [kNA] warps done per A slot
-    uint32_t *icnt = acnt + kNA;                                               // [kND] commits per D slot
-    float *red = reinterpret_cast<float *>(smem + a.o_red);    // [CS][M][128] parts of the owned tile
-
-    // The CTA holding a tile's first item owns it; if its last tile continues
-    // in later CTAs (of the same cluster), it waits for their parts.
-    const bool owns_shared = tl * G >= rg.u0 && tl * G + G > rg.u1;
-    const int own_nc = owns_shared ? (int)(w.cta_of((int64_t)tl * G + G - 1) - blockIdx.x + 1) : 0;
-
-    {
-        const int nb = bar_count(nring, nss, kND);
-        for (int i = threadIdx.x; i < nb; i += kThreads) {
-            uint32_t cnt;
-            if (i < nring) cnt = 1;                                          // full
-            else if (i < 2 * nring) cnt = 4 * kB;                            // empty: decode warps per item
-            else if (i < 2 * nring + nss) cnt = 1;                           // sfull
-            else if (i < 2 * nring + 2 * nss) cnt = 4;                       // sempty: fold warps
-            else if (i < 2 * nring + 2 * nss + kND) cnt = 1;                 // dfull: commit
-            else if (i < 2 * nring + 2 * nss + 2 * kND) cnt = 4;             // dempty: fold warps
-            else if (i == 2 * nring + 2 * nss + 2 * kND)
-                cnt = own_nc > 1 ? 128u * (uint32_t)(own_nc - 1) : 1u;       // rbar: sender threads
-            else cnt = 1;                                                    // xbar
-            mbar_init(bar.full + i, cnt);
-        }
-        if (threadIdx.x < kNA + kND) acnt[threadIdx.x] = 0;
-        if (threadIdx.x == 0) { flags[0] = 0; flags[1] = 0; }
-    }
+    // a batch of 4 items = one pair per team; each team warp frees it once
+    if (threadIdx.x < 2 * nbs) mbar_init(full + threadIdx.x, threadIdx.x < nbs ? 1u : 4u * kTeams);
+    // one commit per MMA issuer of a pair (kIssuers threads per team)
+    if (threadIdx.x < kTeams) mbar_init(dfull + threadIdx.x, (uint32_t)(MT <= 2 ? 4 : 2));
+    // The CTA holding a tile's first item owns it; if the tile continues in
+    // later CTAs (of the same cluster), it waits for their parts.
+    const int64_t tl = (rg.u1 - 1) / G;                  // last tile of the range
+    const int64_t own_last = (tl * G >= rg.u0 && tl * G + G > rg.u1) ? tl : -1;
+    const int own_nc = own_last >= 0 ? (int)(w.cta_of(own_last * G + G - 1) - blockIdx.x + 1) : 0;
+    if (threadIdx.x == 0 && own_nc > 1) mbar_init(rbar + (own_last - tf), (uint32_t)(own_nc - 1));
+    if (threadIdx.x == 0) { flags[0] = 0; flags[1] = 0; flags[2] = 0; }
+    for (int i = threadIdx.x; i < kTeams * ntile * M * 128; i += kThreads) res[i] = 0.f;
     fence_mbar_init();
     __syncthreads();
     // every CTA of the cluster has initialised its barriers before any part is sent
     if (w.CS > 1) cluster_arrive();
-    bool cluster_waited = false;
 
-    if (warp == kProdWarp) {
+    if (warp == kProd) {
         // ---------------------------------------------------------- producer
-        // batch b = items [kB b, kB b + kB): one bulk copy per plane and one
-        // for the scales (consecutive items are consecutive blocks), into
-        // plane ring slot b % nring and scale ring slot b % nss
+        // batch b = items [4b, 4b + 4): one bulk copy per plane and one for the
+        // scales (consecutive items are consecutive blocks), into ring slot b % nbs
         if (lane == 0) {
-            const int nbatch = (L + kB - 1) / kB;
-            int s = 0, ks = 0, ss = 0, kss = 0;
-            for (int b = 0; b < nbatch; ++b) {
-                if (ks > 0 && !mbar_wait_backoff(bar.empty + s, (uint32_t)(ks - 1) & 1u, flags)) break;
-                if (kss > 0 && !mbar_wait_backoff(bar.sempty + ss, (uint32_t)(kss - 1) & 1u, flags)) break;
-                const int i0 = b * kB, n = (L - i0) < kB ? (L - i0) : kB;
+            bool ok = true;
+            for (int b = 0; b < nbatch && ok; ++b) {
+                if (b == kHeadBatches) {
+                    // the next call may start; and X should not queue behind the rest
+                    pdl_launch_dependents();
+                    const uint64_t t0 = global_ns();
+                    while (ld_acquire(&flags[2]) == 0 && ok) {
+                        if (global_ns() - t0 > kWaitNs) ok = false;
+                        __nanosleep(128);
+                    }
+                    if (!ok) break;
+                }
+                const int bs = b % nbs;
+                if (b >= nbs && !bar_wait_sleep(empty + bs, (uint32_t)((b / nbs) - 1) & 1u)) { ok = false; break; }
+                const int i0 = b * kBatch, n = (L - i0) < kBatch ? (L - i0) : kBatch;
                 const int64_t u = rg.u0 + i0;
-                mbar_expect_tx(bar.full + s, (uint32_t)n * kPlaneBlk * R);
+                mbar_expect_tx(full + bs, (uint32_t)n * (kPlaneBlk * R + 256));
 #pragma unroll
                 for (int p = 0; p < R; ++p)
-                    bulk_g2s(smem + a.o_ring + ((size_t)s * R + p) * kB * kPlaneBlk,
-                             a.planes + p * a.plane_bytes + u * kPlaneBlk, (uint32_t)n * kPlaneBlk,
-                             bar.full + s);
-                mbar_expect_tx(bar.sfull + ss, (uint32_t)n * 256);
-                bulk_g2s(smem + a.o_sring + (size_t)ss * kB * 256, a.scales + u * 256, (uint32_t)n * 256,
-                         bar.sfull + ss);
-                flags[1] = b + 1;
-                // the next kernel of the stream may start (it waits for this
-                // one before it reads what this one writes)
-                if (b == 0) pdl_launch_dependents();
-                if (++s == nring) { s = 0; ++ks; }
-                if (++ss == nss) { ss = 0; ++kss; }
+                    bulk_g2s(smem + a.o_ring + ((size_t)p * S + (size_t)bs * kBatch) * kPlaneBlk,
+                             a.planes + p * a.plane_bytes + u * kPlaneBlk, (uint32_t)n * kPlaneBlk, full + bs);
+                bulk_g2s(smem + a.o_sring + (size_t)bs * kBatch * 256, a.scales + u * 256,
+                         (uint32_t)n * 256, full + bs);
+                st_release(&flags[1], b + 1);
             }
+            if (nbatch <= kHeadBatches) pdl_launch_dependents();
+            if (!ok) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
         }
-    } else {
-        // TMEM: eight A slots of 32 columns, then the D slots
+    } else if (warp < kCW) {
+        // ------------------------------------------------------------- teams
+        // TMEM is taken here, off the producer's path
         if (warp == 0) {
             tmem_alloc(tmem_slot, kTmemCols);
             tmem_relinquish();
         }
         tc_fence_before();
-        named_sync(1, kProdWarp * 32);
+        pdl_wait();                              // X comes from the previous kernel
+        build_x_operand<R>(a, smem, w, rg, nslot, flags);       // ends with a team barrier
         tc_fence_after();
         const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
-        const int qq = warp & 3, row = qq * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(32 * qq) << 16;
-
-        if (warp < kDecWarps) {
-            // ---------------------------------------------------------- decode
-            const int quad = warp >> 2;
-            const uint32_t idesc = idesc_u8s8(NB);
-            const uint32_t b0 = smem_u32(smem + a.o_b);
-            int s = 0, k = 0;                            // ring slot of item i's batch, its fill
-            int g = g0 + quad >= G ? g0 + quad - G : g0 + quad;   // group of item i
-            bool xready = false;
-            for (int i = quad; i < L; i += 2) {
-                // (kB == 2: item i is element `quad` of batch i / 2)
-                if (!mbar_wait_backoff(bar.full + s, (uint32_t)k & 1u, flags)) break;
-                uint4 pw[R];
-                const uint8_t *src = smem + a.o_ring + ((size_t)s * R * kB + quad) * kPlaneBlk + row * 16;
+        const int team = warp >> 2, q = warp & 3, row = q * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        const uint32_t col0 = tmem + (uint32_t)team * 128;       // A0 A1 at +0 +32, D0 D1 at +64 +64+NB
+        constexpr int gpb = MT <= 4 ? 4 / MT : 1;      // groups per B tile
+        const float2 *pairs = reinterpret_cast<const float2 *>(smem + a.o_pair);
+        constexpr float kOffset = (float)(128 >> (R - 1)) * 0.5f - 128.0f;   // 2^(7-r) - 128
+        float y[MT];
 #pragma unroll
-                for (int p = 0; p < R; ++p)
-                    pw[p] = *reinterpret_cast<const uint4 *>(src + (size_t)p * kB * kPlaneBlk);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar.empty + s);
-                uint32_t A[32];
+        for (int m = 0; m < MT; ++m) y[m] = 0.f;
+        int cur = -1;                                    // local tile of y
+        // Iteration jj decodes the team's pair jj (items i0 = kBatch jj + 2 team and
+        // i0 + 1) into registers, waits for the MMAs of pair jj - 1, stores
+        // the new A, reads the old D, and folds pair jj - 1.  Indices advance
+        // by kBatch items without divisions: ring stage, X slot, group and tile.
+        const int Jp = (L - 2 * team + kBatch - 1) / kBatch;   // pairs of this team
+        float sp[2] = {0.f, 0.f};                        // previous pair: scales, X slots, tiles
+        int slp[2] = {0, 0}, ltp[2] = {0, 0}, np = 0;
+        int st = 2 * team, fpar = 0;                     // ring stage of i0, parity of its fill
+        int xslot = 2 * team, g = rg.u0 % G + 2 * team, lt = 0;
+        while (xslot >= G) xslot -= G;
+        while (g >= G) { g -= G; ++lt; }
+        bool ok = true;
+        constexpr int ND = 4 * MT;                       // D columns read per item
+        const uint32_t idesc = idesc_u8s8(a.NB);
+        constexpr int gsh = MT == 1 ? 2 : MT == 2 ? 1 : 0;   // log2 groups per B tile
+        const uint32_t b0 = smem_u32(smem + a.o_b);
+        // MMA issuers: for M <= 2 the first thread of each warp q issues K steps
+        // 2(q&1), 2(q&1)+1 of item q>>1 into its own half of D; otherwise the
+        // first thread of warp e < 2 issues all four steps of item e
+        const bool issuer = lane == 0 && (MT <= 2 || q < 2);
+        int issued = 0;                                  // pairs whose MMAs were issued
+        for (int jj = 0; jj <= Jp; ++jj) {
+            const bool have = jj < Jp, back = jj > 0;
+            const int i0 = kBatch * jj + 2 * team;
+            const int n = have ? (i0 + 1 < L ? 2 : 1) : 0;   // items in this pair
+            uint32_t A0[32], A1[32];
+            float sc[2] = {0.f, 0.f};
+            bool good = ok;
+            if (have && good) {
+                const int bs = st / kBatch;              // ring slot of the batch
+                good = __all_sync(0xffffffffu, bar_wait(full + bs, (uint32_t)fpar));
+                if (good) {
+                    uint4 pw[R];
 #pragma unroll
-                for (int t4 = 0; t4 < 4; ++t4) {
-                    uint32_t P[8];
+                    for (int p = 0; p < R; ++p)
+                        pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st) * kPlaneBlk + row * 16);
+                    sc[0] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)st * 256 + row * 2));
 #pragma unroll
-                    for (int p = 0; p < 8; ++p) {
-                        const uint4 &v = pw[p < R ? p : 0];
-                        P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
+                    for (int t4 = 0; t4 < 4; ++t4) {
+                        uint32_t P[8];
+#pragma unroll
+                        for (int p = 0; p < 8; ++p) {
+                            const uint4 &v = pw[p < R ? p : 0];
+                            P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
+                        }
+                        field_operands<R>(P, A0 + 8 * t4);
                     }
-                    field_operands<R>(P, A + 8 * t4);
+                    if (n == 2) {
+#pragma unroll
+                        for (int p = 0; p < R; ++p)
+                            pw[p] = *reinterpret_cast<const uint4 *>(smem + a.o_ring + ((size_t)p * S + st + 1) * kPlaneBlk + row * 16);
+                        sc[1] = __half2float(*reinterpret_cast<const __half *>(smem + a.o_sring + (size_t)(st + 1) * 256 + row * 2));
+#pragma unroll
+                        for (int t4 = 0; t4 < 4; ++t4) {
+                            uint32_t P[8];
+#pragma unroll
+                            for (int p = 0; p < 8; ++p) {
+                                const uint4 &v = pw[p < R ? p : 0];
+                                P[p] = p < R ? (t4 == 0 ? v.x : t4 == 1 ? v.y : t4 == 2 ? v.z : v.w) : 0u;
+                            }
+                            field_operands<R>(P, A1 + 8 * t4);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(empty + bs);
                 }
-                // A slot i % kNA is free once the MMAs of item i - kNA are done:
-                // their commit completes that item's D-slot barrier
-                const int as = i & (kNA - 1);
-                if (i >= kNA) {
-                    const int j = i - kNA;
-                    if (!mbar_wait_backoff(bar.dfull + j % kND, (uint32_t)(j / kND) & 1u, flags)) break;
-                }
+            }
+            if (back && good) {
+                // the MMAs of pair jj - 1 are done: A is free and D holds their sums
+                good = __all_sync(0xffffffffu, bar_wait(dfull + team, (uint32_t)((jj - 1) & 1)));
                 tc_fence_after();
-                tmem_st32(tmem + lane_base + (uint32_t)as * 32, A);
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                uint32_t old = 0;
-                if (lane == 0) old = atom_add_acq_rel(acnt + as, 1u);
-                old = __shfl_sync(0xffffffffu, old, 0);
-                if (old == 4u * (uint32_t)(i / kNA) + 3u && lane == 0) {
-                    // the last warp of the quad for this item: issue its MMAs
-                    bool ok = true;
-                    if (!xready) {
-                        ok = mbar_wait_backoff(bar.xbar, 0u, flags);
-                        xready = ok;
+            }
+            int d0[ND], d1[ND];
+            if (good) {
+                if (have) {
+                    tmem_st32(lane_base + col0, A0);
+                    if (n == 2) tmem_st32(lane_base + col0 + 32, A1);
+                }
+                if (back) {
+                    if constexpr (MT <= 2) {
+                        // each item's D is two halves (K steps 0-1 and 2-3): add them
+                        int h0[ND], h1[ND];
+                        const uint32_t o0 = 4 * M * (slp[0] & (gpb - 1)), o1 = 4 * M * (slp[1] & (gpb - 1));
+                        read_d<MT>(lane_base + col0 + 64 + o0, d0);
+                        read_d<MT>(lane_base + col0 + 64 + 16 + o0, h0);
+                        if (np == 2) {
+                            read_d<MT>(lane_base + col0 + 96 + o1, d1);
+                            read_d<MT>(lane_base + col0 + 112 + o1, h1);
+                        }
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < ND; ++i) {
+                            d0[i] += h0[i];
+                            d1[i] += h1[i];
+                        }
+                    } else if constexpr (MT <= 4) {
+                        read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
+                        if (np == 2) read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
+                        tmem_ld_wait();
+                    } else {
+                        read_d<MT>(lane_base + col0 + 64 + 4 * M * (slp[0] & (gpb - 1)), d0);
+                        tmem_ld_wait();
+                        FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
+                        if (np == 2) {
+                            read_d<MT>(lane_base + col0 + 64 + a.NB + 4 * M * (slp[1] & (gpb - 1)), d1);
+                            tmem_ld_wait();
+                        }
                     }
-                    const int ds = i % kND;
-                    if (ok && i >= kND) ok = mbar_wait_backoff(bar.dempty + ds, (uint32_t)((i / kND) - 1) & 1u, flags);
-                    if (ok) {
-                        tc_fence_after();
-                        const uint32_t baddr = b0 + (uint32_t)(xs.tile_of(g, gpb) * NB * 128);
-                        const uint32_t dcol = tmem + kDCol0 + (uint32_t)(ds * NB);
+                }
+                if (have) tmem_st_wait();
+            }
+            tc_fence_before();
+            // the whole team has stored A and read D (or a wait timed out)
+            if (!named_sync_and(2 + team, 128, good)) { ok = false; break; }
+            if (have && issuer) {
+                // D[team][e] = A[team][e] . B(X slot of item e)^T, K = 128 in 4 steps;
+                // every issuer commits (an empty commit arrives at once)
+                tc_fence_after();
+                if constexpr (MT <= 2) {
+                    const int e = q >> 1, h = q & 1;
+                    if (e < n) {
+                        const int sl = xslot + e >= G ? xslot + e - G : xslot + e;
+                        const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
+#pragma unroll
+                        for (int k2 = 0; k2 < 2; ++k2) {
+                            const int kk = 2 * h + k2;
+                            mma_i8_ts(col0 + 64 + (uint32_t)(32 * e + 16 * h), col0 + 32 * e + 8 * kk,
+                                      smem_desc_sw128(baddr + 32 * kk), idesc, k2 > 0 ? 1u : 0u);
+                        }
+                    }
+                } else {
+                    const int e = q;
+                    if (e < n) {
+                        const int sl = xslot + e >= G ? xslot + e - G : xslot + e;
+                        const uint32_t baddr = b0 + (uint32_t)((sl >> gsh) * a.NB * 128);
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            mma_i8_ts(dcol, tmem + (uint32_t)(as * 32 + 8 * kk), smem_desc_sw128(baddr + 32 * kk),
-                                      idesc, kk > 0 ? 1u : 0u);
-                        mma_commit(bar.dfull + ds);
-                        atomicAdd(icnt + ds, 1u);
+                            mma_i8_ts(col0 + 64 + (uint32_t)(e * a.NB), col0 + 32 * e + 8 * kk,
+                                      smem_desc_sw128(baddr + 32 * kk), idesc, kk > 0 ? 1u : 0u);
                     }
                 }
-                if (flags[0]) break;
-                if (++s == nring) { s = 0; ++k; }
-                g += 2;                                   // (G may be 1)
-                if (g >= G) g -= G;
-                if (g >= G) g -= G;
+                mma_commit(dfull + team);
             }
-        } else {
-            // ------------------------------------------------------------ fold
-            const int fw = warp - kFoldW0;
-            if (fw == 0 && lane == 0) {
-                // the CTA's X tiles and pairs, once the X of this call is ready
-                pdl_wait();
-                const size_t tb = (size_t)NB * 128;
-                const int na_groups = (xs.g0 + nslot - 1 < G ? nslot : G - xs.g0);
-                const uint32_t bytes = (uint32_t)((xs.na + xs.nb) * tb + (size_t)nslot * 64);
-                mbar_expect_tx(bar.xbar, bytes);
-                bulk_g2s(smem + a.o_b, a.xtiles + xs.ta0 * tb, (uint32_t)(xs.na * tb), bar.xbar);
-                if (xs.nb) bulk_g2s(smem + a.o_b + xs.na * tb, a.xtiles, (uint32_t)(xs.nb * tb), bar.xbar);
-                bulk_g2s(smem + a.o_pair, a.xpairs + (size_t)xs.g0 * 8, (uint32_t)(na_groups * 64), bar.xbar);
-                if (na_groups < nslot)
-                    bulk_g2s(smem + a.o_pair + na_groups * 64, a.xpairs, (uint32_t)((nslot - na_groups) * 64),
-                             bar.xbar);
+            if (have) ++issued;
+            if (back) {
+                if constexpr (MT <= 4) FOLD_ITEM(d0, sp[0], slp[0], ltp[0]);
+                if (np == 2) FOLD_ITEM(d1, sp[1], slp[1], ltp[1]);
             }
-            const float2 *pairs = reinterpret_cast<const float2 *>(smem + a.o_pair);
-            constexpr float kOffset = (float)(128 >> (R - 1)) * 0.5f - 128.0f;   // 2^(7-r) - 128
-            float y[MT];
+            // this pair becomes the previous one; advance by kBatch items
+            np = n;
+            sp[0] = sc[0]; sp[1] = sc[1];
+            slp[0] = xslot; ltp[0] = lt;
+            slp[1] = xslot + 1 == G ? 0 : xslot + 1;
+            ltp[1] = g + 1 == G ? lt + 1 : lt;
+            st += kBatch;
+            if (st >= S) { st -= S; fpar ^= 1; }
+            xslot += kBatch;
+            while (xslot >= G) xslot -= G;
+            g += kBatch;
+            while (g >= G) { g -= G; ++lt; }
+        }
+        if (cur >= 0) {
 #pragma unroll
-            for (int m = 0; m < MT; ++m) y[m] = 0.f;
-            int t = tf, g = g0, cur = tf, slot = 0;
-            bool ok = mbar_wait_backoff(bar.xbar, 0u, flags);
-            const uint32_t red_base = smem_u32(red);
-            // a finished tile: into Y, or (a tile that started in an earlier
-            // CTA) into the owner's shared memory
-            auto flush = [&](int tile) {
-                const int64_t ra = (int64_t)tile * G, rb = ra + G;
-                if (ra >= rg.u0 && rb <= rg.u1) {
-                    const int64_t n = (int64_t)tile * 128 + row;
-                    if (n < a.N) {
+            for (int m = 0; m < MT; ++m)
+                if (m < M) res[((team * ntile + cur) * M + m) * 128 + row] = y[m];
+        }
+        if (!ok && issued > 0) {
+            // the team's last MMAs may still run: let them finish before TMEM is freed
+            bar_wait(dfull + team, (uint32_t)((issued - 1) & 1));
+        }
+        if (!ok && lane == 0) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
+        named_sync(1, kCW * 32);
+        // ---- combine the teams per tile (fixed order).  A tile inside this
+        // CTA goes to Y; a tile this CTA owns but shares keeps its part in
+        // slot 0 of `red`; the first tile, if it started in an earlier CTA of
+        // the cluster, is sent to slot j of its owner (j = distance in CTAs).
+        const int64_t ra0 = tf * G;
+        const bool sends = ra0 < rg.u0;                  // the first tile started earlier
+        const int64_t owner = sends ? w.cta_of(ra0) : -1;
+        const int owner_rank = (int)owner % w.CS;
+        const int owner_lt = sends ? (int)tf - (int)w.first(owner) / G : 0;
+        const int jsend = (int)(blockIdx.x - owner);
+        if (sends) cluster_wait();                       // the owner's barrier is initialised
+        const uint32_t red_base = smem_u32(red);
+        for (int idx = threadIdx.x; idx < ntile * M * 128; idx += kCW * 32) {
+            const int lt = idx / (M * 128), rem = idx - lt * M * 128, m = rem >> 7, rr = rem & 127;
+            float v = 0.f;
 #pragma unroll
-                        for (int m = 0; m < MT; ++m)
-                            if (m < M) a.Y[(int64_t)m * a.N + n] = __float2bfloat16_rn(y[m]);
-                    }
-                } else if (ra < rg.u0) {
-                    const int64_t owner = w.cta_of(ra);
-                    const uint32_t orank = (uint32_t)(owner % w.CS);
-                    const int j = (int)(blockIdx.x - owner);
-                    if (!cluster_waited) { cluster_wait(); cluster_waited = true; }
-#pragma unroll
-                    for (int m = 0; m < MT; ++m)
-                        if (m < M)
-                            st_cluster_f32(cluster_map(red_base + (uint32_t)(((j * M + m) * 128 + row) * 4), orank),
-                                           y[m]);
-                    mbar_arrive_remote(cluster_map(smem_u32(bar.rbar), orank));
-                }
-                // else: the owned shared tile (the last one), kept in y
-            };
-            for (int i0 = 0; ok && i0 < L; i0 += CH) {
-                const int n = L - i0 < CH ? L - i0 : CH;
-                // wait for the items' D slots (and each new scale batch)
-#pragma unroll
-                for (int j = 0; j < CH; ++j) {
-                    const int i = i0 + j;
-                    if (j < n && ok) {
-                        if ((i & (kB - 1)) == 0)
-                            ok = mbar_wait_backoff(bar.sfull + (i / kB) % nss, (uint32_t)((i / kB) / nss) & 1u, flags);
-                        if (ok) ok = mbar_wait_backoff(bar.dfull + i % kND, (uint32_t)(i / kND) & 1u, flags);
-                    }
-                }
-                if (!ok) break;
-                tc_fence_after();
-                uint32_t d[CH][4 * MT];
-#pragma unroll
-                for (int j = 0; j < CH; ++j) {
-                    if (j < n) {
-                        const int i = i0 + j, gj = (g0 + slot + j) % G;
-                        read_d<MT>(tmem + lane_base + kDCol0 + (uint32_t)((i % kND) * NB + 4 * M * (gj % gpb)), d[j]);
-                    }
-                }
-                tmem_ld_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) {
-#pragma unroll
-                    for (int j = 0; j < CH; ++j)
-                        if (j < n) mbar_arrive(bar.dempty + (i0 + j) % kND);
-                }
-#pragma unroll
-                for (int j = 0; j < CH; ++j) {
-                    if (j < n) {
-                        const int i = i0 + j, e = i & (kB - 1), ss = (i / kB) % nss;
-                        const float sc = __half2float(*reinterpret_cast<const __half *>(
-                            smem + a.o_sring + ((size_t)ss * kB + e) * 256 + row * 2));
-                        if (e == kB - 1 || i == L - 1) {
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(bar.sempty + ss);
-                        }
-                        if (t != cur) {
-                            flush(cur);
-#pragma unroll
-                            for (int m = 0; m < MT; ++m) y[m] = 0.f;
-                            cur = t;
-                        }
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            if (m < M) {
-                                const float v = (float)(int)d[j][4 * m] + 0x1p-7f * (float)(int)d[j][4 * m + 1] +
-                                                0x1p-14f * (float)(int)d[j][4 * m + 2] +
-                                                0x1p-21f * (float)(int)d[j][4 * m + 3];
-                                const float2 ge = pairs[slot * 8 + m];
-                                y[m] = fmaf(sc * ge.x, v, fmaf(sc * kOffset, ge.y, y[m]));
-                            }
-                        }
-                        if (++slot == G) slot = 0;
-                        if (++g == G) { g = 0; ++t; }
-                    }
-                }
+            for (int tm = 0; tm < kTeams; ++tm) v += res[((tm * ntile + lt) * M + m) * 128 + rr];
+            const int64_t t = tf + lt, ra = t * G, rb = ra + G;
+            if (ra >= rg.u0 && rb <= rg.u1) {
+                const int64_t n = t * 128 + rr;
+                if (n < a.N) a.Y[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
+            } else if (ra >= rg.u0) {
+                red[((size_t)lt * w.CS) * M * 128 + rem] = v;
+            } else {
+                const uint32_t off = (uint32_t)((((size_t)owner_lt * w.CS + jsend) * M * 128 + rem) * 4);
+                st_cluster_f32(cluster_map(red_base + off, (uint32_t)owner_rank), v);
             }
-            if (ok && !flags[0]) {
-                flush(cur);
-                if (own_nc > 1) {
-                    // the owned last tile: wait for the other parts, sum in CTA order
-                    const uint64_t t0 = global_ns();
-                    bool got = true;
-                    while (!mbar_try_wait_cluster(bar.rbar, 0u)) {
-                        if (flags[0] || global_ns() - t0 > kWaitNs) { got = false; flags[0] = 1; break; }
-                    }
-                    if (got) {
-                        const int64_t n = (int64_t)tl * 128 + row;
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) {
-                            if (m < M) {
-                                float v = y[m];
-                                for (int j = 1; j < own_nc; ++j) v += red[(j * M + m) * 128 + row];
-                                if (n < a.N) a.Y[(int64_t)m * a.N + n] = __float2bfloat16_rn(v);
-                            }
-                        }
-                    }
-                }
+        }
+        named_sync(1, kCW * 32);
+        if (sends && threadIdx.x == 0)
+            mbar_arrive_remote(cluster_map(smem_u32(rbar + owner_lt), (uint32_t)owner_rank));
+        if (own_nc > 1) {
+            // the owned last tile: wait for the other parts, sum in CTA order
+            const int lt = (int)(own_last - tf);
+            bool got = true;
+            if (threadIdx.x == 0) {
+                const uint64_t t0 = global_ns();
+                while (!bar_try_cluster(rbar + lt, 0u))
+                    if (global_ns() - t0 > kWaitNs) { got = false; break; }
+                if (!got) { st_release(&flags[0], 1); atomicOr(&g_gemv_timeout, 1u); }
+            }
+            named_sync(1, kCW * 32);
+            for (int idx = threadIdx.x; idx < M * 128; idx += kCW * 32) {
+                float v = 0.f;
+                for (int j = 0; j < own_nc; ++j) v += red[((size_t)lt * w.CS + j) * M * 128 + idx];
+                const int64_t n = own_last * 128 + (idx & 127);
+                if (n < a.N) a.Y[(int64_t)(idx >> 7) * a.N + n] = __float2bfloat16_rn(v);
             }
         }
     }
 
-    // ---- end: after an abort, let the copies and MMAs already issued land;
-    // then meet the cluster (no CTA leaves while another may still write into
-    // its shared memory) and free TMEM
-    __syncwarp();
+    // after a timed-out wait, let the copies already issued land; then free TMEM
+    tc_fence_before();
     __syncthreads();
     if (flags[0] && threadIdx.x == 0) {
         const int issued = flags[1];
-        for (int b = (issued > nring ? issued - nring : 0); b < issued; ++b)
-            mbar_wait_bounded(bar.full + b % nring, (uint32_t)(b / nring) & 1u);
-        for (int b = (issued > nss ? issued - nss : 0); b < issued; ++b)
-            mbar_wait_bounded(bar.sfull + b % nss, (uint32_t)(b / nss) & 1u);
-        for (int ds = 0; ds < kND; ++ds) {
-            const uint32_t c = icnt[ds];
-            if (c) mbar_wait_bounded(bar.dfull + ds, (c - 1) & 1u);
+        for (int bs = 0; bs < nbs && bs < issued; ++bs) {
+            const int last = bs + ((issued - 1 - bs) / nbs) * nbs;
+            bar_wait(full + bs, (uint32_t)(last / nbs) & 1u);
         }
-        atomicOr(&g_gemv_timeout, 1u);
     }
-    // (the X copy is waited for by the fold warps; on an abort before that
-    // wait, let it land here)
-    if (flags[0] && threadIdx.x == 32 * kFoldW0) mbar_wait_bounded(bar.xbar, 0u);
-    tc_fence_before();
-    __syncthreads();
+    // no CTA of a cluster leaves while another may still write into its
+    // shared memory (a sender that was late when its owner gave up waiting):
+    // every wait above is bounded, so every thread of the cluster gets here
     if (w.CS > 1) {
-        if (!cluster_waited) cluster_wait();
+        const bool waited = warp < kCW && (int64_t)(rg.u0 / G) * G < rg.u0;   // senders waited above
+        if (!waited) cluster_wait();
         cluster_arrive();
         cluster_wait();
     }
@@ -671,8 +716,8 @@ nested_gemv_tc_kernel(const __grid_constant__ Args a) {
 // ---------------------------------------------------------------- host side
 struct Plan {
     Work w;
-    int nring, nss, nslot, nxt, L;
-    uint32_t o_ring, o_sring, o_b, o_pair, o_bar, o_red, o_misc;
+    int NB, S, nslot, L, ntile;
+    uint32_t o_ring, o_sring, o_b, o_pair, o_res, o_bar, o_red, o_misc;
     size_t smem;
     bool ok;
 };
@@ -692,63 +737,57 @@ int sm_count() {
 
 inline uint32_t align_up(size_t x, size_t a) { return (uint32_t)((x + a - 1) / a * a); }
 
-// Shared-memory layout for `nring` plane batches and `nss` scale batches;
-// returns its size without the alignment slack.
-size_t layout(Plan &p, int r, int M, int nring, int nss) {
-    const int MT = batch_class(M), NB = class_nb(MT), nd = 256 / NB;
+// Shared-memory layout for S stages; returns its size without slack.
+size_t layout(Plan &p, int r, int M, int S) {
+    const int gpb = p.NB == 16 ? (M == 1 ? 4 : M == 2 ? 2 : 1) : 1;
     size_t o = 0;
     p.o_ring = 0;
-    o = (size_t)nring * kB * r * kPlaneBlk;
+    o = (size_t)r * S * 2048;
     p.o_sring = align_up(o, 128);
-    o = p.o_sring + (size_t)nss * kB * 256;
+    o = p.o_sring + (size_t)S * 256;
     p.o_b = align_up(o, 1024);
-    o = p.o_b + (size_t)p.nxt * NB * 128;
+    o = p.o_b + (size_t)((p.nslot + gpb - 1) / gpb) * p.NB * 128;
     p.o_pair = align_up(o, 16);
     o = p.o_pair + (size_t)p.nslot * 8 * 8;
+    p.o_res = align_up(o, 16);
+    o = p.o_res + (size_t)kTeams * p.ntile * M * 128 * 4;
     p.o_bar = align_up(o, 16);
-    o = p.o_bar + (size_t)bar_count(nring, nss, nd) * 8;
+    o = p.o_bar + (size_t)(2 * (S / kBatch) + kTeams + p.ntile) * 8;
     p.o_red = align_up(o, 16);
-    o = p.o_red + (p.w.CS > 1 ? (size_t)p.w.CS * M * 128 * 4 : 0);
+    o = p.o_red + (p.w.CS > 1 ? (size_t)p.ntile * p.w.CS * M * 128 * 4 : 0);
     p.o_misc = align_up(o, 16);
-    o = p.o_misc + 16 + (size_t)(kNA + nd) * 4;            // flags, TMEM address, counters
+    o = p.o_misc + 64;                                     // flags, TMEM address
     return o;
 }
 
-// Ranges, rings and shared memory for one (clusters, CTAs per cluster) split.
+// Ranges, ring and shared memory for one (clusters, CTAs per cluster) split.
 Plan plan_for(const Work &w, int64_t M, int r) {
     Plan p{};
     p.w = w;
+    p.NB = M <= 4 ? 16 : 32;
     const int64_t G = w.KC;
-    const int gpb = class_gpb(batch_class(M));
-    int64_t L = 0;
-    int nxt = 0;
+    int64_t L = 0, nt = 0;
     for (int64_t b = 0; b < w.ctas(); ++b) {
         const int64_t u0 = w.first(b), u1 = w.first(b + 1);
         if (u1 <= u0) return p;                            // an empty CTA: not a valid split
         L = u1 - u0 > L ? u1 - u0 : L;
-        const int ns = (int)(u1 - u0 < G ? u1 - u0 : G);
-        const XSpan xs((int)(u0 % G), ns, (int)G, gpb);
-        nxt = xs.na + xs.nb > nxt ? xs.na + xs.nb : nxt;
+        const int64_t tt = (u1 - 1) / G - u0 / G + 1;
+        nt = tt > nt ? tt : nt;
     }
     p.L = (int)L;
+    p.ntile = (int)nt;
     p.nslot = (int)(L < G ? L : G);
-    p.nxt = nxt;
-    const int nbatch = (int)((L + kB - 1) / kB);
-    const size_t batch = (size_t)kB * r * kPlaneBlk;
-    // the plane ring: up to kRingBytes, at least one batch (or the whole
-    // range), within the shared memory left by the X operand
-    int nring = (int)(kRingBytes / batch);
-    if (nring < 2) nring = 2;
-    if (nring > nbatch) nring = nbatch;
-    auto total = [&](int nr) {
-        const int ns = nbatch < nr + 8 ? nbatch : nr + 8;
-        return layout(p, r, (int)M, nr, ns) + 1024;
-    };
-    while (nring > 1 && total(nring) > kSmemMax) --nring;
-    if (total(nring) > kSmemMax) return p;
-    p.nring = nring;
-    p.nss = nbatch < nring + 8 ? nbatch : nring + 8;
-    p.smem = layout(p, r, (int)M, p.nring, p.nss) + 1024;
+    const size_t stage = (size_t)2048 * r + 256;
+    const size_t fixed = layout(p, r, (int)M, 0);
+    const int need = (int)((L + kBatch - 1) / kBatch) * kBatch;   // stages for the whole range
+    const int want = need < kBatch ? need : kBatch;                // fewest stages accepted (one batch)
+    if (fixed + (size_t)want * stage + 1024 > kSmemMax) return p;
+    int S = (int)((kSmemMax - 1024 - fixed) / stage) / kBatch * kBatch;
+    if (S > need) S = need;
+    // the ring's barriers and alignment come on top of `fixed`
+    while (S > want && layout(p, r, (int)M, S) + 1024 > kSmemMax) S -= kBatch;
+    p.S = S;
+    p.smem = layout(p, r, (int)M, S) + 1024;
     p.ok = p.smem <= kSmemMax;
     return p;
 }
@@ -757,8 +796,7 @@ int max_clusters(int r, int64_t M, size_t smem, int cs);   // below, per instant
 
 // Choose the split: whole tiles per CTA (CS = 1) or clusters of CS CTAs that
 // share tiles, taking the one with the fewest items on the busiest CTA (a
-// shared tile costs about one extra item of latency for its exchange).  At
-// most one CTA per SM.
+// shared tile costs about one extra item of latency for its exchange).
 Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     const int64_t T = (N + 127) / 128, G = K / kGroup;
     const int sms = sm_count();
@@ -785,14 +823,6 @@ Plan make_plan(int64_t M, int64_t N, int64_t K, int r) {
     return best;
 }
 
-// Workspace of the prepared X: B tiles of all groups, then the pairs.
-size_t xprep_tile_bytes(int64_t M, int64_t K) {
-    const int MT = batch_class(M), gpb = class_gpb(MT);
-    const int64_t G = K / kGroup;
-    return (size_t)((G + gpb - 1) / gpb) * class_nb(MT) * 128;
-}
-size_t xprep_bytes(int64_t M, int64_t K) { return xprep_tile_bytes(M, K) + (size_t)(K / kGroup) * 64; }
-
 // cudaFuncSetAttribute once per (instantiation, device), safe from any host thread.
 template <typename F>
 cudaError_t ensure_smem_attr(F *fn, std::atomic<uint64_t> &done) {
@@ -814,50 +844,34 @@ std::atomic<uint64_t> &attr_done() {
 
 template <int R, int MT>
 mq_status run(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, const Plan &p,
-              void *ws, cudaStream_t st) {
+              cudaStream_t st) {
     cudaError_t e = ensure_smem_attr(nested_gemv_tc_kernel<R, MT>, attr_done<R, MT>());
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    uint8_t *xt = static_cast<uint8_t *>(ws) + kXOff;
-    float2 *xp = reinterpret_cast<float2 *>(xt + xprep_tile_bytes(M, wt->K));
-    const int G = (int)(wt->K / kGroup);
-    // programmatic dependent launch for both kernels: each may start while
-    // the kernel before it finishes, and waits for it before reading its output
-    cudaLaunchAttribute pdl;
-    pdl.id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl.val.programmaticStreamSerializationAllowed = 1;
-    {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3((unsigned)((G * M + kPrepWarps - 1) / kPrepWarps));
-        cfg.blockDim = dim3(kPrepWarps * 32);
-        cfg.stream = st;
-        cfg.attrs = &pdl;
-        cfg.numAttrs = 1;
-        e = cudaLaunchKernelEx(&cfg, x_prep_kernel<R, MT>, X, (int)M, (int64_t)wt->K, G, xt, xp);
-        if (e != cudaSuccess) return cuda_fail(e, "x_prep_kernel launch");
-    }
     Args a{};
+    a.X = reinterpret_cast<const __nv_bfloat16 *>(X);
     a.planes = reinterpret_cast<const uint8_t *>(wt->planes);
     a.scales = reinterpret_cast<const uint8_t *>(wt->scales);
-    a.xtiles = xt;
-    a.xpairs = xp;
     a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
     a.w = p.w;
     a.N = wt->N;
     a.K = wt->K;
-    a.G = G;
+    a.G = wt->K / kGroup;
     a.plane_bytes = (int64_t)mq_plane_bytes(wt->N, wt->K, 1);
     a.M = (int)M;
-    a.nring = p.nring;
-    a.nss = p.nss;
+    a.NB = p.NB;
+    a.S = p.S;
     a.o_ring = p.o_ring; a.o_sring = p.o_sring; a.o_b = p.o_b; a.o_pair = p.o_pair;
-    a.o_bar = p.o_bar; a.o_red = p.o_red; a.o_misc = p.o_misc;
+    a.o_res = p.o_res; a.o_bar = p.o_bar; a.o_red = p.o_red; a.o_misc = p.o_misc;
+    // programmatic dependent launch: this grid may start while the previous
+    // kernel of the stream finishes; it waits for it before reading X
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.w.ctas());
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = p.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
-    attr[0] = pdl;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = (unsigned)p.w.CS;
     attr[1].val.clusterDim.y = 1;
@@ -893,23 +907,19 @@ int occ_clusters(size_t smem, int cs) {
 }
 template <int R>
 int occ_clusters_r(int64_t M, size_t smem, int cs) {
-    switch (batch_class(M)) {
-        case 1: return occ_clusters<R, 1>(smem, cs);
-        case 2: return occ_clusters<R, 2>(smem, cs);
-        case 4: return occ_clusters<R, 4>(smem, cs);
-        default: return occ_clusters<R, 8>(smem, cs);
-    }
+    if (M == 1) return occ_clusters<R, 1>(smem, cs);
+    if (M == 2) return occ_clusters<R, 2>(smem, cs);
+    if (M <= 4) return occ_clusters<R, 4>(smem, cs);
+    return occ_clusters<R, 8>(smem, cs);
 }
 
 template <int R>
 mq_status run_r(const uint16_t *X, const mq_weights *wt, int64_t M, uint16_t *Y, const Plan &p,
-                void *ws, cudaStream_t st) {
-    switch (batch_class(M)) {
-        case 1: return run<R, 1>(X, wt, M, Y, p, ws, st);
-        case 2: return run<R, 2>(X, wt, M, Y, p, ws, st);
-        case 4: return run<R, 4>(X, wt, M, Y, p, ws, st);
-        default: return run<R, 8>(X, wt, M, Y, p, ws, st);
-    }
+                cudaStream_t st) {
+    if (M == 1) return run<R, 1>(X, wt, M, Y, p, st);
+    if (M == 2) return run<R, 2>(X, wt, M, Y, p, st);
+    if (M <= 4) return run<R, 4>(X, wt, M, Y, p, st);
+    return run<R, 8>(X, wt, M, Y, p, st);
 }
 
 int max_clusters(int r, int64_t M, size_t smem, int cs) {
@@ -961,25 +971,24 @@ bool gemv_tc_supported(int64_t M, int64_t N, int64_t K, int r) {
     return M >= 1 && M <= kGemvMaxM && cached_plan(M, N, K, r).ok;
 }
 
-// The GEMV keeps the X operand of the call (built once per call) in the
-// workspace, after the GEMM's ticket region (which it leaves untouched).
-size_t gemv_tc_workspace_bytes(int64_t M, int64_t, int64_t K, int) { return kXOff + xprep_bytes(M, K); }
+// The GEMV sums shared tiles inside clusters: it needs no workspace.
+size_t gemv_tc_workspace_bytes(int64_t, int64_t, int64_t, int) { return 0; }
 
 mq_status launch_gemv_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
                          void *ws, size_t ws_bytes, cudaStream_t st) {
+    (void)ws_bytes;
     const Plan p = cached_plan(M, w->N, w->K, w->r);
     if (!p.ok) return fail(MQ_ERR_UNSUPPORTED, "no tensor-core GEMV plan fits this shape");
-    if (!ws || ws_bytes < gemv_tc_workspace_bytes(M, w->N, w->K, w->r))
-        return fail(MQ_ERR_WORKSPACE, "GEMV workspace missing or too small");
+    (void)ws;
     switch (w->r) {
-        case 1: return run_r<1>(X, w, M, Y, p, ws, st);
-        case 2: return run_r<2>(X, w, M, Y, p, ws, st);
-        case 3: return run_r<3>(X, w, M, Y, p, ws, st);
-        case 4: return run_r<4>(X, w, M, Y, p, ws, st);
-        case 5: return run_r<5>(X, w, M, Y, p, ws, st);
-        case 6: return run_r<6>(X, w, M, Y, p, ws, st);
-        case 7: return run_r<7>(X, w, M, Y, p, ws, st);
-        default: return run_r<8>(X, w, M, Y, p, ws, st);
+        case 1: return run_r<1>(X, w, M, Y, p, st);
+        case 2: return run_r<2>(X, w, M, Y, p, st);
+        case 3: return run_r<3>(X, w, M, Y, p, st);
+        case 4: return run_r<4>(X, w, M, Y, p, st);
+        case 5: return run_r<5>(X, w, M, Y, p, st);
+        case 6: return run_r<6>(X, w, M, Y, p, st);
+        case 7: return run_r<7>(X, w, M, Y, p, st);
+        default: return run_r<8>(X, w, M, Y, p, st);
     }
 }
 
