@@ -62,6 +62,23 @@ def gen_layers():
         return list(ex.map(one, enumerate(wl.LLAMA8B)))
 
 
+# DRAM traffic of one step (dram__bytes_read.sum + dram__bytes_write.sum
+# summed over the 21 launches) from the ncu capture summarised in
+# profiles/gemv_llama8b_m1_step_traffic.md, valid for the kernel source it was
+# taken with (sha256 of csrc/mq_gemv_tc.cu); None once that source changes.
+STEP_TRAFFIC = None
+
+
+def step_traffic():
+    if not STEP_TRAFFIC:
+        return None
+    import hashlib
+    src = os.path.join(ROOT, "nested_bit_weight_b200", "csrc", "mq_gemv_tc.cu")
+    with open(src, "rb") as f:
+        digest = hashlib.sha256(f.read()).hexdigest()
+    return STEP_TRAFFIC["bytes"] if digest == STEP_TRAFFIC["sha256"] else None
+
+
 def read_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -149,6 +166,147 @@ def aggregate_gbps(ws: int, bytes_per_step: float, ms_per_step: float) -> float:
     return round(ws * bytes_per_step / (ms_per_step * 1e-3) / 1e9, 2)
 
 
+def time_point(mq, X, views, Y, ws, n_samples: int = 100):
+    """Device time of one mq_gemm shape over rotated weight copies.
+
+    Returns (median, p10, p90) in µs over >= n_samples launches, each timed
+    alone by an event pair inside a CUDA graph (the events stop consecutive
+    launches from overlapping), and the mean µs per launch of the same
+    launches back to back in a graph without events (overlap allowed)."""
+    import torch
+    n_launch = max(len(views), 25)
+    stream = torch.cuda.Stream()
+    ev = [(torch.cuda.Event(enable_timing=True, external=True),
+           torch.cuda.Event(enable_timing=True, external=True)) for _ in range(n_launch)]
+    with torch.cuda.stream(stream):
+        for v in views:
+            mq.mq_gemm(X, v, Y, ws)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(n_launch):
+                mq.mq_gemm(X, views[j % len(views)], Y, ws)
+        gi = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gi, stream=stream):
+            for j in range(n_launch):
+                ev[j][0].record()
+                mq.mq_gemm(X, views[j % len(views)], Y, ws)
+                ev[j][1].record()
+        for _ in range(3):
+            g.replay()
+            gi.replay()
+        torch.cuda.synchronize()
+        samples = []
+        while len(samples) < n_samples:
+            gi.replay()
+            torch.cuda.synchronize()
+            samples += [a.elapsed_time(b) * 1e3 for a, b in ev]
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        reps = max(1, -(-n_samples // n_launch))
+        e0.record()
+        for _ in range(reps):
+            g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    b2b = e0.elapsed_time(e1) * 1e3 / (reps * n_launch)
+    del g, gi
+    q = np.percentile(np.array(samples), [50, 10, 90])
+    return float(q[0]), float(q[1]), float(q[2]), float(b2b), len(samples)
+
+
+def rotated_parents(mq, codes, s, l2: int):
+    """A packed parent and enough device copies that cycling through them
+    reads more than twice the L2 (every launch streams its planes from HBM)."""
+    import torch
+    p0 = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+    pbytes = p0.planes.numel() * 4 + p0.scales16.numel() * 2
+    copies = max(1, -(-2 * l2 // pbytes))
+    return [p0] + [mq.NestedWeights(p0.planes.clone(), p0.scales16.clone(), p0.N, p0.K)
+                   for _ in range(copies - 1)]
+
+
+PER_POINTS = [("gate_proj", 14336, 4096), ("q_proj", 4096, 4096)]
+PER_POINT_M = (8, 16, 64)
+PER_POINT_R = (4, 2)
+
+
+def run_per_points():
+    """Config 2 points (Llama-3.1-8B gate and q at M in {8, 16, 64}, r in
+    {4, 2}): each timed in isolation over rotated weights (L2-cold)."""
+    import torch
+    import nested_bit_weight_b200 as mq
+    peak, _ = read_peaks()
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    out = {}
+    for name, N, K in PER_POINTS:
+        li = [l.name for l in wl.LLAMA8B].index(name)
+        codes, s, _ = wl.gen_weights(N, K, wl.layer_seed(2, li))
+        parents = rotated_parents(mq, codes, s, l2)
+        del codes
+        for M in PER_POINT_M:
+            xbits, _ = wl.gen_x(M, K, wl.layer_seed(2, li))
+            X = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+            for r in PER_POINT_R:
+                ws = torch.zeros(max(mq.mq_gemm_workspace_bytes(M, N, K, r), 256),
+                                 dtype=torch.uint8, device="cuda")
+                med, p10, p90, b2b, n = time_point(mq, X, [q.view(r) for q in parents], Y, ws)
+                b = algo_bytes(N, K, r, M)
+                out[f"{name}/M{M}/r{r}"] = {
+                    "N": N, "K": K, "M": M, "r": r, "path": "gemv" if mq.uses_gemv(M, N, K, r) else "gemm",
+                    "us_median": round(med, 3), "us_p10": round(p10, 3), "us_p90": round(p90, 3),
+                    "launches": n, "us_back_to_back": round(b2b, 3),
+                    "GBps_median": round(b / (med * 1e-6) / 1e9, 1),
+                    "frac_hbm_median": round(b / (med * 1e-6) / 1e9 / peak, 4)}
+        del parents
+        torch.cuda.empty_cache()
+    return out
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+_ONE_CORE = r"""
+import sys, time, json
+sys.path.insert(0, ROOTDIR)
+import numpy as np
+import oracle, workloads as wl
+out = {}
+for name, N, K, ci in (("config0 512x512 M=1 r=4", 512, 512, 0), ("llama q_proj 4096x4096 M=1 r=4", 4096, 4096, 1)):
+    codes, s, _ = wl.gen_weights(N, K, wl.layer_seed(ci, 0))
+    xbits, X = wl.gen_x(1, K, wl.layer_seed(ci, 0))
+    oracle.gemm(X, codes, s, 4)
+    n, t0 = 0, time.perf_counter()
+    while n == 0 or time.perf_counter() - t0 < 2.0:
+        oracle.gemm(X, codes, s, 4)
+        n += 1
+    dt = (time.perf_counter() - t0) / n
+    b = 4 * N * K // 8 + 2 * N * K // 128 + 2 * K + 2 * N
+    out[name] = {"ms": round(dt * 1e3, 3), "GBps": round(b / dt / 1e9, 4)}
+out["threads"] = oracle.threads()
+print(json.dumps(out))
+"""
+
+
+def one_core_oracle():
+    """The oracle restricted to one thread (OMP_NUM_THREADS=1, a fresh process)."""
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", _ONE_CORE.replace("ROOTDIR", repr(ROOT))],
+                           env=env, capture_output=True, text=True, timeout=120)
+        return json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception as e:  # reported, not fatal: the baseline is context only
+        return {"error": str(e)[:200]}
+
+
 def cpu_oracle_sample(layers, budget_s: float = 12.0):
     """The plain-C oracle on whole layers of the same step for about budget_s."""
     import oracle
@@ -165,7 +323,7 @@ def cpu_oracle_sample(layers, budget_s: float = 12.0):
         done_bytes += algo_bytes(l.N, l.K, r)
         n_layers += 1
     return {"value": done_bytes / t_total / 1e9, "unit": "GB/s", "cores": oracle.threads(),
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(), "one_core": one_core_oracle(),
             "sample": f"{n_layers} layer products of the step (M=1, r in {{4,3,2}}, in step "
                       f"order), fp64 C oracle with OpenMP, {t_total:.1f} s"}
 
@@ -325,8 +483,13 @@ def run_mq(args, ws_n, rank, local):
     peak, peak_kind = read_peaks()
     lay_bytes = np.array([algo_bytes(wl.LLAMA8B[i].N, wl.LLAMA8B[i].K, r)
                           for r in R_LIST for i in range(len(wl.LLAMA8B))], dtype=np.float64)
-    achieved = lay_bytes.sum() / (per.sum() * 1e-3) / 1e9
-    detail = {}
+    # the roofline of the step as timed: algorithmic bytes of the 21 launches
+    # over the graph's device time per step on this GPU (launches overlap
+    # through programmatic dependent launch, so per-launch times do not add up
+    # to the step)
+    achieved = sb / (ms_local / args.steps * 1e-3) / 1e9
+    detail = {"note": "each launch timed alone (an event pair around it stops the overlap "
+                      "with its neighbours): per-launch context, not the step's time"}
     for c, (r, i) in enumerate([(r, i) for r in R_LIST for i in range(len(wl.LLAMA8B))]):
         l = wl.LLAMA8B[i]
         detail[f"r{r}/{l.name}"] = {"us": round(per[c] * 1e3, 3),
@@ -348,27 +511,37 @@ def run_mq(args, ws_n, rank, local):
         "data": "synthetic (seeded; weights, codes and X per the layer recipe)",
         "config": config_dict(),
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                     "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": step_traffic(),
+                     "traffic_unit": "bytes per step (dram read + write of the 21 launches)",
+                     "algorithmic_bytes": sb,
                      "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                                     if peak_kind == "measured" else "fallback 6.65 TB/s",
                      "kernel": "nested_gemv_tc_kernel (one launch per mq_gemm call), "
-                               "all 21 calls of the step",
+                               "all 21 calls of the step, timed as the step",
                      "frac_of_8TBps": round(achieved / 8000.0, 4)},
         "e2e": {"value": aggregate_gbps(ws_n, sb, e2e_ms), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 5)},
         "gpu_launches": len(calls) * args.steps,
         "clocks": clk,
-        "per_layer": detail,
+        "per_launch_isolated": detail,
     }
+    if ws_n == 1:
+        out["per_point"] = {"note": "config 2 points (Llama-3.1-8B gate and q), each shape "
+                                    "alone over rotated weights (L2-cold): median, p10, p90 "
+                                    "of >= 100 launches timed one by one, and the mean of the "
+                                    "same launches back to back",
+                            **run_per_points()}
     return out, layers
 
 
 def run_sweep(args):
     """Per-(layer, M, r) isolated timings for one workload table (configs of
     workloads.CONFIGS), weights rotated over more than twice the L2 so every
-    launch reads its planes from HBM.  Prints one JSON line per point and a
-    markdown table."""
+    launch reads its planes from HBM: median, p10 and p90 of >= 100 launches
+    timed one by one, and the back-to-back mean.  Prints one JSON line per
+    point and a markdown table."""
     import torch
     import nested_bit_weight_b200 as mq
     peak, _ = read_peaks()
@@ -385,12 +558,8 @@ def run_sweep(args):
                     rows.append(dict(r_, layer=layer.name))
                 continue
             codes, s, _ = wl.gen_weights(layer.N, layer.K, wl.layer_seed(ci, li))
-            p0 = mq.pack_parent(torch.from_numpy(codes).cuda(), torch.from_numpy(s).cuda())
+            parents = rotated_parents(mq, codes, s, l2)
             del codes
-            pbytes = p0.planes.numel() * 4 + p0.scales16.numel() * 2
-            copies = max(1, -(-2 * l2 // pbytes))
-            parents = [p0] + [mq.NestedWeights(p0.planes.clone(), p0.scales16.clone(), p0.N, p0.K)
-                              for _ in range(copies - 1)]
             rs = cfg["r"] if cfg["r"] is not None else (wl.QWEN3_R[layer.name],)
             out_rows = []
             for M in cfg["M"]:
@@ -400,49 +569,31 @@ def run_sweep(args):
                 for r in rs:
                     need = mq.mq_gemm_workspace_bytes(M, layer.N, layer.K, r)
                     ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda")
-                    views = [q.view(r) for q in parents]
-                    n_launch = max(len(views), 24)
-                    stream = torch.cuda.Stream()
-                    with torch.cuda.stream(stream):
-                        for v in views:
-                            mq.mq_gemm(X, v, Y, ws)
-                        torch.cuda.synchronize()
-                        g = torch.cuda.CUDAGraph()
-                        with torch.cuda.graph(g, stream=stream):
-                            for j in range(n_launch):
-                                mq.mq_gemm(X, views[j % len(views)], Y, ws)
-                        for _ in range(3):
-                            g.replay()
-                        torch.cuda.synchronize()
-                        e0 = torch.cuda.Event(enable_timing=True)
-                        e1 = torch.cuda.Event(enable_timing=True)
-                        reps = 5
-                        e0.record()
-                        for _ in range(reps):
-                            g.replay()
-                        e1.record()
-                    torch.cuda.synchronize()
-                    us = e0.elapsed_time(e1) * 1e3 / (reps * n_launch)
-                    del g
+                    us, p10, p90, b2b, n = time_point(mq, X, [q.view(r) for q in parents], Y, ws)
                     b = algo_bytes(layer.N, layer.K, r, M)
                     fl = 2.0 * M * layer.N * layer.K
                     row = {"config": ci, "layer": layer.name, "N": layer.N, "K": layer.K, "M": M,
-                           "r": r, "us": round(us, 3), "GBps": round(b / (us * 1e-6) / 1e9, 1),
+                           "r": r, "us": round(us, 3), "us_p10": round(p10, 3),
+                           "us_p90": round(p90, 3), "launches": n,
+                           "us_back_to_back": round(b2b, 3),
+                           "GBps": round(b / (us * 1e-6) / 1e9, 1),
                            "TFLOPs": round(fl / (us * 1e-6) / 1e12, 2),
                            "frac_hbm_measured": round(b / (us * 1e-6) / 1e9 / peak, 3),
                            "frac_8TBps": round(b / (us * 1e-6) / 8e12, 3),
-                           "path": "gemv" if M <= 8 else "tcgen05 gemm"}
+                           "path": "gemv" if mq.uses_gemv(M, layer.N, layer.K, r) else "tcgen05 gemm"}
                     out_rows.append(row)
                     rows.append(row)
                     print(json.dumps(row), flush=True)
             done[key] = out_rows
-            del parents, p0
+            del parents
             torch.cuda.empty_cache()
-    print("| config | layer | N | K | M | r | µs | GB/s | TFLOP/s | frac of measured HBM | frac of 8 TB/s | path |")
-    print("|---|---|---|---|---|---|---|---|---|---|---|---|")
+    print("| config | layer | N | K | M | r | µs median | p10 | p90 | back-to-back µs | GB/s | "
+          "TFLOP/s | frac of measured HBM | frac of 8 TB/s | path |")
+    print("|---|---|---|---|---|---|---|---|---|---|---|---|---|---|---|")
     for r_ in rows:
         print(f"| {r_['config']} | {r_['layer']} | {r_['N']} | {r_['K']} | {r_['M']} | {r_['r']} | "
-              f"{r_['us']} | {r_['GBps']} | {r_['TFLOPs']} | {r_['frac_hbm_measured']} | "
+              f"{r_['us']} | {r_['us_p10']} | {r_['us_p90']} | {r_['us_back_to_back']} | "
+              f"{r_['GBps']} | {r_['TFLOPs']} | {r_['frac_hbm_measured']} | "
               f"{r_['frac_8TBps']} | {r_['path']} |")
 
 

@@ -113,11 +113,12 @@ MQ_API mq_status mq_slice(const mq_weights *parent, int r, mq_weights *out);
 
 /*
  * Bytes of device workspace mq_gemm needs for this problem (0 if none).
- * The workspace holds the M >= 9 GEMM's split-K partial sums, its X operand
- * and arrival counters.  The M <= 8 kernel uses none (tiles shared between
- * CTAs are summed inside thread-block clusters), but for M <= 8 the size
- * still covers the GEMM, which serves shapes the GEMV cannot take and the
- * MQ_GEMV_VIA_GEMM variant.
+ * The workspace holds the M >= 9 GEMM's arrival counters (first 64 KiB) and
+ * the fp32 partial sums of the output tiles whose K range is split between
+ * CTAs.  The M <= 8 kernel uses none (tiles shared between CTAs are summed
+ * inside thread-block clusters), but for M <= 8 the size still covers the
+ * GEMM, which serves shapes the GEMV cannot take and the MQ_GEMV_VIA_GEMM
+ * variant.
  */
 MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
@@ -138,6 +139,20 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * 1 <= w->r <= 8, X/Y/planes/scales/workspace 16-byte aligned, Y does not
  * overlap the inputs.  M == 0 is accepted and does nothing.
  * The fp32 accumulation order is fixed, so results are deterministic.
+ *
+ * Stream order.  The M <= 8 kernel (MQ_GEMV_TC) is launched with programmatic
+ * dependent launch: it may start while the preceding kernel on the stream is
+ * still running, and it begins streaming the weights (planes and scales)
+ * before it waits for that kernel; X is read, and Y and the workspace are
+ * written, only after the preceding kernel has completed and its writes are
+ * visible.  So the weights must not be written by the immediately preceding
+ * kernel on the same stream if that kernel lets its dependents launch early
+ * (griddepcontrol.launch_dependents or its CUDA equivalent).  Kernels that
+ * never do so -- mq_pack, torch's kernels, cudaMemcpy -- are safe: their
+ * dependents start only after they have completed.  Weights written by a
+ * kernel that does trigger early need a cudaStreamSynchronize or an event
+ * wait on another stream before mq_gemm.  The M >= 9 GEMM is launched
+ * without programmatic dependent launch and reads nothing early.
  */
 MQ_API mq_status mq_gemm(const uint16_t *X_dev, const mq_weights *w,
                   int64_t M, int64_t N, int64_t K, uint16_t *Y_dev,
@@ -147,7 +162,7 @@ MQ_API mq_status mq_gemm(const uint16_t *X_dev, const mq_weights *w,
 enum {
     MQ_GEMV_TC = 0,        /* default: 128 rows per tensor-core MMA, int8 operands,
                               decoded weights stored in tensor memory */
-    MQ_GEMV_VIA_GEMM = 1   /* the M >= 9 tcgen05 GEMM (bf16 operands), M padded to 16 */
+    MQ_GEMV_VIA_GEMM = 1   /* the M >= 9 tcgen05 GEMM (bf16 operands), X rows padded to 32 */
 };
 
 /*
@@ -161,6 +176,21 @@ MQ_API mq_status mq_set_gemv_variant(int variant);
 
 /* The M <= 8 kernel in use (MQ_GEMV_TC or MQ_GEMV_VIA_GEMM). */
 MQ_API int mq_get_gemv_variant(void);
+
+/* Kernels that serve an mq_gemm call. */
+enum {
+    MQ_KERNEL_GEMV = 1,    /* the M <= 8 tensor-core GEMV */
+    MQ_KERNEL_GEMM = 2     /* the tcgen05 GEMM */
+};
+
+/*
+ * Which kernel mq_gemm(M, N, K, r) would run under the current variant
+ * (host only, no device work): MQ_KERNEL_GEMV or MQ_KERNEL_GEMM, 0 for an
+ * invalid problem (M < 1, N < 1, K not a positive multiple of 128, r outside
+ * 1..8).  Lets a caller or a benchmark label its timings; it has no effect on
+ * the call itself.
+ */
+MQ_API int mq_gemm_kernel(int64_t M, int64_t N, int64_t K, int r);
 
 /*
  * Test helper: codes_out[n, k] = q_r[n, k] read back from the first r planes

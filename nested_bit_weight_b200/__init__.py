@@ -17,7 +17,7 @@ __all__ = [
     "mq_plane_bytes", "mq_scale_bytes", "mq_pack", "mq_slice", "mq_gemm",
     "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
     "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
-    "mq_device_status",
+    "mq_device_status", "mq_gemm_kernel", "uses_gemv", "KERNEL_GEMV", "KERNEL_GEMM",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "mq_version": (ctypes.c_char_p, []),
         "mq_set_gemv_variant": (I, [I]),
         "mq_get_gemv_variant": (I, []),
+        "mq_gemm_kernel": (I, [I64, I64, I64, I]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -110,6 +111,18 @@ def mq_set_gemv_variant(variant: int) -> None:
 
 def mq_get_gemv_variant() -> int:
     return lib.mq_get_gemv_variant()
+
+
+KERNEL_GEMV, KERNEL_GEMM = 1, 2
+
+
+def mq_gemm_kernel(M: int, N: int, K: int, r: int) -> int:
+    """KERNEL_GEMV or KERNEL_GEMM: the kernel mq_gemm would run (0: invalid)."""
+    return lib.mq_gemm_kernel(M, N, K, r)
+
+
+def uses_gemv(M: int, N: int, K: int, r: int) -> bool:
+    return mq_gemm_kernel(M, N, K, r) == KERNEL_GEMV
 
 
 def mq_device_status() -> None:

@@ -158,6 +158,11 @@ mq_status mq_set_gemv_variant(int variant) {
 
 int mq_get_gemv_variant(void) { return __atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED); }
 
+int mq_gemm_kernel(int64_t M, int64_t N, int64_t K, int r) {
+    if (M < 1 || N < 1 || K < kGroup || K % kGroup || r < 1 || r > 8) return 0;
+    return M <= kGemvMaxM && small_m_uses_gemv(M, N, K, r) ? MQ_KERNEL_GEMV : MQ_KERNEL_GEMM;
+}
+
 mq_status mq_last_error(void) { return g_last; }
 
 mq_status mq_device_status(void) {

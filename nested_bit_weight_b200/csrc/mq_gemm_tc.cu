@@ -1,17 +1,48 @@
-// Batched path (M >= 9): tcgen05 tensor-core GEMM over decoded r-bit tiles.
+// Batched path (M >= 9, and the M <= 8 fallback): tcgen05 tensor-core GEMM
+// over decoded r-bit tiles.
 //
 // The r-bit levels v_r = 2^(8-r) q_r + 2^(7-r) - 128 are exact in bf16 (at
 // most 8 significant bits), so the MMA operands are exact:
 //     D_g[n, m] = sum_{k in group g} v_r[n, k] * x[m, k]     (fp32, in TMEM)
 //     Y[m, n]   = sum_g s[n, g] * D_g[n, m]                  (fp32 registers)
-// One CTA owns 128 weight rows and BM rows of X.  Per 128-column group it
-// decodes its rows' r planes into a 128 x 128 bf16 tile (K-major, 128-byte
-// swizzle) in shared memory, stages the matching X tile, issues eight
-// 128 x BM x 16 MMAs from one thread, and folds the group into fp32
-// accumulators with the group's scale.  Decoding emits columns within each
-// 32-column word in the order 4e + j <- k = 8j + e, so X is first copied into
-// the workspace in that order (prep kernel); the contraction is unchanged.
+// (the fp16 scale is applied per 128-column group in fp32: folding s * v
+// into one 16-bit operand rounds every weight, which the tolerance does not
+// allow on large layers).
+//
+// Work: items (X block mb, 128-row tile t, group g) in that order, cut into
+// one contiguous range per CTA (about 148 CTAs, one per SM).  A tile whose
+// groups are spread over several CTAs is summed by the CTA that finishes it
+// last, from the fp32 partial sums the others leave in the workspace, in
+// CTA order (deterministic).
+//
+// Roles (warp-specialised; every hand-off an mbarrier):
+//   decode warps    8 (two threads per weight row) or 4 (BM = 128): each
+//                   thread copies its share of the row's r plane words of the
+//                   items ahead into a ring of shared memory with cp.async
+//                   (up to 16 items, up to 96 KB in flight per SM), then
+//                   decodes the current group to bf16 levels in natural column
+//                   order and stores them to its TMEM lane in one of two A
+//                   stages (tcgen05.st; the MMA reads A from TMEM);
+//   X warp          one thread loads the group's BM x 128 block of X into one
+//                   of 3 or 4 B stages with one tensor-map (TMA) copy, in the
+//                   same layout; rows beyond M read as zeros;
+//   MMA warp        one thread issues eight 128 x BM x 16 MMAs per group into
+//                   one of two TMEM accumulators and commits to the A stage,
+//                   B stage (free) and accumulator (full) barriers;
+//   fold warps      4 (BM <= 64) or 8 (BM = 128), one or two per TMEM lane
+//                   quarter: y += s[n, g] * D_g, the tile's fp32 sums kept in
+//                   registers until the tile ends.
+// Every wait is bounded (about a second); a wait that gives up sets a CTA
+// abort flag that ends the others at once, and a device flag read by
+// mq_device_status.  Arrival tickets always return to zero, also after a
+// timeout (the output is then unspecified).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+
 #include "mq_common.cuh"
+#include "mq_bits.cuh"
 #include "mq_sm100.cuh"
 
 namespace mq {
@@ -19,316 +50,492 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 128;
-constexpr int kTileN = 128;
+constexpr int kTileN = 128;                  // weight rows per tile (MMA M)
+constexpr int kMinItems = 4;                 // fewest items a CTA is given
 
-__device__ unsigned int g_tc_timeout;      // set when a bounded wait gave up
+// Per (r, BM) configuration.  14 warps, so 128 registers a thread: decode
+// warps (two threads per row, or one for BM = 128), fold warps, then the X
+// and MMA warps.  Shared memory: kNX X stages and a ring of kD items of plane
+// words (the loads in flight that keep HBM busy).  Tensor memory: two A
+// stages (64 columns each) and two accumulators (BM columns each).
+__host__ __device__ constexpr int ring_items(int r, int BM) {
+    return (96 * 1024) / (r * 2048) < 16 ? (96 * 1024) / (r * 2048) : 16;
+}
+__host__ __device__ constexpr int x_stages(int BM) { return BM == 128 ? 3 : 4; }
+__host__ __device__ constexpr size_t tc_smem_bytes(int r, int BM) {
+    return 1024 + (size_t)x_stages(BM) * BM * 256 + (size_t)ring_items(r, BM) * r * 2048 + 256;
+}
 
-// Stage A/B/C transposition (same network as the GEMV): byte j of out[e] is
-// q_r << (8 - r) of column 8 j + e.
+template <int R, int BM>
+struct TcCfg {
+    static constexpr int kDecW = BM == 128 ? 4 : 8;
+    static constexpr int kFoldW = BM == 128 ? 8 : 4;
+    static constexpr int kThreads = (kDecW + kFoldW + 2) * 32;
+    static constexpr int kParts = kDecW / 4;                  // decode threads per row
+    static constexpr int kWP = 4 / kParts;                    // plane words per decode thread
+    static constexpr int kNX = x_stages(BM);
+    static constexpr int kD = ring_items(R, BM);
+    static constexpr uint32_t kXStage = BM * 256;             // BM rows x 128 bf16
+    static constexpr uint32_t kTmemCols = 128 + 2 * BM <= 256 ? 256 : 512;
+    static constexpr uint32_t kSlot = R * 2048;               // plane words of one item
+};
+
+__device__ unsigned int g_tc_timeout;        // set when a bounded wait gave up
+
+// The 16 A words of one 32-column plane word, before centring: word 4b + j
+// holds columns 8b + 2j and 8b + 2j + 1 (low, high half), as bf16 256 + e
+// for r <= 6 and as the bytes e0 | e1 << 8 for r >= 7 (e = q_r << (8 - r)).
 template <int R>
-__device__ __forceinline__ void tc_planes_to_bytes(const uint32_t (&P)[8], uint32_t (&out)[8]) {
-    uint32_t A[4][2];
+__host__ __device__ __forceinline__ void word_pairs(const uint32_t (&P)[8], uint32_t (&v)[16]) {
+    uint32_t E[8];
+    if constexpr (R <= 6) {
+        half_byte_words<R>(P, E);                      // byte b of E[e]: (column 8b + e) / 2
 #pragma unroll
-    for (int pp = 0; pp < 4; ++pp) {
-        const uint32_t a = (2 * pp < R) ? P[2 * pp] : 0u;
-        const uint32_t b = (2 * pp + 1 < R) ? P[2 * pp + 1] : 0u;
-        A[pp][1] = (a & 0xAAAAAAAAu) | ((b >> 1) & 0x55555555u);
-        A[pp][0] = ((a << 1) & 0xAAAAAAAAu) | (b & 0x55555555u);
-    }
-    uint32_t Bq[2][4];
+        for (int b = 0; b < 4; ++b)
 #pragma unroll
-    for (int qd = 0; qd < 2; ++qd)
+            for (int j = 0; j < 4; ++j) v[4 * b + j] = bf16_pair_from_halves(E[2 * j], E[2 * j + 1], b);
+    } else {
+        byte_words<R>(P, E);                           // byte b of E[e]: column 8b + e
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-            const uint32_t x = A[2 * qd][c], y = A[2 * qd + 1][c];
-            Bq[qd][c] = ((x << 2) & 0xCCCCCCCCu) | (y & 0x33333333u);
-            Bq[qd][2 + c] = (x & 0xCCCCCCCCu) | ((y >> 2) & 0x33333333u);
-        }
+        for (int b = 0; b < 4; ++b)
 #pragma unroll
-    for (int d = 0; d < 4; ++d) {
-        const uint32_t x = Bq[0][d], y = Bq[1][d];
-        out[d] = ((x << 4) & 0xF0F0F0F0u) | (y & 0x0F0F0F0Fu);
-        out[4 + d] = (x & 0xF0F0F0F0u) | ((y >> 4) & 0x0F0F0F0Fu);
+            for (int j = 0; j < 4; ++j) v[4 * b + j] = byte_pair(E[2 * j], E[2 * j + 1], b);
     }
 }
 
-// Two bf16 levels (bytes j0 and j0+1 of E, E's bytes hold q_r << (8 - r)).
+// Centre a word of word_pairs to the two bf16 levels v_r = e - 128 + 2^(7-r).
 template <int R>
-__device__ __forceinline__ uint32_t levels_bf16x2(uint32_t E, int j0) {
+__device__ __forceinline__ uint32_t centre(uint32_t w) {
     if constexpr (R <= 6) {
-        // bf16 bits 0x4380 | (b >> 1) encode 256 + b (b even): one byte
-        // permute builds two of them, one exact subtraction centres them
-        // (384 - 2^(7-r) is exact in bf16 for r <= 6).
-        const uint32_t F = ((E >> 1) & 0x7F7F7F7Fu) | 0x80808080u;
-        const uint32_t h = __byte_perm(F, 0x43434343u, j0 == 0 ? 0x4140 : 0x4342);
+        // one exact bf16 subtraction (384 - 2^(7-r) is exact in bf16 for r <= 6)
         const float c = 384.0f - (float)(1 << (7 - R));
-        const __nv_bfloat162 off = __floats2bfloat162_rn(c, c);
-        __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&h);
-        v = __hsub2(v, off);
+        __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&w);
+        v = __hsub2(v, __floats2bfloat162_rn(c, c));
         return *reinterpret_cast<uint32_t *>(&v);
     } else {
-        // through fp32: 2^22 + b has a 0.5 ulp, so subtracting
+        // through fp32: 2^22 + e has a 0.5 ulp, so subtracting
         // 2^22 + 128 - 2^(7-r) is exact and leaves v_r
         constexpr float c = 4194432.0f - (R == 8 ? 0.5f : 1.0f);
-        const uint32_t b0 = (E >> (8 * j0)) & 0xFFu, b1 = (E >> (8 * j0 + 8)) & 0xFFu;
-        const float f0 = __uint_as_float(0x4A800000u | (b0 << 1)) - c;
-        const float f1 = __uint_as_float(0x4A800000u | (b1 << 1)) - c;
+        const float f0 = __uint_as_float(0x4A800000u | ((w & 0xFFu) << 1)) - c;
+        const float f1 = __uint_as_float(0x4A800000u | ((w >> 8) << 1)) - c;
         __nv_bfloat162 v = __floats2bfloat162_rn(f0, f1);
         return *reinterpret_cast<uint32_t *>(&v);
     }
 }
 
-// X rows, each 32-column block permuted to the decode order 4e + j <- 8j + e;
-// rows M..Mp-1 are zero.
-__global__ void __launch_bounds__(256)
-x_permute_kernel(const uint16_t *__restrict__ X, int M, int Mp, int64_t K,
-                 uint16_t *__restrict__ Xp) {
-    const int64_t blocks = (int64_t)Mp * (K / 32);
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < blocks;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t m = i / (K / 32), b = i % (K / 32);
-        uint16_t in[32], out[32];
-        if (m < M) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(X + m * K + b * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) *reinterpret_cast<uint4 *>(in + 8 * v) = src[v];
-        } else {
-#pragma unroll
-            for (int v = 0; v < 32; ++v) in[v] = 0;
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) out[4 * e + j] = in[8 * j + e];
-        uint4 *dst = reinterpret_cast<uint4 *>(Xp + m * K + b * 32);
-#pragma unroll
-        for (int v = 0; v < 4; ++v) dst[v] = *reinterpret_cast<uint4 *>(out + 8 * v);
+// Kernel arguments.
+struct GArgs {
+    CUtensorMap xmap;           // X as (64 columns, M rows, K/64 halves), boxes 64 x BM x 2
+    const uint32_t *planes;     // tiled planes
+    const __half *scales;       // tiled fp16 scales
+    __nv_bfloat16 *Y;           // M x N
+    float *part;                // partial sums of shared tiles [tile * maxc + slot][BM][128]
+    unsigned *tickets;          // one per (X block, tile)
+    int64_t N, K;
+    int M, T, G, MB, P, maxc;   // rows of X, row tiles, groups, X blocks, CTAs, CTAs per tile
+    int64_t plane_words;        // uint32 words of one plane
+};
+
+__host__ __device__ inline int64_t range_first(int64_t b, int64_t W, int P) { return b * W / P; }
+__host__ __device__ inline int cta_of(int64_t u, int64_t W, int P) { return (int)(((u + 1) * P - 1) / W); }
+
+// Wait (bounded) for the last phase issued to every slot of a ring of n
+// barriers that received `issued` phases in slot order.
+__device__ __forceinline__ void drain_ring(uint64_t *bars, int n, int issued) {
+    for (int s = 0; s < n && s < issued; ++s) {
+        const int k = (issued - 1 - s) / n + 1;
+        mbar_wait_bounded(bars + s, (uint32_t)(k - 1) & 1u);
     }
 }
 
 template <int R, int BM>
-__global__ void __launch_bounds__(kTcThreads)
-gemm_tc_kernel(const uint16_t *__restrict__ Xp, const uint32_t *__restrict__ planes,
-               const __half *__restrict__ scales, int M, int64_t N, int64_t K,
-               int groups_per_split, int KS, float *__restrict__ part,
-               unsigned *__restrict__ tickets, __nv_bfloat16 *__restrict__ Y) {
-    constexpr int kCols = BM < 32 ? 32 : BM;                // TMEM columns (power of 2)
+__global__ void __launch_bounds__(TcCfg<R, BM>::kThreads, 1)
+gemm_tc_kernel(const __grid_constant__ GArgs a) {
+    using C = TcCfg<R, BM>;
+    constexpr int kDecW = C::kDecW, kFoldW = C::kFoldW, kNX = C::kNX, kD = C::kD, kWP = C::kWP;
+    constexpr int kFoldW0 = kDecW, kXW = kDecW + kFoldW, kMmaW = kXW + 1;
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTileN, BM);
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    // align the base by an offset so the compiler keeps the shared address space
-    uint8_t *base = smem_raw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smem_raw)) & 1023u)) & 1023u);
-    uint8_t *sA = base;
-    uint8_t *sB = base + 2 * kTileN * 128;
-    __shared__ uint64_t bar;
-    __shared__ uint32_t tmem_slot;
-    __shared__ int s_last;
+    constexpr uint32_t kD0 = 128;                              // TMEM: A stages [0, 128), accumulators after
+    constexpr int kCW = BM * 4 / kFoldW;                       // columns per fold thread
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *sX = smem;                                        // [kNX][2 halves][BM][128 B]
+    uint8_t *ring = sX + kNX * C::kXStage;                     // [kD][plane][part][128][kWP words]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kD * C::kSlot);
+    uint64_t *afull = bars, *aempty = bars + 2, *dfull = bars + 4, *dempty = bars + 6;
+    uint64_t *xfull = bars + 8, *xempty = xfull + kNX;
+    // [0] abort  [2] items issued to the MMA  [3] X items loaded
+    // [4] tiles this CTA sums at the end  [5, 6] their indices  [7, 8] their CTA counts
+    volatile int *flags = reinterpret_cast<volatile int *>(xempty + kNX);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xempty + kNX) + 10;
 
-    const int t = threadIdx.x, warp = t >> 5;
-    const int64_t G = K / kGroup;
-    const int64_t n0 = (int64_t)blockIdx.x * kTileN;
-    const int m0 = blockIdx.y * BM;
-    const int64_t gbeg = (int64_t)blockIdx.z * groups_per_split;
-    const int64_t gend = (gbeg + groups_per_split < G) ? gbeg + groups_per_split : G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t W = (int64_t)a.MB * a.T * a.G;
+    const int64_t u0 = range_first(blockIdx.x, W, a.P), u1 = range_first(blockIdx.x + 1, W, a.P);
+    const int L = (int)(u1 - u0);
+    const int G = a.G, TG = a.T * a.G;
 
-    if (warp == 0) { tmem_alloc(&tmem_slot, kCols); tmem_relinquish(); }
-    if (t == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(afull + i, kDecW);
+            mbar_init(aempty + i, 1);
+            mbar_init(dfull + i, 1);
+            mbar_init(dempty + i, kFoldW);
+        }
+        for (int i = 0; i < kNX; ++i) {
+            mbar_init(xfull + i, 1);
+            mbar_init(xempty + i, 1);
+        }
+        for (int i = 0; i < 9; ++i) flags[i] = 0;      // [1] unused
+        fence_mbar_init();
+    }
+    if (warp == kMmaW) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t taddr = tmem_slot;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(tmem_slot);
 
-    const int64_t n = n0 + t;
-    const bool row_ok = n < N;
-    const int64_t plane_words = (N + 127) / 128 * 128 * (K / 32);   // tiled planes
-    float y[BM];
+    if (warp < kDecW) {
+        // ------------------------------------------------------------ decode
+        const int n = threadIdx.x & (kTileN - 1);              // row of the tile
+        const int hp = threadIdx.x >> 7;                       // part of the row
+        const int w0 = hp * kWP;                               // first word (32 columns) of the part
+        uint8_t *mine = ring + ((size_t)hp * kTileN + n) * (kWP * 4);   // + slot, + plane
+        constexpr uint32_t kPlaneStride = C::kParts * kTileN * kWP * 4; // 2 KB
+        // the plane words of item j (this thread's part) into ring slot j % kD
+        auto issue = [&](int j) {
+            const uint32_t *src = a.planes + ((u0 + j) % TG) * 512 + n * 4 + w0;
+            uint8_t *dst = mine + (j % kD) * C::kSlot;
 #pragma unroll
-    for (int c = 0; c < BM; ++c) y[c] = 0.f;
-    uint32_t phase = 0;
-    bool ok = true;
-
-    // The next group's plane words, scale and X chunks are loaded into
-    // registers while the current group is decoded and multiplied (the loop
-    // is otherwise bound by the global-load latency of every group).
-    constexpr bool kPrefetch = R * 8 + BM <= 96;
-    constexpr int kXv = BM * 16 / kTcThreads;            // X chunks per thread (BM <= 32)
-    uint4 pvn[R];
-    float sn = 0.f;
-    uint4 xvn[kXv > 0 && BM <= 32 ? kXv : 1];
-    auto load_group = [&](int64_t g) {
-#pragma unroll
-        for (int p = 0; p < R; ++p)
-            pvn[p] = *reinterpret_cast<const uint4 *>(planes + p * plane_words +
-                                                      ((int64_t)blockIdx.x * G + g) * 512 + t * 4);
-        sn = __half2float(scales[((int64_t)blockIdx.x * G + g) * 128 + t]);
-        if constexpr (BM <= 32) {
-#pragma unroll
-            for (int i = 0; i < kXv; ++i) {
-                const int idx = t + i * kTcThreads, row = idx >> 4, c = idx & 15;
-                xvn[i] = *reinterpret_cast<const uint4 *>(Xp + (int64_t)(m0 + row) * K + g * kGroup + c * 8);
+            for (int p = 0; p < R; ++p) {
+                if constexpr (kWP == 4) cp_async_16(dst + p * kPlaneStride, src + p * a.plane_words);
+                else cp_async_8(dst + p * kPlaneStride, src + p * a.plane_words);
             }
+        };
+#pragma unroll 1
+        for (int j = 0; j < kD; ++j) {
+            if (j < L) issue(j);
+            cp_async_commit();
         }
-    };
-    if (kPrefetch && gbeg < gend) load_group(gbeg);
-
-    for (int64_t g = gbeg; g < gend; ++g) {
-        // ---- decode this thread's row of the A tile
-        uint4 pv[R];
-        float s;
-        uint4 xv[kXv > 0 && BM <= 32 ? kXv : 1];
-        if constexpr (kPrefetch) {
+        for (int i = 0; i < L; ++i) {
+            const int st = i & 1;
+            cp_async_wait<kD - 1>();                           // item i's words are in
+            uint32_t pv[R][kWP];
+            const uint8_t *src = mine + (i % kD) * C::kSlot;
 #pragma unroll
-            for (int p = 0; p < R; ++p) pv[p] = pvn[p];
-            s = sn;
-            if constexpr (BM <= 32) {
-#pragma unroll
-                for (int i = 0; i < kXv; ++i) xv[i] = xvn[i];
+            for (int p = 0; p < R; ++p) {
+                if constexpr (kWP == 4) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(src + p * kPlaneStride);
+                    pv[p][0] = v.x; pv[p][1] = v.y; pv[p][2] = v.z; pv[p][3] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(src + p * kPlaneStride);
+                    pv[p][0] = v.x; pv[p][1] = v.y;
+                }
             }
-            if (g + 1 < gend) load_group(g + 1);
-        } else {
+            if (i + kD < L) issue(i + kD);                     // refill the slot just read
+            cp_async_commit();
+            bool ok = i < 2 || mbar_wait_backoff(aempty + st, (uint32_t)((i >> 1) - 1) & 1u, flags);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            tc_fence_after();
+            // this row's 32-column words -> 16 TMEM columns each of A stage st
+            const uint32_t a_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(st * 64);
 #pragma unroll
-            for (int p = 0; p < R; ++p)
-                pv[p] = *reinterpret_cast<const uint4 *>(planes + p * plane_words +
-                                                         ((int64_t)blockIdx.x * G + g) * 512 + t * 4);
-            s = __half2float(scales[((int64_t)blockIdx.x * G + g) * 128 + t]);
+            for (int w = 0; w < kWP; ++w) {
+                uint32_t P[8], v[16];
+#pragma unroll
+                for (int p = 0; p < 8; ++p) P[p] = p < R ? pv[p < R ? p : 0][w] : 0u;
+                word_pairs<R>(P, v);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = centre<R>(v[j]);
+                tmem_st16(a_row + (uint32_t)(16 * (w0 + w)), v);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(afull + st);
         }
+        cp_async_wait<0>();                                    // no copy left in flight
+    } else if (warp < kXW) {
+        // -------------------------------------------------------------- fold
+        const int f = warp - kFoldW0, q = f & 3, c0 = (f >> 2) * kCW;
+        const int n = 32 * q + lane;                           // row of the tile
+        const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        float y[kCW];
 #pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            uint32_t P[8], E[8];
-#pragma unroll
-            for (int p = 0; p < 8; ++p) {
-                const uint4 &v = pv[p < R ? p : 0];
-                P[p] = p < R ? (w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w) : 0u;
-            }
-            tc_planes_to_bytes<R>(P, E);
-#pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {              // 8 columns: words 2cq, 2cq+1
-                uint4 chunk;
-                chunk.x = levels_bf16x2<R>(E[2 * cq], 0);
-                chunk.y = levels_bf16x2<R>(E[2 * cq], 2);
-                chunk.z = levels_bf16x2<R>(E[2 * cq + 1], 0);
-                chunk.w = levels_bf16x2<R>(E[2 * cq + 1], 2);
-                const int c = 4 * w + cq;                 // 16-byte chunk of the row
-                *reinterpret_cast<uint4 *>(sA + (c >> 3) * (kTileN * 128) +
-                                           sw128_offset(t, c & 7)) = chunk;
-            }
-        }
-        // ---- stage the X tile (already in decode order)
-        if constexpr (kPrefetch && BM <= 32) {
-#pragma unroll
-            for (int i = 0; i < kXv; ++i) {
-                const int idx = t + i * kTcThreads, row = idx >> 4, c = idx & 15;
-                *reinterpret_cast<uint4 *>(sB + (c >> 3) * (BM * 128) + sw128_offset(row, c & 7)) = xv[i];
-            }
-        } else {
-            for (int idx = t; idx < BM * 16; idx += kTcThreads) {
-                const int row = idx >> 4, c = idx & 15;
-                const uint4 v = *reinterpret_cast<const uint4 *>(
-                    Xp + (int64_t)(m0 + row) * K + g * kGroup + c * 8);
-                *reinterpret_cast<uint4 *>(sB + (c >> 3) * (BM * 128) + sw128_offset(row, c & 7)) = v;
-            }
-        }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        // ---- eight K=16 MMAs into TMEM, one issuing thread
-        if (t == 0) {
+        for (int j = 0; j < kCW; ++j) y[j] = 0.f;
+        bool ok = true;
+        int64_t tile_u0 = u0 - (u0 % G);                       // first item of the current tile
+        float sn = L > 0 ? __half2float(a.scales[(u0 % TG) * 128 + n]) : 0.f;
+        for (int i = 0; i < L; ++i) {
+            const int64_t u = u0 + i;
+            const int db = i & 1;
+            const float s = sn;
+            if (i + 1 < L) sn = __half2float(a.scales[((u + 1) % TG) * 128 + n]);
+            ok = mbar_wait_backoff(dfull + db, (uint32_t)(i >> 1) & 1u, flags);
+            // every fold thread takes the same branch (the tile end below
+            // has barriers of its own)
+            ok = named_sync_and(3, kFoldW * 32, ok);
+            if (!ok) break;
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const int h = ks >> 2, kk = ks & 3;
-                const uint64_t ad = smem_desc_sw128(smem_u32(sA + h * (kTileN * 128) + kk * 32));
-                const uint64_t bd = smem_desc_sw128(smem_u32(sB + h * (BM * 128) + kk * 32));
-                mma_bf16(taddr, ad, bd, kIdesc, ks > 0 ? 1u : 0u);
+            for (int cb = 0; cb < kCW; cb += 16) {
+                uint32_t v[16];
+                tmem_ld16(tmem + lane_base + kD0 + (uint32_t)(db * BM + c0 + cb), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) y[cb + j] = fmaf(s, __uint_as_float(v[j]), y[cb + j]);
             }
-            mma_commit(&bar);
-        }
-        const bool mine = mbar_wait_bounded(&bar, phase);
-        phase ^= 1u;
-        if (!__syncthreads_and(mine)) { ok = false; break; }
-        tc_fence_after();
-
-        // ---- fold this group in: y[m] += s[n, g] * D_g[n, m]
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(dempty + db);
+            // the tile ends with this item (or the range does): write it out
+            const bool tile_end = (u + 1) % G == 0 || i == L - 1;
+            if (!tile_end) continue;
+            const int64_t tu = u / G;                          // tile index over (mb, t)
+            const int mb = (int)(tu / a.T), t = (int)(tu % a.T);
+            const int64_t tn0 = tile_u0, tn1 = tile_u0 + G;    // the tile's items
+            const int64_t nrow = (int64_t)t * kTileN + n;
+            const int mlim = a.M - (mb * BM + c0);             // columns of this thread inside M
+            const bool own = tn0 >= u0 && tn1 <= u1;           // the whole tile is in this range
+            int cf = 0, cnt = 1;
+            if (!own) {
+                cf = cta_of(tn0, W, a.P);
+                cnt = cta_of(tn1 - 1, W, a.P) - cf + 1;
+            }
+            // own tile: Y directly; shared tile: this CTA's fp32 partial sums,
+            // as float4 (4 columns of one row) at [column / 4][row]
+            float4 *pp = reinterpret_cast<float4 *>(a.part + ((size_t)tu * a.maxc + (own ? 0 : blockIdx.x - cf)) * (BM * kTileN)) +
+                         (c0 / 4) * kTileN + n;
+            __nv_bfloat16 *yp = a.Y + (int64_t)(mb * BM + c0) * a.N + nrow;
+            if (own ? nrow < a.N : true) {
 #pragma unroll
-        for (int cb = 0; cb < BM / 16; ++cb) {
-            float v[16];
-            { uint32_t u[16]; tmem_ld16(taddr + ((uint32_t)(32 * warp) << 16) + cb * 16, u); for (int q = 0; q < 16; ++q) v[q] = __uint_as_float(u[q]); }
-            tmem_ld_wait();
+                for (int j = 0; j < kCW; j += 4) {
+                    if (!own) {
+                        pp[(j / 4) * kTileN] = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+                    } else {
 #pragma unroll
-            for (int i = 0; i < 16; ++i) y[cb * 16 + i] = fmaf(s, v[i], y[cb * 16 + i]);
+                        for (int q = 0; q < 4; ++q)
+                            if (j + q < mlim) yp[(int64_t)(j + q) * a.N] = __float2bfloat16_rn(y[j + q]);
+                    }
+                }
+            }
+            if (!own) {
+                // take a ticket; the last CTA to arrive sums the tile after
+                // its own range (all threads of the CTA, in CTA order)
+                __threadfence();
+                named_sync(3, kFoldW * 32);
+                if (f == 0 && lane == 0) {
+                    if (atomicAdd(a.tickets + tu, 1u) == (unsigned)(cnt - 1)) {
+                        a.tickets[tu] = 0u;                    // every part is in: reset for the next launch
+                        const int k = flags[4];
+                        flags[5 + k] = (int)tu;
+                        flags[7 + k] = cnt;
+                        flags[4] = k + 1;
+                    }
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kCW; ++j) y[j] = 0.f;
+            tile_u0 += G;
         }
-        tc_fence_before();
-        __syncthreads();
+        if (!ok && f == 0 && lane == 0) {
+            // a wait gave up: still take the tickets of the shared tiles left
+            // in the range so that they return to zero (Y is then unspecified)
+            for (int64_t tn0 = tile_u0; tn0 < u1; tn0 += G) {
+                const int64_t tn1 = tn0 + G;
+                if (tn0 >= u0 && tn1 <= u1) continue;
+                const int cnt = cta_of(tn1 - 1, W, a.P) - cta_of(tn0, W, a.P) + 1;
+                const int64_t tu = tn0 / G;
+                if (atomicAdd(a.tickets + tu, 1u) == (unsigned)(cnt - 1)) a.tickets[tu] = 0u;
+            }
+        }
+    } else if (warp == kXW) {
+        // ----------------------------------------------------------------- X
+        if (lane == 0) {
+            for (int i = 0; i < L; ++i) {
+                const int xs = i % kNX, kx = i / kNX;
+                const int64_t u = u0 + i;
+                const int mb = (int)(u / TG), g = (int)(u % G);
+                if (kx > 0 && !mbar_wait_abortable(xempty + xs, (uint32_t)(kx - 1) & 1u, flags)) break;
+                mbar_expect_tx(xfull + xs, C::kXStage);
+                tma_load_3d(sX + xs * C::kXStage, &a.xmap, 0, mb * BM, 2 * g, xfull + xs);
+                flags[3] = i + 1;
+            }
+        }
+    } else {
+        // --------------------------------------------------------------- MMA
+        if (lane == 0) {
+            const uint32_t x0 = smem_u32(sX);
+            for (int i = 0; i < L; ++i) {
+                const int st = i & 1, db = i & 1, xs = i % kNX;
+                if (!mbar_wait_abortable(afull + st, (uint32_t)(i >> 1) & 1u, flags)) break;
+                if (!mbar_wait_abortable(xfull + xs, (uint32_t)(i / kNX) & 1u, flags)) break;
+                if (i >= 2 && !mbar_wait_abortable(dempty + db, (uint32_t)((i >> 1) - 1) & 1u, flags)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    const int h = ks >> 2, kk = ks & 3;
+                    const uint64_t bd = smem_desc_sw128(x0 + xs * C::kXStage + h * (BM * 128) + kk * 32);
+                    mma_bf16_ts(tmem + kD0 + (uint32_t)(db * BM), tmem + (uint32_t)(st * 64 + 8 * ks), bd, kIdesc,
+                                ks > 0 ? 1u : 0u);
+                }
+                mma_commit(aempty + st);                       // A stage free
+                mma_commit(xempty + xs);                       // X stage free
+                mma_commit(dfull + db);                        // accumulator full
+                flags[2] = i + 1;
+            }
+        }
     }
 
-    if (!ok) {
-        if (t == 0) atomicOr(&g_tc_timeout, 1u);
-    } else if (KS == 1) {
-        if (row_ok)
-#pragma unroll
-            for (int c = 0; c < BM; ++c)
-                if (m0 + c < M) Y[(int64_t)(m0 + c) * N + n] = __float2bfloat16_rn(y[c]);
-    } else {
-        if (row_ok) {
-#pragma unroll
-            for (int c = 0; c < BM; ++c)
-                if (m0 + c < M) part[((int64_t)blockIdx.z * M + m0 + c) * N + n] = y[c];
-            __threadfence();
-        }
-        __syncthreads();
-        const unsigned tk = blockIdx.y * gridDim.x + blockIdx.x;
-        if (t == 0) s_last = atomicAdd(&tickets[tk], 1u) == (unsigned)KS - 1;
-        __syncthreads();
-        if (s_last) {
-            __threadfence();
-            if (row_ok)
-                for (int c = 0; c < BM && m0 + c < M; ++c) {
-                    float a = 0.f;
-                    for (int z = 0; z < KS; ++z)
-                        a += __ldcg(part + ((int64_t)z * M + m0 + c) * N + n);
-                    Y[(int64_t)(m0 + c) * N + n] = __float2bfloat16_rn(a);
-                }
-            if (t == 0) tickets[tk] = 0u;
-        }
+    // ---- end: let the copies, MMAs and barrier arrivals issued land before
+    // the CTA exits (already the case unless a wait gave up)
+    __syncwarp();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const int issued = flags[2], loaded = flags[3];
+        drain_ring(aempty, 2, issued);
+        drain_ring(xempty, kNX, issued);
+        drain_ring(dfull, 2, issued);
+        drain_ring(xfull, kNX, loaded);
+        if (flags[0]) atomicOr(&g_tc_timeout, 1u);
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) { tc_fence_after(); tmem_dealloc(taddr, kCols); }
+    if (warp == kMmaW) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+
+    // ---- shared tiles whose last part this CTA delivered: Y = sum of the
+    // parts in CTA order, every thread of the CTA taking float4 positions
+    if (flags[0]) return;
+    __threadfence();
+    for (int k = 0; k < flags[4]; ++k) {
+        const int64_t tu = flags[5 + k];
+        const int cnt = flags[7 + k];
+        const int mb = (int)(tu / a.T), t = (int)(tu % a.T);
+        const float4 *p0 = reinterpret_cast<const float4 *>(a.part + (size_t)tu * a.maxc * (BM * kTileN));
+        constexpr int kPos = BM * kTileN / 4;                  // float4 positions of one part
+        constexpr int kPer = (kPos + C::kThreads - 1) / C::kThreads;
+        constexpr int kBatch = kPer <= 5 ? 2 : 1;              // parts loaded per round
+        float4 acc[kPer];
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sl = 0; sl < cnt; sl += kBatch) {
+            float4 v[kBatch][kPer];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    const int pos = threadIdx.x + e * C::kThreads;
+                    v[b][e] = (sl + b < cnt && pos < kPos) ? __ldcg(p0 + (size_t)(sl + b) * kPos + pos)
+                                                           : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+#pragma unroll
+                for (int e = 0; e < kPer; ++e) {
+                    acc[e].x += v[b][e].x;
+                    acc[e].y += v[b][e].y;
+                    acc[e].z += v[b][e].z;
+                    acc[e].w += v[b][e].w;
+                }
+        }
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) {
+            const int pos = threadIdx.x + e * C::kThreads;
+            if (pos >= kPos) break;
+            const int nn = pos % kTileN, m0 = mb * BM + (pos / kTileN) * 4;
+            const int64_t nrow = (int64_t)t * kTileN + nn;
+            if (nrow >= a.N) continue;
+            const float vals[4] = {acc[e].x, acc[e].y, acc[e].z, acc[e].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (m0 + q < a.M) a.Y[(int64_t)(m0 + q) * a.N + nrow] = __float2bfloat16_rn(vals[q]);
+        }
+    }
 }
 
 struct TcPlan {
-    int BM, tiles_m, Mp, KS, gps;
-    int64_t tiles_n;
-    size_t part_off, xp_off, ws_bytes, smem;
+    int BM, MB, T, G, P, maxc;
+    size_t part_off, ws_bytes;
 };
 
-TcPlan tc_plan(int64_t M, int64_t N, int64_t K) {
+int tc_sm_count() {
+    static std::atomic<int> cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    int n = cached[dev].load(std::memory_order_relaxed);
+    if (!n) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+TcPlan tc_plan(int64_t M, int64_t N, int64_t K, int sms) {
     TcPlan p{};
-    p.BM = M <= 16 ? 16 : 32;                 // more CTAs beat larger X tiles (measured)
-    p.tiles_m = (int)((M + p.BM - 1) / p.BM);
-    p.Mp = p.tiles_m * p.BM;
-    p.tiles_n = (N + kTileN - 1) / kTileN;
-    const int64_t G = K / kGroup;
-    int64_t ks = (2 * 148 + p.tiles_n * p.tiles_m - 1) / (p.tiles_n * p.tiles_m);
-    if (ks < 1) ks = 1;
-    if (ks > G) ks = G;
-    p.gps = (int)((G + ks - 1) / ks);
-    p.KS = (int)((G + p.gps - 1) / p.gps);
+    p.BM = M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    p.MB = (int)((M + p.BM - 1) / p.BM);
+    p.T = (int)((N + kTileN - 1) / kTileN);
+    p.G = (int)(K / kGroup);
+    const int64_t W = (int64_t)p.MB * p.T * p.G;
+    int64_t P = W / kMinItems;
+    if (P > sms) P = sms;
+    if (P < 1) P = 1;
+    p.P = (int)P;
+    // CTAs that can share one tile (its G items over ranges of >= floor(W/P))
+    int maxc = 1;
+    for (int64_t tu = 0; tu < (int64_t)p.MB * p.T; ++tu) {
+        const int c = cta_of(tu * p.G + p.G - 1, W, p.P) - cta_of(tu * p.G, W, p.P) + 1;
+        maxc = c > maxc ? c : maxc;
+    }
+    p.maxc = maxc;
     p.part_off = kTicketBytes;
-    const size_t part = p.KS > 1 ? (size_t)p.KS * M * N * sizeof(float) : 0;
-    p.xp_off = (p.part_off + part + 1023) & ~(size_t)1023;
-    p.ws_bytes = p.xp_off + (size_t)p.Mp * K * sizeof(uint16_t);
-    p.smem = 1024 + 2 * kTileN * 128 + 2 * (size_t)p.BM * 128;
+    const size_t part = (size_t)p.MB * p.T * p.maxc * p.BM * kTileN * sizeof(float);
+    p.ws_bytes = p.part_off + part;
     return p;
 }
 
-using TcFn = void (*)(const uint16_t *, const uint32_t *, const __half *, int, int64_t, int64_t,
-                      int, int, float *, unsigned *, __nv_bfloat16 *);
+// cuTensorMapEncodeTiled from the driver (looked up once, no -lcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static std::atomic<void *> cached{nullptr};
+    void *f = cached.load(std::memory_order_acquire);
+    if (!f) {
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        cached.store(f, std::memory_order_release);
+    }
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+}
+
+// Tensor map of X (M x K bf16, row stride K) seen as (64 columns, M rows,
+// K/64 halves): one box of 64 x BM x 2 is the BM x 128 block of one group,
+// two halves of BM rows of 128 bytes in the 128-byte swizzle, the layout of
+// the MMA's B operand; rows past M read as zeros.
+bool encode_x_map(CUtensorMap *map, const uint16_t *X, int64_t M, int64_t K, int BM) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {64, (cuuint64_t)M, (cuuint64_t)(K / 64)};
+    const cuuint64_t strides[2] = {(cuuint64_t)K * 2, 128};
+    const cuuint32_t box[3] = {64, (cuuint32_t)BM, 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(X), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+using TcFn = void (*)(GArgs);
 
 template <int R>
 TcFn tc_pick_bm(int BM) {
     switch (BM) {
-        case 16: return gemm_tc_kernel<R, 16>;
         case 32: return gemm_tc_kernel<R, 32>;
         case 64: return gemm_tc_kernel<R, 64>;
         default: return gemm_tc_kernel<R, 128>;
@@ -348,35 +555,58 @@ TcFn tc_pick(int r, int BM) {
     }
 }
 
+// cudaFuncSetAttribute once per (kernel, device), safe from any host thread.
+cudaError_t tc_smem_attr(TcFn fn, int r, int BM, size_t smem) {
+    static std::atomic<uint64_t> done[8][3];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const int bi = BM == 32 ? 0 : BM == 64 ? 1 : 2;
+    const uint64_t bit = 1ull << (dev & 63);
+    std::atomic<uint64_t> &d = done[r - 1][bi];
+    if (d.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(227 * 1024));
+    (void)smem;
+    if (e == cudaSuccess) d.fetch_or(bit, std::memory_order_acq_rel);
+    return e;
+}
+
 }  // namespace
 
 size_t gemm_tc_workspace_bytes(int64_t M, int64_t N, int64_t K, int r) {
     (void)r;
-    return tc_plan(M, N, K).ws_bytes;
+    return tc_plan(M, N, K, tc_sm_count()).ws_bytes;
 }
 
 mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
                          void *ws, size_t ws_bytes, cudaStream_t st) {
-    const TcPlan p = tc_plan(M, w->N, w->K);
-    if (p.ws_bytes > ws_bytes) return fail(MQ_ERR_WORKSPACE, "GEMM workspace too small");
-    if (p.tiles_n * p.tiles_m > (int64_t)(kTicketBytes / sizeof(unsigned)))
+    const TcPlan p = tc_plan(M, w->N, w->K, tc_sm_count());
+    if (!ws || p.ws_bytes > ws_bytes) return fail(MQ_ERR_WORKSPACE, "GEMM workspace too small");
+    if ((int64_t)p.MB * p.T > (int64_t)(kTicketBytes / sizeof(unsigned)))
         return fail(MQ_ERR_UNSUPPORTED, "too many output tiles for the ticket region");
-    char *wsb = static_cast<char *>(ws);
-    uint16_t *Xp = reinterpret_cast<uint16_t *>(wsb + p.xp_off);
-    const int64_t blocks = (int64_t)p.Mp * (w->K / 32);
-    int grid = (int)((blocks + 255) / 256);
-    if (grid > 148 * 16) grid = 148 * 16;
-    x_permute_kernel<<<grid, 256, 0, st>>>(X, (int)M, p.Mp, w->K, Xp);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "x_permute_kernel");
     TcFn fn = tc_pick(w->r, p.BM);
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
+    const int threads = p.BM == 128 ? TcCfg<1, 128>::kThreads : TcCfg<1, 32>::kThreads;
+    const size_t smem = tc_smem_bytes(w->r, p.BM);
+    cudaError_t e = tc_smem_attr(fn, w->r, p.BM, smem);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-    dim3 g3((unsigned)p.tiles_n, (unsigned)p.tiles_m, (unsigned)p.KS);
-    fn<<<g3, kTcThreads, p.smem, st>>>(
-        Xp, w->planes, reinterpret_cast<const __half *>(w->scales), (int)M, w->N, w->K,
-        p.gps, p.KS, reinterpret_cast<float *>(wsb + p.part_off),
-        reinterpret_cast<unsigned *>(wsb), reinterpret_cast<__nv_bfloat16 *>(Y));
+    char *wsb = static_cast<char *>(ws);
+    GArgs a{};
+    if (!encode_x_map(&a.xmap, X, M, w->K, p.BM)) return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled (X)");
+    a.planes = w->planes;
+    a.scales = reinterpret_cast<const __half *>(w->scales);
+    a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
+    a.part = reinterpret_cast<float *>(wsb + p.part_off);
+    a.tickets = reinterpret_cast<unsigned *>(wsb);
+    a.N = w->N;
+    a.K = w->K;
+    a.M = (int)M;
+    a.T = p.T;
+    a.G = p.G;
+    a.MB = p.MB;
+    a.P = p.P;
+    a.maxc = p.maxc;
+    a.plane_words = (int64_t)p.T * kTileN * (w->K / 32);
+    fn<<<p.P, threads, smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_fail(e, "gemm_tc_kernel");
     return MQ_OK;

@@ -146,15 +146,6 @@ __device__ __forceinline__ bool bar_try_cluster(uint64_t *b, uint32_t parity) {
                  : "=r"(ok) : "r"(smem_u32(b)), "r"(parity) : "memory");
     return ok != 0;
 }
-// Named barrier that also returns the AND of `v` over its threads, so that a
-// whole team takes the same branch after a wait that may have timed out.
-__device__ __forceinline__ bool named_sync_and(int id, int n, bool v) {
-    uint32_t r;
-    asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 q, %2, 0;\n"
-                 " bar.red.and.pred p, %1, %3, q;\n selp.u32 %0, 1, 0, p;\n}"
-                 : "=r"(r) : "r"(id), "r"((uint32_t)v), "r"(n) : "memory");
-    return r != 0;
-}
 
 // ------------------------------------------------------------ decomposition
 // Items u = 0 .. W-1, W = T * KC (T 128-row tiles, KC = K / 128 groups), in

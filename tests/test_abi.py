@@ -99,3 +99,20 @@ def test_pack_unpack_argument_errors():
     assert L.mq_unpack(ctypes.byref(w), FAKE + 3, None) == 3
     assert L.mq_unpack(None, FAKE, None) == 1
     assert b"16-byte" in L.mq_last_error_string() or L.mq_last_error() == 1
+
+
+def test_gemm_kernel_query():
+    # which kernel serves a shape (host only): invalid problems give 0,
+    # M >= 9 always the GEMM, the MQ_GEMV_VIA_GEMM variant the GEMM for M <= 8
+    assert mq.mq_gemm_kernel(0, 64, 128, 4) == 0
+    assert mq.mq_gemm_kernel(1, 64, 100, 4) == 0
+    assert mq.mq_gemm_kernel(1, 64, 128, 9) == 0
+    for M in (9, 16, 64, 300):
+        assert mq.mq_gemm_kernel(M, 4096, 4096, 4) == mq.KERNEL_GEMM
+    old = mq.mq_get_gemv_variant()
+    mq.mq_set_gemv_variant(mq.GEMV_VIA_GEMM)
+    try:
+        for M in range(1, 9):
+            assert mq.mq_gemm_kernel(M, 4096, 4096, 4) == mq.KERNEL_GEMM
+    finally:
+        mq.mq_set_gemv_variant(old)

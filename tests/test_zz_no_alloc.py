@@ -87,12 +87,13 @@ def test_noalloc_rejects_oversized_and_large_m():
     Y = torch.zeros((9, N), dtype=torch.bfloat16, device="cuda")
     assert fn(X.data_ptr(), ctypes.byref(w), 9, N, K, Y.data_ptr(), None) == 1
     # a scratch need above 16 MiB is refused before any launch: on the GEMM
-    # route (M = 1, N = 128, K = 2^20) the GEMM's scratch alone exceeds it
+    # route (M = 1, N = 2^17, K = 4096) the partial sums of the row tiles
+    # shared between CTAs alone exceed it
     old = mq.mq_get_gemv_variant()
     mq.mq_set_gemv_variant(mq.GEMV_VIA_GEMM)
     try:
-        big = mq.MqWeights(w.planes, w.scales, 128, 1 << 20, 128, 2)
-        assert mq.mq_gemm_workspace_bytes(1, 128, 1 << 20, 2) > (16 << 20)
-        assert fn(X.data_ptr(), ctypes.byref(big), 1, 128, 1 << 20, Y.data_ptr(), None) == 6
+        big = mq.MqWeights(w.planes, w.scales, 1 << 17, 4096, 128, 2)
+        assert mq.mq_gemm_workspace_bytes(1, 1 << 17, 4096, 2) > (16 << 20)
+        assert fn(X.data_ptr(), ctypes.byref(big), 1, 1 << 17, 4096, Y.data_ptr(), None) == 6
     finally:
         mq.mq_set_gemv_variant(old)
