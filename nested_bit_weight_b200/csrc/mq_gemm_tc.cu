@@ -24,11 +24,11 @@
 //                   order and stores them to its TMEM lane in one of two A
 //                   stages (tcgen05.st; the MMA reads A from TMEM);
 //   X warp          one thread loads the group's BM x 128 block of X into one
-//                   of 3 or 4 B stages with one tensor-map (TMA) copy, in the
+//                   of 2 or 4 B stages with one tensor-map (TMA) copy, in the
 //                   same layout; rows beyond M read as zeros;
 //   MMA warp        one thread issues eight 128 x BM x 16 MMAs per group into
-//                   one of two TMEM accumulators and commits to the A stage,
-//                   B stage (free) and accumulator (full) barriers;
+//                   the stage's TMEM accumulator and commits once: the
+//                   stage's A and B operands are free, its accumulator full;
 //   fold warps      4 (BM <= 64) or 8 (BM = 128), one or two per TMEM lane
 //                   quarter: y += s[n, g] * D_g, the tile's fp32 sums kept in
 //                   registers until the tile ends.
@@ -40,6 +40,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <type_traits>
 
 #include "mq_common.cuh"
 #include "mq_bits.cuh"
@@ -53,34 +54,45 @@ using namespace sm100;
 constexpr int kTileN = 128;                  // weight rows per tile (MMA M)
 constexpr int kMinItems = 4;                 // fewest items a CTA is given
 
-// Per (r, BM) configuration.  14 warps, so 128 registers a thread: decode
-// warps (two threads per row, or one for BM = 128), fold warps, then the X
-// and MMA warps.  Shared memory: kNX X stages and a ring of kD items of plane
-// words (the loads in flight that keep HBM busy).  Tensor memory: two A
-// stages (64 columns each) and two accumulators (BM columns each).
+// Per (r, BM) configuration.  15 warps, so 128 registers a thread: decode
+// warps (two groups of four taking alternate items, or one group for
+// BM = 128), fold warps, the X warp and two MMA warps.  Shared memory: kS X stages and a ring of kD items of plane
+// words (the loads in flight that keep HBM busy).  Tensor memory (512
+// columns): kS A stages of 64 columns and kS accumulators of BM columns, with
+// kS = 4 for BM <= 64 (the decode, the MMA and the fold run up to three
+// groups apart) and 2 for BM = 128.  Item i uses stage i % kS of all three,
+// so one commit per item frees its A and X stages and fills its accumulator.
 __host__ __device__ constexpr int ring_items(int r, int BM) {
     return (96 * 1024) / (r * 2048) < 16 ? (96 * 1024) / (r * 2048) : 16;
 }
-__host__ __device__ constexpr int x_stages(int BM) { return BM == 128 ? 3 : 4; }
+// Pipeline stages: item i uses A stage, X stage and accumulator i % stages.
+__host__ __device__ constexpr int x_stages(int BM) { return BM == 128 ? 2 : 4; }
+constexpr int kScaleAhead = 8;                // items of scales in flight per fold thread
 __host__ __device__ constexpr size_t tc_smem_bytes(int r, int BM) {
-    return 1024 + (size_t)x_stages(BM) * BM * 256 + (size_t)ring_items(r, BM) * r * 2048 + 256;
+    return 1024 + (size_t)x_stages(BM) * BM * 256 + (size_t)ring_items(r, BM) * r * 2048 +
+           (size_t)256 * kScaleAhead * 4 + 512;
 }
 
 template <int R, int BM>
 struct TcCfg {
     static constexpr int kDecW = BM == 128 ? 4 : 8;
     static constexpr int kFoldW = BM == 128 ? 8 : 4;
-    static constexpr int kThreads = (kDecW + kFoldW + 2) * 32;
-    static constexpr int kParts = kDecW / 4;                  // decode threads per row
-    static constexpr int kWP = 4 / kParts;                    // plane words per decode thread
-    static constexpr int kNX = x_stages(BM);
-    static constexpr int kD = ring_items(R, BM);
+    static constexpr int kThreads = (kDecW + kFoldW + 3) * 32;  // + X warp + 2 MMA warps
+    static constexpr int kGroups = kDecW / 4;                 // decode groups (alternate items)
+    static constexpr int kS = x_stages(BM);
+    static constexpr int kD = ring_items(R, BM) / kGroups;    // ring items per decode group
     static constexpr uint32_t kXStage = BM * 256;             // BM rows x 128 bf16
-    static constexpr uint32_t kTmemCols = 128 + 2 * BM <= 256 ? 256 : 512;
+    static constexpr uint32_t kTmemCols = 512;
+    static_assert(kS * 64 + kS * BM <= (int)kTmemCols, "TMEM columns");
     static constexpr uint32_t kSlot = R * 2048;               // plane words of one item
 };
 
 __device__ unsigned int g_tc_timeout;        // set when a bounded wait gave up
+
+// Wait of the decode and fold warps for their hand-offs.
+#ifndef MQ_GEMM_WAIT
+#define MQ_GEMM_WAIT mbar_wait_abortable
+#endif
 
 // The 16 A words of one 32-column plane word, before centring: word 4b + j
 // holds columns 8b + 2j and 8b + 2j + 1 (low, high half), as bf16 256 + e
@@ -152,22 +164,25 @@ template <int R, int BM>
 __global__ void __launch_bounds__(TcCfg<R, BM>::kThreads, 1)
 gemm_tc_kernel(const __grid_constant__ GArgs a) {
     using C = TcCfg<R, BM>;
-    constexpr int kDecW = C::kDecW, kFoldW = C::kFoldW, kNX = C::kNX, kD = C::kD, kWP = C::kWP;
+    constexpr int kDecW = C::kDecW, kFoldW = C::kFoldW, kS = C::kS, kD = C::kD;
     constexpr int kFoldW0 = kDecW, kXW = kDecW + kFoldW, kMmaW = kXW + 1;
     constexpr uint32_t kIdesc = idesc_bf16_f32(kTileN, BM);
-    constexpr uint32_t kD0 = 128;                              // TMEM: A stages [0, 128), accumulators after
+    constexpr uint32_t kD0 = kS * 64;                          // TMEM: A stages, then the accumulators
     constexpr int kCW = BM * 4 / kFoldW;                       // columns per fold thread
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *sX = smem;                                        // [kNX][2 halves][BM][128 B]
-    uint8_t *ring = sX + kNX * C::kXStage;                     // [kD][plane][part][128][kWP words]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + kD * C::kSlot);
-    uint64_t *afull = bars, *aempty = bars + 2, *dfull = bars + 4, *dempty = bars + 6;
-    uint64_t *xfull = bars + 8, *xempty = xfull + kNX;
-    // [0] abort  [2] items issued to the MMA  [3] X items loaded
-    // [4] tiles this CTA sums at the end  [5, 6] their indices  [7, 8] their CTA counts
-    volatile int *flags = reinterpret_cast<volatile int *>(xempty + kNX);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(xempty + kNX) + 10;
+    uint8_t *sX = smem;                                        // [kS][2 halves][BM][128 B]
+    uint8_t *ring = sX + kS * C::kXStage;                      // [group][kD][plane][128 rows][16 B]
+    uint32_t *sring = reinterpret_cast<uint32_t *>(ring + C::kGroups * kD * C::kSlot);  // [fold thread][kScaleAhead]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sring + kFoldW * 32 * kScaleAhead);
+    // afull: A stage decoded; xfull: X stage loaded; sempty: the stage's MMAs
+    // done (A and X free, accumulator full); dempty: accumulator read
+    uint64_t *afull = bars, *xfull = afull + kS, *sempty = xfull + kS, *dempty = sempty + kS;
+    // [0] abort  [2], [9] last item + 1 issued by the even / odd MMA thread
+    // [3] X items loaded  [4] tiles this CTA sums at the end  [5, 6] their
+    // indices  [7, 8] their CTA counts
+    volatile int *flags = reinterpret_cast<volatile int *>(dempty + kS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dempty + kS) + 12;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t W = (int64_t)a.MB * a.T * a.G;
@@ -176,17 +191,13 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
     const int G = a.G, TG = a.T * a.G;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(afull + i, kDecW);
-            mbar_init(aempty + i, 1);
-            mbar_init(dfull + i, 1);
+        for (int i = 0; i < kS; ++i) {
+            mbar_init(afull + i, 4);                           // the 4 warps of one decode group
+            mbar_init(xfull + i, 1);
+            mbar_init(sempty + i, 1);
             mbar_init(dempty + i, kFoldW);
         }
-        for (int i = 0; i < kNX; ++i) {
-            mbar_init(xfull + i, 1);
-            mbar_init(xempty + i, 1);
-        }
-        for (int i = 0; i < 9; ++i) flags[i] = 0;      // [1] unused
+        for (int i = 0; i < 10; ++i) flags[i] = 0;     // [1] unused
         fence_mbar_init();
     }
     if (warp == kMmaW) {
@@ -200,57 +211,56 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
 
     if (warp < kDecW) {
         // ------------------------------------------------------------ decode
+        // group g (warps 4g .. 4g + 3) takes items g, g + kGroups, ...; thread
+        // n of the group owns row n of the tile and copies exactly what it
+        // decodes: 16 bytes (32 columns x 4 words) of each plane per item,
+        // with L1-bypassing cp.async into the group's ring of kD items
+        constexpr int kGroups = C::kGroups;
         const int n = threadIdx.x & (kTileN - 1);              // row of the tile
-        const int hp = threadIdx.x >> 7;                       // part of the row
-        const int w0 = hp * kWP;                               // first word (32 columns) of the part
-        uint8_t *mine = ring + ((size_t)hp * kTileN + n) * (kWP * 4);   // + slot, + plane
-        constexpr uint32_t kPlaneStride = C::kParts * kTileN * kWP * 4; // 2 KB
-        // the plane words of item j (this thread's part) into ring slot j % kD
-        auto issue = [&](int j) {
-            const uint32_t *src = a.planes + ((u0 + j) % TG) * 512 + n * 4 + w0;
+        const int g = threadIdx.x >> 7;                        // item group
+        uint8_t *mine = ring + (size_t)g * kD * C::kSlot + n * 16;   // + slot, + plane
+        int next_tg = (int)((u0 + g) % TG);                    // (tile, group) of the next item copied
+        auto issue = [&](int j) {                              // the group's j-th item, in order
+            const uint32_t *src = a.planes + (int64_t)next_tg * 512 + n * 4;
             uint8_t *dst = mine + (j % kD) * C::kSlot;
 #pragma unroll
-            for (int p = 0; p < R; ++p) {
-                if constexpr (kWP == 4) cp_async_16(dst + p * kPlaneStride, src + p * a.plane_words);
-                else cp_async_8(dst + p * kPlaneStride, src + p * a.plane_words);
-            }
+            for (int p = 0; p < R; ++p) cp_async_16(dst + p * 2048, src + p * a.plane_words);
+            next_tg += kGroups;
+            while (next_tg >= TG) next_tg -= TG;               // TG may be 1
         };
+        const int Lg = L > g ? (L - g + kGroups - 1) / kGroups : 0;   // items of this group
 #pragma unroll 1
         for (int j = 0; j < kD; ++j) {
-            if (j < L) issue(j);
+            if (j < Lg) issue(j);
             cp_async_commit();
         }
-        for (int i = 0; i < L; ++i) {
-            const int st = i & 1;
+        for (int j = 0; j < Lg; ++j) {
+            const int i = g + j * kGroups;                     // item of the range
+            const int st = i % kS;
             cp_async_wait<kD - 1>();                           // item i's words are in
-            uint32_t pv[R][kWP];
-            const uint8_t *src = mine + (i % kD) * C::kSlot;
+            uint32_t pv[R][4];
+            const uint8_t *src = mine + (j % kD) * C::kSlot;
 #pragma unroll
             for (int p = 0; p < R; ++p) {
-                if constexpr (kWP == 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(src + p * kPlaneStride);
-                    pv[p][0] = v.x; pv[p][1] = v.y; pv[p][2] = v.z; pv[p][3] = v.w;
-                } else {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(src + p * kPlaneStride);
-                    pv[p][0] = v.x; pv[p][1] = v.y;
-                }
+                const uint4 v = *reinterpret_cast<const uint4 *>(src + p * 2048);
+                pv[p][0] = v.x; pv[p][1] = v.y; pv[p][2] = v.z; pv[p][3] = v.w;
             }
-            if (i + kD < L) issue(i + kD);                     // refill the slot just read
+            if (j + kD < Lg) issue(j + kD);                    // refill the slot just read
             cp_async_commit();
-            bool ok = i < 2 || mbar_wait_backoff(aempty + st, (uint32_t)((i >> 1) - 1) & 1u, flags);
+            bool ok = i < kS || MQ_GEMM_WAIT(sempty + st, (uint32_t)(i / kS - 1) & 1u, flags);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
             tc_fence_after();
-            // this row's 32-column words -> 16 TMEM columns each of A stage st
+            // the row's four 32-column words -> 16 TMEM columns each of A stage st
             const uint32_t a_row = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(st * 64);
 #pragma unroll
-            for (int w = 0; w < kWP; ++w) {
+            for (int w = 0; w < 4; ++w) {
                 uint32_t P[8], v[16];
 #pragma unroll
                 for (int p = 0; p < 8; ++p) P[p] = p < R ? pv[p < R ? p : 0][w] : 0u;
                 word_pairs<R>(P, v);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) v[j] = centre<R>(v[j]);
-                tmem_st16(a_row + (uint32_t)(16 * (w0 + w)), v);
+                for (int q = 0; q < 16; ++q) v[q] = centre<R>(v[q]);
+                tmem_st16(a_row + (uint32_t)(16 * w), v);
             }
             tmem_st_wait();
             tc_fence_before();
@@ -266,127 +276,163 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
         float y[kCW];
 #pragma unroll
         for (int j = 0; j < kCW; ++j) y[j] = 0.f;
+        // ok turns false for good once a wait of this warp gave up: the warp
+        // then skips its waits and tensor-memory reads but still runs every
+        // tile end, so the barriers below always match and every ticket is
+        // taken (Y is then unspecified)
         bool ok = true;
-        int64_t tile_u0 = u0 - (u0 % G);                       // first item of the current tile
-        float sn = L > 0 ? __half2float(a.scales[(u0 % TG) * 128 + n]) : 0.f;
+        int gi = (int)(u0 % G);                                // group of item i inside its tile
+        int64_t tu = u0 / G;                                   // tile of item i over (mb, t)
+        int64_t tile_u0 = u0 - gi;                             // first item of that tile
+        // the fp16 scales of the next kScaleAhead items in flight: each thread
+        // copies the 4 bytes holding its row's scale (rows n & ~1 and n | 1)
+        // into its own slots (cp.async groups are per thread: no barrier)
+        uint32_t *slots = sring + (threadIdx.x - kFoldW0 * 32) * kScaleAhead;
+        const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales) + (n & ~1);
+        int next_tg = (int)(u0 % TG);                          // (tile, group) of the next scale copied
+        auto scale_issue = [&](int i) {
+            cp_async_4(slots + i % kScaleAhead, sc + (int64_t)next_tg * 128);
+            if (++next_tg == TG) next_tg = 0;
+        };
+#pragma unroll 1
+        for (int k = 0; k < kScaleAhead; ++k) {
+            if (k < L) scale_issue(k);
+            cp_async_commit();
+        }
         for (int i = 0; i < L; ++i) {
-            const int64_t u = u0 + i;
-            const int db = i & 1;
-            const float s = sn;
-            if (i + 1 < L) sn = __half2float(a.scales[((u + 1) % TG) * 128 + n]);
-            ok = mbar_wait_backoff(dfull + db, (uint32_t)(i >> 1) & 1u, flags);
-            // every fold thread takes the same branch (the tile end below
-            // has barriers of its own)
-            ok = named_sync_and(3, kFoldW * 32, ok);
-            if (!ok) break;
-            tc_fence_after();
+            const int db = i % kS;
+            cp_async_wait<kScaleAhead - 1>();                  // item i's scale is in
+            const uint32_t sw = slots[i % kScaleAhead];
+            const float s = __half2float(__ushort_as_half((unsigned short)((n & 1) ? sw >> 16 : sw & 0xFFFFu)));
+            if (i + kScaleAhead < L) scale_issue(i + kScaleAhead);
+            cp_async_commit();
+            if (ok) ok = MQ_GEMM_WAIT(sempty + db, (uint32_t)(i / kS) & 1u, flags);
+            ok = __all_sync(0xFFFFFFFFu, ok);                  // tcgen05.ld is warp-wide
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-            for (int cb = 0; cb < kCW; cb += 16) {
-                uint32_t v[16];
-                tmem_ld16(tmem + lane_base + kD0 + (uint32_t)(db * BM + c0 + cb), v);
-                tmem_ld_wait();
+                for (int cb = 0; cb < kCW; cb += 16) {
+                    uint32_t v[16];
+                    tmem_ld16(tmem + lane_base + kD0 + (uint32_t)(db * BM + c0 + cb), v);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) y[cb + j] = fmaf(s, __uint_as_float(v[j]), y[cb + j]);
+                    for (int j = 0; j < 16; ++j) y[cb + j] = fmaf(s, __uint_as_float(v[j]), y[cb + j]);
+                }
+                tc_fence_before();
             }
-            tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(dempty + db);
             // the tile ends with this item (or the range does): write it out
-            const bool tile_end = (u + 1) % G == 0 || i == L - 1;
-            if (!tile_end) continue;
-            const int64_t tu = u / G;                          // tile index over (mb, t)
-            const int mb = (int)(tu / a.T), t = (int)(tu % a.T);
-            const int64_t tn0 = tile_u0, tn1 = tile_u0 + G;    // the tile's items
-            const int64_t nrow = (int64_t)t * kTileN + n;
-            const int mlim = a.M - (mb * BM + c0);             // columns of this thread inside M
-            const bool own = tn0 >= u0 && tn1 <= u1;           // the whole tile is in this range
-            int cf = 0, cnt = 1;
-            if (!own) {
-                cf = cta_of(tn0, W, a.P);
-                cnt = cta_of(tn1 - 1, W, a.P) - cf + 1;
-            }
-            // own tile: Y directly; shared tile: this CTA's fp32 partial sums,
-            // as float4 (4 columns of one row) at [column / 4][row]
-            float4 *pp = reinterpret_cast<float4 *>(a.part + ((size_t)tu * a.maxc + (own ? 0 : blockIdx.x - cf)) * (BM * kTileN)) +
-                         (c0 / 4) * kTileN + n;
-            __nv_bfloat16 *yp = a.Y + (int64_t)(mb * BM + c0) * a.N + nrow;
-            if (own ? nrow < a.N : true) {
+            const bool tile_end = gi == G - 1 || i == L - 1;
+            if (tile_end) {
+                const int mb = (int)(tu / a.T), t = (int)(tu % a.T);
+                const int64_t tn0 = tile_u0, tn1 = tile_u0 + G;    // the tile's items
+                const int64_t nrow = (int64_t)t * kTileN + n;
+                const int mlim = a.M - (mb * BM + c0);             // columns of this thread inside M
+                const bool own = tn0 >= u0 && tn1 <= u1;           // the whole tile is in this range
+                int cf = 0, cnt = 1;
+                if (!own) {
+                    cf = cta_of(tn0, W, a.P);
+                    cnt = cta_of(tn1 - 1, W, a.P) - cf + 1;
+                }
+                // own tile: Y directly; shared tile: this CTA's fp32 partial
+                // sums, as float4 (4 columns of one row) at [column / 4][row]
+                float4 *pp = reinterpret_cast<float4 *>(a.part + ((size_t)tu * a.maxc + (own ? 0 : blockIdx.x - cf)) *
+                                                                     (BM * kTileN)) + (c0 / 4) * kTileN + n;
+                __nv_bfloat16 *yp = a.Y + (int64_t)(mb * BM + c0) * a.N + nrow;
+                if (own ? nrow < a.N : true) {
 #pragma unroll
-                for (int j = 0; j < kCW; j += 4) {
-                    if (!own) {
-                        pp[(j / 4) * kTileN] = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-                    } else {
+                    for (int j = 0; j < kCW; j += 4) {
+                        if (!own) {
+                            pp[(j / 4) * kTileN] = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+                        } else {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            if (j + q < mlim) yp[(int64_t)(j + q) * a.N] = __float2bfloat16_rn(y[j + q]);
+                            for (int q = 0; q < 4; ++q)
+                                if (j + q < mlim) yp[(int64_t)(j + q) * a.N] = __float2bfloat16_rn(y[j + q]);
+                        }
                     }
                 }
-            }
-            if (!own) {
-                // take a ticket; the last CTA to arrive sums the tile after
-                // its own range (all threads of the CTA, in CTA order)
-                __threadfence();
-                named_sync(3, kFoldW * 32);
-                if (f == 0 && lane == 0) {
-                    if (atomicAdd(a.tickets + tu, 1u) == (unsigned)(cnt - 1)) {
-                        a.tickets[tu] = 0u;                    // every part is in: reset for the next launch
-                        const int k = flags[4];
-                        flags[5 + k] = (int)tu;
-                        flags[7 + k] = cnt;
-                        flags[4] = k + 1;
+                if (!own) {
+                    // take a ticket (one thread, after the fold warps' partial
+                    // sums: the fence is cumulative over the barrier); the last
+                    // CTA to arrive sums the tile after its own range (all
+                    // threads of the CTA, in CTA order)
+                    named_sync(3, kFoldW * 32);
+                    if (f == 0 && lane == 0) {
+                        __threadfence();
+                        if (atomicAdd(a.tickets + tu, 1u) == (unsigned)(cnt - 1)) {
+                            a.tickets[tu] = 0u;                // every part is in: reset for the next launch
+                            const int k = flags[4];
+                            flags[5 + k] = (int)tu;
+                            flags[7 + k] = cnt;
+                            flags[4] = k + 1;
+                        }
                     }
                 }
-            }
 #pragma unroll
-            for (int j = 0; j < kCW; ++j) y[j] = 0.f;
-            tile_u0 += G;
-        }
-        if (!ok && f == 0 && lane == 0) {
-            // a wait gave up: still take the tickets of the shared tiles left
-            // in the range so that they return to zero (Y is then unspecified)
-            for (int64_t tn0 = tile_u0; tn0 < u1; tn0 += G) {
-                const int64_t tn1 = tn0 + G;
-                if (tn0 >= u0 && tn1 <= u1) continue;
-                const int cnt = cta_of(tn1 - 1, W, a.P) - cta_of(tn0, W, a.P) + 1;
-                const int64_t tu = tn0 / G;
-                if (atomicAdd(a.tickets + tu, 1u) == (unsigned)(cnt - 1)) a.tickets[tu] = 0u;
+                for (int j = 0; j < kCW; ++j) y[j] = 0.f;
+                tile_u0 += G;
+            }
+            if (++gi == G) {
+                gi = 0;
+                ++tu;
             }
         }
+        cp_async_wait<0>();                                    // no scale copy left in flight
     } else if (warp == kXW) {
         // ----------------------------------------------------------------- X
         if (lane == 0) {
+            int mb = (int)(u0 / TG), g = (int)(u0 % G);        // X block and group of item i
             for (int i = 0; i < L; ++i) {
-                const int xs = i % kNX, kx = i / kNX;
-                const int64_t u = u0 + i;
-                const int mb = (int)(u / TG), g = (int)(u % G);
-                if (kx > 0 && !mbar_wait_abortable(xempty + xs, (uint32_t)(kx - 1) & 1u, flags)) break;
+                const int xs = i % kS, kx = i / kS;
+                if (kx > 0 && !mbar_wait_abortable(sempty + xs, (uint32_t)(kx - 1) & 1u, flags)) break;
                 mbar_expect_tx(xfull + xs, C::kXStage);
                 tma_load_3d(sX + xs * C::kXStage, &a.xmap, 0, mb * BM, 2 * g, xfull + xs);
                 flags[3] = i + 1;
+                if (++g == G) {
+                    g = 0;
+                    if ((int64_t)(i + 1 + u0) % TG == 0) ++mb;   // rare: once per pass over the tiles
+                }
             }
         }
     } else {
         // --------------------------------------------------------------- MMA
+        // two issuing threads (lane 0 of each MMA warp): parity p takes the
+        // items p, p + 2, ..., so one thread's barrier waits overlap the
+        // other's MMAs; within a round of kS items the stage of each item is
+        // a constant, and every operand a constant offset from one base
         if (lane == 0) {
-            const uint32_t x0 = smem_u32(sX);
-            for (int i = 0; i < L; ++i) {
-                const int st = i & 1, db = i & 1, xs = i % kNX;
-                if (!mbar_wait_abortable(afull + st, (uint32_t)(i >> 1) & 1u, flags)) break;
-                if (!mbar_wait_abortable(xfull + xs, (uint32_t)(i / kNX) & 1u, flags)) break;
-                if (i >= 2 && !mbar_wait_abortable(dempty + db, (uint32_t)((i >> 1) - 1) & 1u, flags)) break;
-                tc_fence_after();
+            const uint64_t bdesc0 = smem_desc_sw128(smem_u32(sX));
+            auto run = [&](auto P) {
+                constexpr int p = decltype(P)::value;
+                for (int q = 0;; ++q) {                        // round q: items q * kS + s
+                    bool more = true;
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const int h = ks >> 2, kk = ks & 3;
-                    const uint64_t bd = smem_desc_sw128(x0 + xs * C::kXStage + h * (BM * 128) + kk * 32);
-                    mma_bf16_ts(tmem + kD0 + (uint32_t)(db * BM), tmem + (uint32_t)(st * 64 + 8 * ks), bd, kIdesc,
-                                ks > 0 ? 1u : 0u);
+                    for (int e = 0; e < kS / 2; ++e) {
+                        const int st = p + 2 * e, i = q * kS + st;
+                        if (i >= L) { more = false; break; }
+                        if (!mbar_wait_abortable(afull + st, (uint32_t)q & 1u, flags) ||
+                            !mbar_wait_abortable(xfull + st, (uint32_t)q & 1u, flags) ||
+                            (q > 0 && !mbar_wait_abortable(dempty + st, (uint32_t)(q - 1) & 1u, flags))) {
+                            more = false;
+                            break;
+                        }
+                        tc_fence_after();
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const int h = ks >> 2, kk = ks & 3;
+                            const uint64_t bd = bdesc0 + (uint64_t)((st * C::kXStage + h * (BM * 128) + kk * 32) >> 4);
+                            mma_bf16_ts(tmem + kD0 + (uint32_t)(st * BM), tmem + (uint32_t)(st * 64 + 8 * ks), bd,
+                                        kIdesc, ks > 0 ? 1u : 0u);
+                        }
+                        mma_commit(sempty + st);               // A, X free; accumulator full
+                        flags[p ? 9 : 2] = i + 1;              // last item issued by this thread, + 1
+                    }
+                    if (!more) break;
                 }
-                mma_commit(aempty + st);                       // A stage free
-                mma_commit(xempty + xs);                       // X stage free
-                mma_commit(dfull + db);                        // accumulator full
-                flags[2] = i + 1;
-            }
+            };
+            if (warp == kMmaW) run(std::integral_constant<int, 0>{});
+            else run(std::integral_constant<int, 1>{});
         }
     }
 
@@ -396,11 +442,13 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
     tc_fence_before();
     __syncthreads();
     if (threadIdx.x == 0) {
-        const int issued = flags[2], loaded = flags[3];
-        drain_ring(aempty, 2, issued);
-        drain_ring(xempty, kNX, issued);
-        drain_ring(dfull, 2, issued);
-        drain_ring(xfull, kNX, loaded);
+        // stage s is committed by the thread of parity s % 2, for its items
+        // s, s + kS, ... below its last item issued
+        for (int st = 0; st < kS; ++st) {
+            const int last = flags[(st & 1) ? 9 : 2];
+            if (last > st) mbar_wait_bounded(sempty + st, (uint32_t)((last - 1 - st) / kS) & 1u);
+        }
+        drain_ring(xfull, kS, flags[3]);
         if (flags[0]) atomicOr(&g_tc_timeout, 1u);
     }
     tc_fence_before();

@@ -274,9 +274,12 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *map, int x, i
         ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)) : "memory");
 }
 
-// Per-thread asynchronous copies global -> shared (8 or 16 bytes, both
+// Per-thread asynchronous copies global -> shared (4, 8 or 16 bytes, both
 // addresses aligned to the size), grouped per thread: commit closes a group,
 // wait<N> returns once at most N of this thread's newest groups are pending.
+__device__ __forceinline__ void cp_async_4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
 __device__ __forceinline__ void cp_async_8(void *dst, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
