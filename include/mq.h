@@ -124,8 +124,11 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
 
 /*
  * Y = X . W_r^T (MatGPTQ abstract: kernels for the nested format that serve
- * batch sizes beyond one).  M <= 8 runs the tcgen05 GEMV (decoded weights in
- * tensor memory; see mq_set_gemv_variant); M >= 9 runs the tcgen05 GEMM.
+ * batch sizes beyond one).  Small batches run the tcgen05 GEMV (decoded
+ * weights in tensor memory; see mq_set_gemv_variant): M <= 3 on every shape,
+ * M = 4 when N * K < 2^25, M = 5..6 when N * K <= 2^23, where it is measured
+ * faster; every other call runs the tcgen05 GEMM (mq_gemm_kernel tells
+ * which).
  *   X_dev      bf16 M x K row-major
  *   w          r-bit view (from mq_slice, or a parent with r = 8)
  *   Y_dev      bf16 M x N row-major (written, not accumulated)
@@ -140,7 +143,7 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * overlap the inputs.  M == 0 is accepted and does nothing.
  * The fp32 accumulation order is fixed, so results are deterministic.
  *
- * Stream order.  The M <= 8 kernel (MQ_GEMV_TC) is launched with programmatic
+ * Stream order.  The GEMV (MQ_KERNEL_GEMV) is launched with programmatic
  * dependent launch: it may start while the preceding kernel on the stream is
  * still running, and it begins streaming the weights (planes and scales)
  * before it waits for that kernel; X is read, and Y and the workspace are

@@ -26,11 +26,11 @@ def _headers_mtime() -> float:
     return max([os.path.getmtime(h) for h in hs] + [0.0])
 
 
-def _compile(src: str, hdr_mtime: float, verbose: bool) -> str:
-    obj = os.path.join(OBJ, os.path.basename(src) + ".o")
+def _compile(src: str, hdr_mtime: float, verbose: bool, obj_dir: str = OBJ, extra=()) -> str:
+    obj = os.path.join(obj_dir, os.path.basename(src) + ".o")
     if os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_mtime):
         return obj
-    cmd = [NVCC, *ARCH, *FLAGS, "-c", src, "-o", obj + ".tmp"]
+    cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj + ".tmp"]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)
@@ -38,19 +38,36 @@ def _compile(src: str, hdr_mtime: float, verbose: bool) -> str:
     return obj
 
 
-def build(verbose: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def _build_lib(lib: str, obj_dir: str, extra: list, verbose: bool) -> str:
+    os.makedirs(obj_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hm = _headers_mtime()
     with cf.ThreadPoolExecutor(max_workers=len(srcs)) as ex:
-        objs = list(ex.map(lambda s: _compile(s, hm, verbose), srcs))
-    if not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        tmp = LIB + ".tmp%d" % os.getpid()
+        objs = list(ex.map(lambda s: _compile(s, hm, verbose, obj_dir, extra), srcs))
+    if not os.path.exists(lib) or os.path.getmtime(lib) < max(os.path.getmtime(o) for o in objs):
+        tmp = lib + ".tmp%d" % os.getpid()
         subprocess.check_call([NVCC, *ARCH, "-shared", "--cudart", "static", "-Xlinker",
                                "--exclude-libs,ALL", "-o", tmp, *objs])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
+
+
+def build(verbose: bool = False) -> str:
+    return _build_lib(LIB, OBJ, [], verbose)
+
+
+# Test-hook build (tests only, never loaded by the package): every bounded
+# wait gives up after 5 ms instead of about a second, and
+# mq_test_drop_x_arrivals() makes a GEMM CTA drop one arrival, so a test can
+# run the timeout path on a GPU without a fault or a trap.
+HOOKS_LIB = os.path.join(HERE, "libmq_testhooks.so")
+HOOKS_OBJ = os.path.join(HERE, "_build_hooks")
+
+
+def build_test_hooks(verbose: bool = False) -> str:
+    return _build_lib(HOOKS_LIB, HOOKS_OBJ, ["-DMQ_TEST_HOOKS", "-DMQ_WAIT_NS=5000000ull"], verbose)
 
 
 if __name__ == "__main__":
     print(build(verbose=os.environ.get("MQ_VERBOSE") == "1"))
+    print(build_test_hooks())

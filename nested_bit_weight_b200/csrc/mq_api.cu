@@ -81,9 +81,17 @@ mq_status check_weights(const mq_weights *w, int64_t N, int64_t K) {
     return MQ_OK;
 }
 
+// M <= 8 dispatch, from the measured crossover of the two kernels on the
+// Llama-3.1-8B shapes (CUDA-graph back-to-back launches over L2-cold
+// weights): the GEMV is ahead up to M = 3 on every shape, at M = 4 on the
+// q/o-size shapes and below, and at M = 5..6 only on the k/v-size shapes;
+// from there the GEMM (whose time barely grows with M) is ahead.
 bool small_m_uses_gemv(int64_t M, int64_t N, int64_t K, int r) {
-    return __atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) == MQ_GEMV_TC &&
-           gemv_tc_supported(M, N, K, r);
+    if (__atomic_load_n(&g_gemv_variant, __ATOMIC_RELAXED) != MQ_GEMV_TC) return false;
+    const int64_t weights = N * K;
+    const bool gemv_ahead = M <= 3 || (M == 4 && weights < (int64_t)32 << 20) ||
+                            (M <= 6 && weights <= (int64_t)8 << 20);
+    return gemv_ahead && gemv_tc_supported(M, N, K, r);
 }
 
 mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,

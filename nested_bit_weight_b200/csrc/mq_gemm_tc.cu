@@ -89,6 +89,13 @@ struct TcCfg {
 
 __device__ unsigned int g_tc_timeout;        // set when a bounded wait gave up
 
+#ifdef MQ_TEST_HOOKS
+// Test-hook builds only: while positive, the X warp of a CTA that takes a
+// unit drops its first load and arrival, so that the MMA's bounded wait runs
+// out (the timeout path, with no fault and no trap).
+__device__ int g_test_drop_x;
+#endif
+
 // Wait of the decode and fold warps for their hand-offs.
 #ifndef MQ_GEMM_WAIT
 #define MQ_GEMM_WAIT mbar_wait_abortable
@@ -386,6 +393,15 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
             for (int i = 0; i < L; ++i) {
                 const int xs = i % kS, kx = i / kS;
                 if (kx > 0 && !mbar_wait_abortable(sempty + xs, (uint32_t)(kx - 1) & 1u, flags)) break;
+#ifdef MQ_TEST_HOOKS
+                if (i == 0 && atomicSub(&g_test_drop_x, 1) > 0) {  // item 0 never arrives
+                    if (++g == G) {
+                        g = 0;
+                        if ((int64_t)(i + 1 + u0) % TG == 0) ++mb;
+                    }
+                    continue;
+                }
+#endif
                 mbar_expect_tx(xfull + xs, C::kXStage);
                 tma_load_3d(sX + xs * C::kXStage, &a.xmap, 0, mb * BM, 2 * g, xfull + xs);
                 flags[3] = i + 1;
@@ -669,3 +685,10 @@ bool gemm_tc_take_timeout(bool *set) {
 }
 
 }  // namespace mq
+
+#ifdef MQ_TEST_HOOKS
+// Test-hook builds only: make the next `n` GEMM CTAs drop one X arrival.
+extern "C" __attribute__((visibility("default"))) int mq_test_drop_x_arrivals(int n) {
+    return (int)cudaMemcpyToSymbol(mq::g_test_drop_x, &n, sizeof(n));
+}
+#endif

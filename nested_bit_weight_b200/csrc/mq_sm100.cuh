@@ -11,8 +11,12 @@
 namespace mq {
 namespace sm100 {
 
-// Bound on every wait inside a kernel: about one second of GPU time.
-constexpr uint64_t kWaitNs = 1000000000ull;
+// Bound on every wait inside a kernel: about one second of GPU time (a
+// test-hook build of the library sets a few milliseconds).
+#ifndef MQ_WAIT_NS
+#define MQ_WAIT_NS 1000000000ull
+#endif
+constexpr uint64_t kWaitNs = MQ_WAIT_NS;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

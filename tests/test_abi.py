@@ -116,3 +116,20 @@ def test_gemm_kernel_query():
             assert mq.mq_gemm_kernel(M, 4096, 4096, 4) == mq.KERNEL_GEMM
     finally:
         mq.mq_set_gemv_variant(old)
+
+
+def test_small_batch_dispatch_table():
+    # the GEMV serves M <= 3 everywhere, M = 4 below 2^25 weights, M = 5..6 up
+    # to 2^23 weights; the GEMM everything else (host logic, no GPU)
+    G, E = mq.KERNEL_GEMV, mq.KERNEL_GEMM
+    table = {(4096, 4096): [G, G, G, G, E, E, E, E],        # q/o: 2^24 weights
+             (1024, 4096): [G, G, G, G, G, G, E, E],        # k/v: 2^22
+             (14336, 4096): [G, G, G, E, E, E, E, E],       # gate/up
+             (4096, 14336): [G, G, G, E, E, E, E, E]}       # down
+    for (N, K), want in table.items():
+        got = [mq.mq_gemm_kernel(M, N, K, 4) for M in range(1, 9)]
+        # without a GPU the GEMV's cluster-occupancy query fails and plans
+        # that need clusters fall back to the GEMM: only the GEMM side of the
+        # table is fixed here (tests/test_gpu_configs.py checks all of it)
+        assert all(g == E for g, w in zip(got, want) if w == E), (N, K, got)
+        assert all(g in (G, E) for g in got)

@@ -133,3 +133,26 @@ def test_gemv_wide_range_x():
         for r in (8, 4, 2):
             Y = mq.gemm(Xd, parent, r).float().cpu().numpy()
             assert oracle.violation_ratio(Y, oracle.gemm(X, codes, s, r)) <= 1.0, (M, r)
+
+
+def test_dispatch_table_on_gpu():
+    # the small-batch dispatch on the Llama-3.1-8B shapes: GEMV up to M = 3
+    # everywhere, M = 4 on q/o and k/v, M = 5..6 on k/v only
+    import nested_bit_weight_b200 as mq
+    G, E = mq.KERNEL_GEMV, mq.KERNEL_GEMM
+    table = {(4096, 4096): [G, G, G, G, E, E, E, E],
+             (1024, 4096): [G, G, G, G, G, G, E, E],
+             (14336, 4096): [G, G, G, E, E, E, E, E],
+             (4096, 14336): [G, G, G, E, E, E, E, E]}
+    for (N, K), want in table.items():
+        for r in (4, 2):
+            assert [mq.mq_gemm_kernel(M, N, K, r) for M in range(1, 9)] == want, (N, K, r)
+
+
+@pytest.mark.parametrize("r", [4, 2])
+@pytest.mark.parametrize("M", [3, 4, 5, 6, 7])
+@pytest.mark.parametrize("li,name,N,K", LLAMA_SHAPES)
+def test_dispatch_boundaries(li, name, N, K, M, r):
+    # both sides of every GEMV / GEMM boundary of the small-batch dispatch
+    # (gate/down 3|4, q 4|5, k 6|7), each kernel on its side
+    assert _check(2, li, N, K, M, r) <= 1.0

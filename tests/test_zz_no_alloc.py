@@ -55,8 +55,8 @@ def _check_twice(N, K, M, r, seed):
 
 @pytest.mark.parametrize("M,r", [(1, 3), (3, 2), (8, 4)])
 def test_noalloc_matches_mq_gemm_twice(M, r):
-    # the default kernel for these shapes is the tensor-core GEMV, which
-    # needs no scratch
+    # by default M = 1 and 3 take the tensor-core GEMV (no scratch) and M = 8
+    # the GEMM, which uses the built-in scratch
     _check_twice(1024, 4096, M, r, seed=31 + M)
 
 
