@@ -264,6 +264,54 @@ def run_per_points():
     return out
 
 
+def run_chain(layers, steps: int):
+    """Config 1 as one decoder layer per r: fused q|k|v, o, fused gate|up and
+    down (4 launches per r, 12 per step), each r on its own parents (L2-cold),
+    enqueued by mq_gemm_chain and timed as a CUDA graph."""
+    import torch
+    import nested_bit_weight_b200 as mq
+    peak, _ = read_peaks()
+    idx = {l.name: i for i, l in enumerate(wl.LLAMA8B)}
+    dev = lambda a: torch.from_numpy(a).cuda()
+    C = {n: dev(layers[idx[n]][0]) for n in idx}
+    S = {n: dev(layers[idx[n]][1]) for n in idx}
+    X = {n: torch.from_numpy(layers[idx[n]][2].view(np.int16)).cuda().view(torch.bfloat16) for n in idx}
+    calls, nbytes = [], 0
+    for r in R_LIST:
+        qkv = mq.pack_fused([C["q_proj"], C["k_proj"], C["v_proj"]], [S["q_proj"], S["k_proj"], S["v_proj"]])
+        gu = mq.pack_fused([C["gate_proj"], C["up_proj"]], [S["gate_proj"], S["up_proj"]])
+        o = mq.pack_parent(C["o_proj"], S["o_proj"])
+        dn = mq.pack_parent(C["down_proj"], S["down_proj"])
+        for w, xn in ((qkv, "q_proj"), (o, "o_proj"), (gu, "gate_proj"), (dn, "down_proj")):
+            Y = torch.empty((M, w.N), dtype=torch.bfloat16, device="cuda")
+            calls.append((X[xn], w, r, Y))
+            nbytes += algo_bytes(w.N, w.K, r, M)
+    stream = torch.cuda.Stream()
+    with torch.cuda.stream(stream):
+        mq.gemm_chain(calls)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            mq.gemm_chain(calls)
+        for _ in range(3):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(steps):
+            g.replay()
+        e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    gbps = nbytes / (ms * 1e-3) / 1e9
+    del g
+    return {"note": "config 1 as one decoder layer per r: fused q|k|v, o, fused gate|up, "
+                    "down (4 launches per r, 12 per step), mq_gemm_chain in a CUDA graph, "
+                    "each r on its own parents (L2-cold)",
+            "ms_per_step": round(ms, 5), "bytes_per_step": nbytes, "GBps": round(gbps, 1),
+            "frac_hbm": round(gbps / peak, 4), "launches_per_step": len(calls)}
+
+
 def cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -528,6 +576,7 @@ def run_mq(args, ws_n, rank, local):
         "per_launch_isolated": detail,
     }
     if ws_n == 1:
+        out["decoder_layer_chain"] = run_chain(layers, max(args.steps, 20))
         out["per_point"] = {"note": "config 2 points (Llama-3.1-8B gate and q), each shape "
                                     "alone over rotated weights (L2-cold): median, p10, p90 "
                                     "of >= 100 launches timed one by one, and the mean of the "

@@ -143,23 +143,46 @@ MQ_API size_t mq_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K, int r);
  * overlap the inputs.  M == 0 is accepted and does nothing.
  * The fp32 accumulation order is fixed, so results are deterministic.
  *
- * Stream order.  The GEMV (MQ_KERNEL_GEMV) is launched with programmatic
- * dependent launch: it may start while the preceding kernel on the stream is
- * still running, and it begins streaming the weights (planes and scales)
- * before it waits for that kernel; X is read, and Y and the workspace are
- * written, only after the preceding kernel has completed and its writes are
- * visible.  So the weights must not be written by the immediately preceding
- * kernel on the same stream if that kernel lets its dependents launch early
+ * Stream order.  Both kernels are launched with programmatic dependent
+ * launch: a call may start while the preceding kernel on the stream is still
+ * running, and it begins streaming the weights (planes and scales) before it
+ * waits for that kernel; X is read, and Y and the workspace are written, only
+ * after the preceding kernel has completed and its writes are visible.  So
+ * the weights must not be written by the immediately preceding kernel on the
+ * same stream if that kernel lets its dependents launch early
  * (griddepcontrol.launch_dependents or its CUDA equivalent).  Kernels that
  * never do so -- mq_pack, torch's kernels, cudaMemcpy -- are safe: their
- * dependents start only after they have completed.  Weights written by a
- * kernel that does trigger early need a cudaStreamSynchronize or an event
- * wait on another stream before mq_gemm.  The M >= 9 GEMM is launched
- * without programmatic dependent launch and reads nothing early.
+ * dependents start only after they have completed.  mq_gemm's own kernels
+ * do trigger early, so weights produced by an mq_gemm call need a
+ * cudaStreamSynchronize or an event wait on another stream first (outputs Y
+ * used as the next call's X are fine).
  */
 MQ_API mq_status mq_gemm(const uint16_t *X_dev, const mq_weights *w,
                   int64_t M, int64_t N, int64_t K, uint16_t *Y_dev,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* One product of a chain: Y = X . W_r^T with N = w->N, K = w->K. */
+typedef struct mq_call {
+    const uint16_t *X;       /* bf16 M x K, device */
+    const mq_weights *w;     /* r-bit view */
+    int64_t M;               /* rows of X (>= 0) */
+    uint16_t *Y;             /* bf16 M x N, device */
+} mq_call;
+
+/*
+ * A chain of products, such as the linear layers of one decoder layer (the
+ * fused q|k|v, o, fused gate|up and down projections at their own bit widths:
+ * MatGPTQ author page, abstract: heterogeneous per-layer bit-widths served as
+ * one mixed-precision model), enqueued back to back on one stream in array
+ * order.  Consecutive launches overlap through programmatic dependent launch
+ * (see mq_gemm, Stream order): a call may read the previous call's Y as its
+ * X.  Each call follows mq_gemm's preconditions; the workspace must hold
+ * mq_gemm_workspace_bytes of every call (they run in stream order, so one
+ * workspace serves all).  Validation of every call happens before the first
+ * launch: on an error nothing is enqueued.  n == 0 does nothing.
+ */
+MQ_API mq_status mq_gemm_chain(const mq_call *calls, int n, void *workspace,
+                               size_t workspace_bytes, void *stream);
 
 /* Kernels for M <= 8 (both compute the same Y within the stated tolerance). */
 enum {

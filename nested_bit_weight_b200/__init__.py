@@ -18,6 +18,7 @@ __all__ = [
     "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
     "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
     "mq_device_status", "mq_gemm_kernel", "uses_gemv", "KERNEL_GEMV", "KERNEL_GEMM",
+    "MqCall", "mq_gemm_chain", "gemm_chain", "pack_fused", "workspace_for",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +41,12 @@ class MqWeights(ctypes.Structure):
     _fields_ = [("planes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64),
                 ("group", ctypes.c_int32), ("r", ctypes.c_int32)]
+
+
+class MqCall(ctypes.Structure):
+    """One product of mq_gemm_chain (mq_call in include/mq.h)."""
+    _fields_ = [("X", ctypes.c_void_p), ("w", ctypes.POINTER(MqWeights)),
+                ("M", ctypes.c_int64), ("Y", ctypes.c_void_p)]
 
 
 def _load() -> ctypes.CDLL:
@@ -66,6 +73,7 @@ def _load() -> ctypes.CDLL:
         "mq_set_gemv_variant": (I, [I]),
         "mq_get_gemv_variant": (I, []),
         "mq_gemm_kernel": (I, [I64, I64, I64, I]),
+        "mq_gemm_chain": (I, [ctypes.POINTER(MqCall), I, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -158,6 +166,20 @@ def mq_gemm(X, w: MqWeights, Y, workspace=None, stream=None) -> None:
                        ws_ptr, ws_bytes, _stream(stream)))
 
 
+def mq_gemm_chain(calls, workspace=None, stream=None) -> None:
+    """Enqueue the products [(X, w, Y), ...] back to back (X, Y bf16 device
+    tensors, w an MqWeights view): a call may read the previous call's Y."""
+    arr = (MqCall * len(calls))()
+    keep = []
+    for i, (X, w, Y) in enumerate(calls):
+        wp = ctypes.pointer(w)
+        keep.append(wp)
+        arr[i] = MqCall(X.data_ptr(), wp, X.shape[0], Y.data_ptr())
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.mq_gemm_chain(arr, len(calls), ws_ptr, ws_bytes, _stream(stream)))
+
+
 def mq_unpack(w: MqWeights, codes_out, stream=None) -> None:
     _check(lib.mq_unpack(ctypes.byref(w), codes_out.data_ptr(), _stream(stream)))
 
@@ -185,6 +207,50 @@ def pack_parent(codes, scales, stream=None) -> NestedWeights:
     return NestedWeights(planes, s16, N, K)
 
 
+def pack_fused(codes_list, scales_list, stream=None) -> NestedWeights:
+    """One parent for several layers that share X (q|k|v, gate|up): their
+    rows concatenated (codes uint8 [N_i, K], scales fp32 [N_i, K/128] device
+    tensors), so one launch computes all of them; Y's columns follow the same
+    order (layer i at rows offsets[i] .. offsets[i] + N_i of W)."""
+    import torch
+    codes = torch.cat(list(codes_list), dim=0).contiguous()
+    scales = torch.cat(list(scales_list), dim=0).contiguous()
+    w = pack_parent(codes, scales, stream)
+    offs, o = [], 0
+    for c in codes_list:
+        offs.append(o)
+        o += c.shape[0]
+    w.offsets = offs
+    return w
+
+
+def workspace_for(device, need: int):
+    """The cached zero-initialised workspace of `device`, at least `need` bytes."""
+    import torch
+    key = device.index
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def gemm_chain(calls, stream=None):
+    """[(X, NestedWeights, r, Y or None), ...] -> the Y tensors, enqueued as
+    one mq_gemm_chain (consecutive launches overlap)."""
+    import torch
+    views, outs, need = [], [], 0
+    for X, weights, r, Y in calls:
+        if Y is None:
+            Y = torch.empty((X.shape[0], weights.N), dtype=torch.bfloat16, device=X.device)
+        views.append((X, weights.view(r), Y))
+        outs.append(Y)
+        need = max(need, mq_gemm_workspace_bytes(X.shape[0], weights.N, weights.K, r))
+    ws = workspace_for(calls[0][0].device, need) if need else None
+    mq_gemm_chain(views, ws, stream)
+    return outs
+
+
 _ws_cache: dict = {}
 
 
@@ -196,12 +262,6 @@ def gemm(X, weights: NestedWeights, r: int, Y=None, stream=None):
     if Y is None:
         Y = torch.empty((M, weights.N), dtype=torch.bfloat16, device=X.device)
     need = mq_gemm_workspace_bytes(M, weights.N, K, r)
-    ws = None
-    if need:
-        key = X.device.index
-        ws = _ws_cache.get(key)
-        if ws is None or ws.numel() < need:
-            ws = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=X.device)
-            _ws_cache[key] = ws
+    ws = workspace_for(X.device, need) if need else None
     mq_gemm(X, w, Y, ws, stream)
     return Y

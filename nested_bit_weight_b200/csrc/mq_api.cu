@@ -101,6 +101,13 @@ mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M, uint
     return launch_gemm_tc(X, w, M, Y, ws, ws_bytes, st);
 }
 
+// fail() with a formatted message.
+template <class... A>
+mq_status failf(mq_status s, const char *fmt, A... args) {
+    set_error(s, fmt, args...);
+    return s;
+}
+
 }  // namespace mq
 
 using namespace mq;
@@ -155,6 +162,38 @@ mq_status mq_gemm(const uint16_t *X, const mq_weights *w, int64_t M, int64_t N,
     if ((s = bind_device(st)) != MQ_OK) return s;
     if (M <= kGemvMaxM) return launch_small_m(X, w, M, Y, workspace, workspace_bytes, st);
     return launch_gemm_tc(X, w, M, Y, workspace, workspace_bytes, st);
+}
+
+mq_status mq_gemm_chain(const mq_call *calls, int n, void *workspace, size_t workspace_bytes,
+                        void *stream) {
+    if (n < 0 || (n > 0 && !calls)) return fail(MQ_ERR_INVALID_ARG, "bad chain (n < 0 or calls NULL)");
+    if (workspace && !aligned16(workspace)) return fail(MQ_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    // validate every call before launching any
+    for (int i = 0; i < n; ++i) {
+        const mq_call &c = calls[i];
+        if (!c.w) return failf(MQ_ERR_INVALID_ARG, "chain call %d: weights are NULL", i);
+        mq_status s = check_weights(c.w, c.w->N, c.w->K);
+        if (s != MQ_OK) return s;
+        if (c.M < 0) return failf(MQ_ERR_INVALID_ARG, "chain call %d: M must be >= 0", i);
+        if (c.M == 0) continue;
+        if (!c.X || !c.Y) return failf(MQ_ERR_INVALID_ARG, "chain call %d: X or Y is NULL", i);
+        if (!aligned16(c.X) || !aligned16(c.Y))
+            return failf(MQ_ERR_MISALIGNED, "chain call %d: X and Y must be 16-byte aligned", i);
+        const size_t need = mq_gemm_workspace_bytes(c.M, c.w->N, c.w->K, c.w->r);
+        if (need && (!workspace || workspace_bytes < need))
+            return failf(MQ_ERR_WORKSPACE, "chain call %d: workspace smaller than mq_gemm_workspace_bytes", i);
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    mq_status s = bind_device(st);
+    if (s != MQ_OK) return s;
+    for (int i = 0; i < n; ++i) {
+        const mq_call &c = calls[i];
+        if (c.M == 0) continue;
+        s = c.M <= kGemvMaxM ? launch_small_m(c.X, c.w, c.M, c.Y, workspace, workspace_bytes, st)
+                             : launch_gemm_tc(c.X, c.w, c.M, c.Y, workspace, workspace_bytes, st);
+        if (s != MQ_OK) return s;
+    }
+    return MQ_OK;
 }
 
 mq_status mq_set_gemv_variant(int variant) {

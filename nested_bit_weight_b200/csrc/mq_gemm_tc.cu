@@ -32,6 +32,9 @@
 //   fold warps      4 (BM <= 64) or 8 (BM = 128), one or two per TMEM lane
 //                   quarter: y += s[n, g] * D_g, the tile's fp32 sums kept in
 //                   registers until the tile ends.
+// Launched with programmatic dependent launch: the decode warps stream the
+// weights before the previous kernel of the stream has completed; X is read
+// and Y and the workspace written only after griddepcontrol.wait.
 // Every wait is bounded (about a second); a wait that gives up sets a CTA
 // abort flag that ends the others at once, and a device flag read by
 // mq_device_status.  Arrival tickets always return to zero, also after a
@@ -192,6 +195,10 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(dempty + kS) + 12;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // programmatic dependent launch: the next kernel of the stream may start
+    // its prologue as SMs free up (it reads our output only after its own
+    // wait, which returns once this grid has completed)
+    if (threadIdx.x == 0) pdl_launch_dependents();
     const int64_t W = (int64_t)a.MB * a.T * a.G;
     const int64_t u0 = range_first(blockIdx.x, W, a.P), u1 = range_first(blockIdx.x + 1, W, a.P);
     const int L = (int)(u1 - u0);
@@ -306,6 +313,7 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
             if (k < L) scale_issue(k);
             cp_async_commit();
         }
+        pdl_wait();                                            // Y and the workspace: after the previous kernel
         for (int i = 0; i < L; ++i) {
             const int db = i % kS;
             cp_async_wait<kScaleAhead - 1>();                  // item i's scale is in
@@ -389,6 +397,7 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
     } else if (warp == kXW) {
         // ----------------------------------------------------------------- X
         if (lane == 0) {
+            pdl_wait();                                        // X may come from the previous kernel
             int mb = (int)(u0 / TG), g = (int)(u0 % G);        // X block and group of item i
             for (int i = 0; i < L; ++i) {
                 const int xs = i % kS, kx = i / kS;
@@ -670,8 +679,17 @@ mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint
     a.P = p.P;
     a.maxc = p.maxc;
     a.plane_words = (int64_t)p.T * kTileN * (w->K / 32);
-    fn<<<p.P, threads, smem, st>>>(a);
-    e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)p.P);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, fn, a);
     if (e != cudaSuccess) return cuda_fail(e, "gemm_tc_kernel");
     return MQ_OK;
 }

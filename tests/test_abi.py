@@ -133,3 +133,27 @@ def test_small_batch_dispatch_table():
         # table is fixed here (tests/test_gpu_configs.py checks all of it)
         assert all(g == E for g, w in zip(got, want) if w == E), (N, K, got)
         assert all(g in (G, E) for g in got)
+
+
+def test_chain_argument_errors_before_launch():
+    # every call of a chain is validated before anything is enqueued (no GPU)
+    import ctypes
+    w = _parent(N=64, K=256, r=4)
+    X, Y = FAKE, FAKE * 4
+    ok_call = mq.MqCall(X, ctypes.pointer(w), 16, Y)
+    bad_m = mq.MqCall(X, ctypes.pointer(w), -1, Y)
+    bad_align = mq.MqCall(X + 8, ctypes.pointer(w), 16, Y)
+    no_w = mq.MqCall(X, None, 16, Y)
+    arr = lambda *c: (mq.MqCall * len(c))(*c)
+    WS, BIG = FAKE * 8, 1 << 30      # a workspace that passes the size check
+    assert mq.lib.mq_gemm_chain(arr(ok_call), -1, WS, BIG, None) == 1
+    assert mq.lib.mq_gemm_chain(None, 0, None, 0, None) == 0
+    # a bad call anywhere in the chain: refused, nothing enqueued
+    assert mq.lib.mq_gemm_chain(arr(ok_call, bad_m), 2, WS, BIG, None) == 1
+    assert mq.lib.mq_gemm_chain(arr(ok_call, no_w), 2, WS, BIG, None) == 1
+    assert mq.lib.mq_gemm_chain(arr(ok_call, bad_align), 2, WS, BIG, None) == 3
+    assert mq.lib.mq_gemm_chain(arr(ok_call), 1, WS + 4, BIG, None) == 3
+    # M = 16 needs the GEMM's workspace: missing or too small is refused
+    assert mq.mq_gemm_workspace_bytes(16, 64, 256, 4) > 0
+    assert mq.lib.mq_gemm_chain(arr(ok_call), 1, None, 0, None) == 6
+    assert mq.lib.mq_gemm_chain(arr(ok_call), 1, FAKE * 8, 1024, None) == 6
