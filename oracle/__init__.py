@@ -50,9 +50,11 @@ def _load():
         lib.oracle_unpack.argtypes = [P, I64, I64, I, P]
         lib.oracle_gemm_f64.argtypes = [P, P, P, I64, I64, I64, I, P]
         lib.oracle_gemm_f64_at.argtypes = [P, P, P, I64, I, I64, P, P, P]
+        lib.oracle_gemm_asym_f64.argtypes = [P, P, P, P, I64, I64, I64, I, P]
+        lib.oracle_gemm_asym_f64_at.argtypes = [P, P, P, P, I64, I, I64, P, P, P]
         lib.oracle_threads.restype = I
         for f in (lib.oracle_pack, lib.oracle_unpack, lib.oracle_gemm_f64,
-                  lib.oracle_gemm_f64_at):
+                  lib.oracle_gemm_f64_at, lib.oracle_gemm_asym_f64, lib.oracle_gemm_asym_f64_at):
             f.restype = None
         _lib = lib
     return _lib
@@ -92,6 +94,29 @@ def dequant(codes: np.ndarray, s: np.ndarray, r: int) -> np.ndarray:
     s16 = scales_f16(s).astype(np.float64)
     v = level(slice_codes(codes, r), r)
     return v * np.repeat(s16, 128, axis=1)
+
+
+# Asymmetric variant ("MatGPTQ: Efficient and Accurate Inference over Nested
+# Quantized Models", captions of Tables 4-7, "asymmetric MatGPTQ"; no formula
+# on the pages): a per-group zero point z, real, in units of the 8-bit code,
+# stored as fp16 and shared by every r; the level is measured from it.
+
+def level_asym(q_r: np.ndarray, r: int, z: np.ndarray) -> np.ndarray:
+    """u_r = 2^(8-r) q_r + 2^(7-r) - z, in fp64 (z = 128: the symmetric level)."""
+    return (2.0 ** (8 - r)) * q_r.astype(np.float64) + 2.0 ** (7 - r) - np.asarray(z, np.float64)
+
+
+def zeros_f16(z: np.ndarray) -> np.ndarray:
+    """The stored zero point: fp32 z rounded to fp16 (round-to-nearest-even)."""
+    with np.errstate(over="ignore"):
+        return np.asarray(z, np.float32).astype(np.float16)
+
+
+def dequant_asym(codes: np.ndarray, s: np.ndarray, z: np.ndarray, r: int) -> np.ndarray:
+    """W_r[n, k] = s16[n, k // 128] * u_r(q_r[n, k], z16[n, k // 128]) in fp64."""
+    s16 = np.repeat(scales_f16(s).astype(np.float64), 128, axis=1)
+    z16 = np.repeat(zeros_f16(z).astype(np.float64), 128, axis=1)
+    return s16 * level_asym(slice_codes(codes, r), r, z16)
 
 
 # ------------------------------------------------------------- plain-C kernels
@@ -149,6 +174,38 @@ def gemm(X: np.ndarray, codes: np.ndarray, s: np.ndarray, r: int) -> np.ndarray:
     Y = np.empty((M, N), np.float64)
     _load().oracle_gemm_f64(_ptr(X), _ptr(codes), _ptr(s16), M, N, K, r, _ptr(Y))
     return Y
+
+
+def zeros_stored(z: np.ndarray) -> np.ndarray:
+    """The stored zero points: fp16 (RNE) in the same tiled order as the scales."""
+    return scales_stored(np.asarray(zeros_f16(z), np.float32))
+
+
+def gemm_asym(X: np.ndarray, codes: np.ndarray, s: np.ndarray, z: np.ndarray, r: int) -> np.ndarray:
+    """Y = X . W_r^T for the asymmetric variant (fp64, ascending k)."""
+    X = np.ascontiguousarray(X, np.float64)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    s16 = np.ascontiguousarray(scales_f16(s).astype(np.float64))
+    z16 = np.ascontiguousarray(zeros_f16(z).astype(np.float64))
+    M, K = X.shape
+    N = codes.shape[0]
+    Y = np.empty((M, N), np.float64)
+    _load().oracle_gemm_asym_f64(_ptr(X), _ptr(codes), _ptr(s16), _ptr(z16), M, N, K, r, _ptr(Y))
+    return Y
+
+
+def gemm_asym_at(X, codes, s, z, r, ms, ns) -> np.ndarray:
+    """The asymmetric Y[ms[i], ns[i]] for a list of output positions."""
+    X = np.ascontiguousarray(X, np.float64)
+    codes = np.ascontiguousarray(codes, np.uint8)
+    s16 = np.ascontiguousarray(scales_f16(s).astype(np.float64))
+    z16 = np.ascontiguousarray(zeros_f16(z).astype(np.float64))
+    ms = np.ascontiguousarray(ms, np.int64)
+    ns = np.ascontiguousarray(ns, np.int64)
+    out = np.empty(ms.shape[0], np.float64)
+    _load().oracle_gemm_asym_f64_at(_ptr(X), _ptr(codes), _ptr(s16), _ptr(z16), X.shape[1], r,
+                                    ms.shape[0], _ptr(ms), _ptr(ns), _ptr(out))
+    return out
 
 
 def gemm_at(X, codes, s, r, ms, ns) -> np.ndarray:

@@ -123,6 +123,61 @@ void oracle_gemm_f64_at(const double *X, const uint8_t *codes,
     }
 }
 
+/*
+ * Asymmetric variant (MatGPTQ paper page, captions of Tables 4-7:
+ * "asymmetric MatGPTQ"; the pages give no formula, the reading taken: each
+ * 128-column group also has a zero point z, real-valued in units of the
+ * 8-bit code and stored as fp16, shared by every r like the scale):
+ *
+ *   level:   u_r = 2^(8-r) * q_r + 2^(7-r) - z16[n, k/128]
+ *   weight:  w[n,k] = s16[n, k/128] * u_r[n,k]
+ *
+ * z = 128 gives the symmetric level v_r above.
+ */
+static double level_asym(unsigned q_r, int r, double z)
+{
+    double a = (double)(1u << (8 - r));                 /* 2^(8-r) */
+    double b = (r == 8) ? 0.5 : (double)(1u << (7 - r)); /* 2^(7-r) */
+    return a * (double)q_r + b - z;
+}
+
+void oracle_gemm_asym_f64(const double *X, const uint8_t *codes, const double *s16,
+                          const double *z16, int64_t M, int64_t N, int64_t K, int r,
+                          double *Y)
+{
+    int64_t G = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t m = 0; m < M; ++m) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                unsigned q_r = (unsigned)codes[n * K + k] >> (8 - r);
+                double w = s16[n * G + k / 128] * level_asym(q_r, r, z16[n * G + k / 128]);
+                acc += X[m * K + k] * w;
+            }
+            Y[m * N + n] = acc;
+        }
+    }
+}
+
+void oracle_gemm_asym_f64_at(const double *X, const uint8_t *codes, const double *s16,
+                             const double *z16, int64_t K, int r, int64_t count,
+                             const int64_t *ms, const int64_t *ns, double *out)
+{
+    int64_t G = K / 128;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < count; ++i) {
+        int64_t m = ms[i], n = ns[i];
+        double acc = 0.0;
+        for (int64_t k = 0; k < K; ++k) {
+            unsigned q_r = (unsigned)codes[n * K + k] >> (8 - r);
+            double w = s16[n * G + k / 128] * level_asym(q_r, r, z16[n * G + k / 128]);
+            acc += X[m * K + k] * w;
+        }
+        out[i] = acc;
+    }
+}
+
 /* Number of OpenMP threads the gemm loops use (1 without OpenMP). */
 int oracle_threads(void)
 {

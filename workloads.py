@@ -101,6 +101,41 @@ def gen_weights(N: int, K: int, seed: int, outlier_frac: float = 0.01):
     return codes, s, W
 
 
+def gen_weights_asym(N: int, K: int, seed: int, outlier_frac: float = 0.01):
+    """Asymmetric codes: (codes uint8 [N, K], scales fp32 [N, K/128], zero
+    points fp32 [N, K/128], W fp32 [N, K]).
+
+    W as gen_weights plus a per-(row, group) offset ~ N(0, 0.02^2), so that
+    groups are not centred; per group s = (max W - min W) / 255 and
+    z = -min W / s (real, in code units); q = clamp(rint(W / s + z - 0.5),
+    0, 255), so that the midpoint level s (q + 0.5 - z) is nearest to W.  A
+    constant group gets s = 0, z = 128, codes 128.
+    """
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    rng = np.random.default_rng(seed + 7919)
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    n_out = int(np.floor(outlier_frac * N * K))
+    if n_out:
+        idx = rng.choice(N * K, size=n_out, replace=False)
+        W.reshape(-1)[idx] *= np.float32(10.0)
+    G = K // GROUP
+    Wg = W.reshape(N, G, GROUP)
+    Wg += (rng.standard_normal((N, G, 1), dtype=np.float32) * np.float32(0.02))
+    lo, hi = Wg.min(axis=2), Wg.max(axis=2)
+    s = ((hi - lo) / np.float32(255.0)).astype(np.float32)
+    z = np.full((N, G), 128.0, np.float32)
+    nz = s != 0
+    z[nz] = (-lo[nz] / s[nz]).astype(np.float32)
+    t = np.zeros_like(Wg)
+    np.divide(Wg, s[:, :, None], out=t, where=nz[:, :, None])
+    t += z[:, :, None] - np.float32(0.5)
+    np.rint(t, out=t)
+    t[np.broadcast_to(~nz[:, :, None], t.shape)] = 128.0
+    np.clip(t, 0, 255, out=t)
+    return t.astype(np.uint8).reshape(N, K), s, z, W
+
+
 def gen_x(M: int, K: int, seed: int, outlier_channels: bool = False):
     """Return X as (bf16 bit patterns uint16 [M, K], exact fp32 values [M, K]).
 
