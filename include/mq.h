@@ -75,6 +75,8 @@ typedef struct {
     int64_t K;                /* input features, multiple of 128 */
     int32_t group;            /* columns per scale; must be 128 */
     int32_t r;                /* bits per weight, 1..8 */
+    const uint16_t *zeros;    /* device: fp16 zero points in the scales' order (mq_pack_zeros),
+                                 or NULL for the symmetric format (the zero point 128) */
 } mq_weights;
 
 /* Bytes of the first r planes: r * N128 * K / 8 (0 on invalid arguments). */
@@ -101,6 +103,21 @@ MQ_API size_t mq_scale_bytes(int64_t N, int64_t K, int group);
 MQ_API mq_status mq_pack(const uint8_t *codes_dev, const float *scales_dev,
                   int64_t N, int64_t K, int group,
                   uint32_t *planes_out, uint16_t *scales_out, void *stream);
+
+/*
+ * Asymmetric variant (MatGPTQ paper page, captions of Tables 4-7: asymmetric
+ * MatGPTQ): a zero point z per 128-column group, real, in units of the 8-bit
+ * code, shared by every r; the weight is s * (2^(8-r) q_r + 2^(7-r) - z)
+ * (z = 128 is the symmetric format).  Round the fp32 zero points to fp16 in
+ * the tiled block order of the scales.
+ *   zeros_dev  fp32 N x (K/group)
+ *   zeros_out  fp16 bits, mq_scale_bytes(N, K, 128) bytes (padding rows 0)
+ * Preconditions as mq_pack; synchronous, MQ_ERR_UNSUPPORTED when a zero
+ * point is NaN or rounds to an fp16 infinity.  Set the result as
+ * mq_weights.zeros of the parent (mq_slice keeps it).
+ */
+MQ_API mq_status mq_pack_zeros(const float *zeros_dev, int64_t N, int64_t K, int group,
+                               uint16_t *zeros_out, void *stream);
 
 /*
  * Select the r-bit model of a parent: host-only, O(1), no device work and no
@@ -210,10 +227,11 @@ enum {
 };
 
 /*
- * Which kernel mq_gemm(M, N, K, r) would run under the current variant
- * (host only, no device work): MQ_KERNEL_GEMV or MQ_KERNEL_GEMM, 0 for an
- * invalid problem (M < 1, N < 1, K not a positive multiple of 128, r outside
- * 1..8).  Lets a caller or a benchmark label its timings; it has no effect on
+ * Which kernel mq_gemm(M, N, K, r) would run under the current variant for
+ * symmetric weights (host only, no device work): MQ_KERNEL_GEMV or
+ * MQ_KERNEL_GEMM, 0 for an invalid problem (M < 1, N < 1, K not a positive
+ * multiple of 128, r outside 1..8).  Weights with zero points always run the
+ * GEMM.  Lets a caller or a benchmark label its timings; it has no effect on
  * the call itself.
  */
 MQ_API int mq_gemm_kernel(int64_t M, int64_t N, int64_t K, int r);

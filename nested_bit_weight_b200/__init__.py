@@ -18,7 +18,7 @@ __all__ = [
     "mq_gemm_workspace_bytes", "mq_unpack", "mq_version", "pack_parent", "gemm",
     "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
     "mq_device_status", "mq_gemm_kernel", "uses_gemv", "KERNEL_GEMV", "KERNEL_GEMM",
-    "MqCall", "mq_gemm_chain", "gemm_chain", "pack_fused", "workspace_for",
+    "MqCall", "mq_gemm_chain", "gemm_chain", "pack_fused", "workspace_for", "mq_pack_zeros",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +40,8 @@ class MqWeights(ctypes.Structure):
     """Mirror of the C struct mq_weights (a view, owns nothing)."""
     _fields_ = [("planes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64),
-                ("group", ctypes.c_int32), ("r", ctypes.c_int32)]
+                ("group", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("zeros", ctypes.c_void_p)]                # fp16 zero points or None (symmetric)
 
 
 class MqCall(ctypes.Structure):
@@ -74,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "mq_get_gemv_variant": (I, []),
         "mq_gemm_kernel": (I, [I64, I64, I64, I]),
         "mq_gemm_chain": (I, [ctypes.POINTER(MqCall), I, P, SZ, P]),
+        "mq_pack_zeros": (I, [P, I64, I64, I, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -187,24 +189,38 @@ def mq_unpack(w: MqWeights, codes_out, stream=None) -> None:
 # ------------------------------------------------------------- owning helpers
 
 class NestedWeights:
-    """A packed 8-bit parent (device tensors) and its r-bit views."""
+    """A packed 8-bit parent (device tensors) and its r-bit views; zeros16
+    (fp16 zero points, asymmetric variant) or None."""
 
-    def __init__(self, planes, scales16, N: int, K: int):
+    def __init__(self, planes, scales16, N: int, K: int, zeros16=None):
         self.planes, self.scales16, self.N, self.K = planes, scales16, N, K
-        self.parent = MqWeights(planes.data_ptr(), scales16.data_ptr(), N, K, 128, 8)
+        self.zeros16 = zeros16
+        self.parent = MqWeights(planes.data_ptr(), scales16.data_ptr(), N, K, 128, 8,
+                                zeros16.data_ptr() if zeros16 is not None else None)
 
     def view(self, r: int) -> MqWeights:
         return mq_slice(self.parent, r)
 
 
-def pack_parent(codes, scales, stream=None) -> NestedWeights:
-    """Allocate the 8-plane buffer and fp16 scales with torch, then mq_pack."""
+def mq_pack_zeros(zeros, zeros_out, stream=None) -> None:
+    """zero points fp32 [N, K/128] -> fp16 in the scales' tiled order (device)."""
+    N, G = zeros.shape
+    _check(lib.mq_pack_zeros(zeros.data_ptr(), N, G * 128, 128, zeros_out.data_ptr(), _stream(stream)))
+
+
+def pack_parent(codes, scales, stream=None, zeros=None) -> NestedWeights:
+    """Allocate the 8-plane buffer and fp16 scales with torch, then mq_pack;
+    with `zeros` (fp32 [N, K/128]) the asymmetric variant."""
     import torch
     N, K = codes.shape
     planes = torch.empty(mq_plane_bytes(N, K, 8) // 4, dtype=torch.int32, device=codes.device)
     s16 = torch.empty(mq_scale_bytes(N, K, 128) // 2, dtype=torch.float16, device=codes.device)
     mq_pack(codes, scales, planes, s16, stream)
-    return NestedWeights(planes, s16, N, K)
+    z16 = None
+    if zeros is not None:
+        z16 = torch.empty(mq_scale_bytes(N, K, 128) // 2, dtype=torch.float16, device=codes.device)
+        mq_pack_zeros(zeros, z16, stream)
+    return NestedWeights(planes, s16, N, K, z16)
 
 
 def pack_fused(codes_list, scales_list, stream=None) -> NestedWeights:

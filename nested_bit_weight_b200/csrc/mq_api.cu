@@ -76,8 +76,8 @@ mq_status check_weights(const mq_weights *w, int64_t N, int64_t K) {
         return fail(MQ_ERR_INVALID_ARG, "weights view shape differs from (N, K)");
     if (N < 1 || K < kGroup || K % kGroup)
         return fail(MQ_ERR_INVALID_ARG, "need N >= 1 and K a positive multiple of 128");
-    if (!aligned16(w->planes) || !aligned16(w->scales))
-        return fail(MQ_ERR_MISALIGNED, "planes and scales must be 16-byte aligned");
+    if (!aligned16(w->planes) || !aligned16(w->scales) || (w->zeros && !aligned16(w->zeros)))
+        return fail(MQ_ERR_MISALIGNED, "planes, scales and zero points must be 16-byte aligned");
     return MQ_OK;
 }
 
@@ -96,7 +96,8 @@ bool small_m_uses_gemv(int64_t M, int64_t N, int64_t K, int r) {
 
 mq_status launch_small_m(const uint16_t *X, const mq_weights *w, int64_t M, uint16_t *Y,
                          void *ws, size_t ws_bytes, cudaStream_t st) {
-    if (small_m_uses_gemv(M, w->N, w->K, w->r))
+    // the asymmetric variant runs on the GEMM for every M
+    if (!w->zeros && small_m_uses_gemv(M, w->N, w->K, w->r))
         return launch_gemv_tc(X, w, M, Y, ws, ws_bytes, st);
     return launch_gemm_tc(X, w, M, Y, ws, ws_bytes, st);
 }

@@ -73,7 +73,9 @@ __host__ __device__ constexpr int x_stages(int BM) { return BM == 128 ? 2 : 4; }
 constexpr int kScaleAhead = 8;                // items of scales in flight per fold thread
 __host__ __device__ constexpr size_t tc_smem_bytes(int r, int BM) {
     return 1024 + (size_t)x_stages(BM) * BM * 256 + (size_t)ring_items(r, BM) * r * 2048 +
-           (size_t)256 * kScaleAhead * 4 + 512;
+           (size_t)2 * 256 * kScaleAhead * 4      // scale and zero-point rings of the fold
+           + (size_t)x_stages(BM) * BM * 4           // sum of X per stage (asymmetric variant)
+           + 512;
 }
 
 template <int R, int BM>
@@ -150,6 +152,9 @@ struct GArgs {
     CUtensorMap xmap;           // X as (64 columns, M rows, K/64 halves), boxes 64 x BM x 2
     const uint32_t *planes;     // tiled planes
     const __half *scales;       // tiled fp16 scales
+    const __half *zeros;        // tiled fp16 zero points (asymmetric variant) or null
+    const float *sumx;          // [G][Mpad] sums of X over each group (asymmetric variant)
+    int Mpad;                   // MB * BM
     __nv_bfloat16 *Y;           // M x N
     float *part;                // partial sums of shared tiles [tile * maxc + slot][BM][128]
     unsigned *tickets;          // one per (X block, tile)
@@ -184,7 +189,10 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
     uint8_t *sX = smem;                                        // [kS][2 halves][BM][128 B]
     uint8_t *ring = sX + kS * C::kXStage;                      // [group][kD][plane][128 rows][16 B]
     uint32_t *sring = reinterpret_cast<uint32_t *>(ring + C::kGroups * kD * C::kSlot);  // [fold thread][kScaleAhead]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sring + kFoldW * 32 * kScaleAhead);
+    uint32_t *zring = sring + kFoldW * 32 * kScaleAhead;       // zero points, same shape
+    float *sx = reinterpret_cast<float *>(zring + kFoldW * 32 * kScaleAhead);   // [kS][BM] sums of X
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sx + kS * BM);
+    const bool asym = a.zeros != nullptr;                      // asymmetric variant (uniform)
     // afull: A stage decoded; xfull: X stage loaded; sempty: the stage's MMAs
     // done (A and X free, accumulator full); dempty: accumulator read
     uint64_t *afull = bars, *xfull = afull + kS, *sempty = xfull + kS, *dempty = sempty + kS;
@@ -302,10 +310,13 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
         // copies the 4 bytes holding its row's scale (rows n & ~1 and n | 1)
         // into its own slots (cp.async groups are per thread: no barrier)
         uint32_t *slots = sring + (threadIdx.x - kFoldW0 * 32) * kScaleAhead;
+        uint32_t *zslots = zring + (threadIdx.x - kFoldW0 * 32) * kScaleAhead;
         const uint16_t *sc = reinterpret_cast<const uint16_t *>(a.scales) + (n & ~1);
+        const uint16_t *zc = asym ? reinterpret_cast<const uint16_t *>(a.zeros) + (n & ~1) : nullptr;
         int next_tg = (int)(u0 % TG);                          // (tile, group) of the next scale copied
         auto scale_issue = [&](int i) {
             cp_async_4(slots + i % kScaleAhead, sc + (int64_t)next_tg * 128);
+            if (asym) cp_async_4(zslots + i % kScaleAhead, zc + (int64_t)next_tg * 128);
             if (++next_tg == TG) next_tg = 0;
         };
 #pragma unroll 1
@@ -319,9 +330,16 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
             cp_async_wait<kScaleAhead - 1>();                  // item i's scale is in
             const uint32_t sw = slots[i % kScaleAhead];
             const float s = __half2float(__ushort_as_half((unsigned short)((n & 1) ? sw >> 16 : sw & 0xFFFFu)));
+            float cz = 0.f;                                    // 128 - z (asymmetric variant)
+            if (asym) {
+                const uint32_t zw = zslots[i % kScaleAhead];
+                cz = 128.f - __half2float(__ushort_as_half((unsigned short)((n & 1) ? zw >> 16 : zw & 0xFFFFu)));
+            }
             if (i + kScaleAhead < L) scale_issue(i + kScaleAhead);
             cp_async_commit();
             if (ok) ok = MQ_GEMM_WAIT(sempty + db, (uint32_t)(i / kS) & 1u, flags);
+            // the stage's sums of X (asymmetric variant) land with its X tile
+            if (asym && ok) ok = MQ_GEMM_WAIT(xfull + db, (uint32_t)(i / kS) & 1u, flags);
             ok = __all_sync(0xFFFFFFFFu, ok);                  // tcgen05.ld is warp-wide
             if (ok) {
                 tc_fence_after();
@@ -330,8 +348,22 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
                     uint32_t v[16];
                     tmem_ld16(tmem + lane_base + kD0 + (uint32_t)(db * BM + c0 + cb), v);
                     tmem_ld_wait();
+                    if (asym) {
+                        // sum_k x w = s (D + (128 - z) sum_k x): the level
+                        // measured from z instead of 128
+                        const float4 *sxp = reinterpret_cast<const float4 *>(sx + db * BM + c0 + cb);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) y[cb + j] = fmaf(s, __uint_as_float(v[j]), y[cb + j]);
+                        for (int j4 = 0; j4 < 4; ++j4) {
+                            const float4 t = sxp[j4];
+                            y[cb + 4 * j4 + 0] = fmaf(s, fmaf(cz, t.x, __uint_as_float(v[4 * j4 + 0])), y[cb + 4 * j4 + 0]);
+                            y[cb + 4 * j4 + 1] = fmaf(s, fmaf(cz, t.y, __uint_as_float(v[4 * j4 + 1])), y[cb + 4 * j4 + 1]);
+                            y[cb + 4 * j4 + 2] = fmaf(s, fmaf(cz, t.z, __uint_as_float(v[4 * j4 + 2])), y[cb + 4 * j4 + 2]);
+                            y[cb + 4 * j4 + 3] = fmaf(s, fmaf(cz, t.w, __uint_as_float(v[4 * j4 + 3])), y[cb + 4 * j4 + 3]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) y[cb + j] = fmaf(s, __uint_as_float(v[j]), y[cb + j]);
+                    }
                 }
                 tc_fence_before();
             }
@@ -401,7 +433,10 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
             int mb = (int)(u0 / TG), g = (int)(u0 % G);        // X block and group of item i
             for (int i = 0; i < L; ++i) {
                 const int xs = i % kS, kx = i / kS;
-                if (kx > 0 && !mbar_wait_abortable(sempty + xs, (uint32_t)(kx - 1) & 1u, flags)) break;
+                // the stage is free once its MMAs are done; in the asymmetric
+                // variant its sums of X also once the fold has read them
+                if (kx > 0 && !mbar_wait_abortable(asym ? dempty + xs : sempty + xs, (uint32_t)(kx - 1) & 1u, flags))
+                    break;
 #ifdef MQ_TEST_HOOKS
                 if (i == 0 && atomicSub(&g_test_drop_x, 1) > 0) {  // item 0 never arrives
                     if (++g == G) {
@@ -411,8 +446,9 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
                     continue;
                 }
 #endif
-                mbar_expect_tx(xfull + xs, C::kXStage);
+                mbar_expect_tx(xfull + xs, C::kXStage + (asym ? BM * 4 : 0));
                 tma_load_3d(sX + xs * C::kXStage, &a.xmap, 0, mb * BM, 2 * g, xfull + xs);
+                if (asym) bulk_g2s(sx + xs * BM, a.sumx + (int64_t)g * a.Mpad + mb * BM, BM * 4, xfull + xs);
                 flags[3] = i + 1;
                 if (++g == G) {
                     g = 0;
@@ -535,7 +571,7 @@ gemm_tc_kernel(const __grid_constant__ GArgs a) {
 
 struct TcPlan {
     int BM, MB, T, G, P, maxc;
-    size_t part_off, ws_bytes;
+    size_t part_off, sumx_off, ws_bytes;
 };
 
 int tc_sm_count() {
@@ -570,8 +606,37 @@ TcPlan tc_plan(int64_t M, int64_t N, int64_t K, int sms) {
     p.maxc = maxc;
     p.part_off = kTicketBytes;
     const size_t part = (size_t)p.MB * p.T * p.maxc * p.BM * kTileN * sizeof(float);
-    p.ws_bytes = p.part_off + part;
+    p.sumx_off = p.part_off + part;                    // a multiple of 16 bytes
+    // sums of X per (group, X row) for the asymmetric variant
+    p.ws_bytes = p.sumx_off + (size_t)p.G * p.MB * p.BM * sizeof(float);
     return p;
+}
+
+// sumx[g][m] = sum over group g of X[m, k] (fp32), rows m in [M, Mpad) zero:
+// the factor of the zero-point term of the asymmetric variant.
+__global__ void __launch_bounds__(256)
+sumx_kernel(const uint16_t *__restrict__ X, int M, int64_t K, int Mpad, float *__restrict__ sumx) {
+    pdl_wait();                                        // X may come from the previous kernel
+    pdl_launch_dependents();
+    const int64_t G = K / kGroup;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < G * Mpad;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t g = i / Mpad;
+        const int m = (int)(i - g * Mpad);
+        float acc = 0.f;
+        if (m < M) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(X + (int64_t)m * K + g * kGroup);
+#pragma unroll 4
+            for (int c = 0; c < kGroup / 8; ++c) {
+                const uint4 v = __ldg(p + c);
+                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    acc += __uint_as_float(w[e] << 16) + __uint_as_float(w[e] & 0xFFFF0000u);
+            }
+        }
+        sumx[i] = acc;
+    }
 }
 
 // cuTensorMapEncodeTiled from the driver (looked up once, no -lcuda).
@@ -667,6 +732,9 @@ mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint
     if (!encode_x_map(&a.xmap, X, M, w->K, p.BM)) return fail(MQ_ERR_CUDA, "cuTensorMapEncodeTiled (X)");
     a.planes = w->planes;
     a.scales = reinterpret_cast<const __half *>(w->scales);
+    a.zeros = reinterpret_cast<const __half *>(w->zeros);
+    a.sumx = reinterpret_cast<const float *>(wsb + p.sumx_off);
+    a.Mpad = p.MB * p.BM;
     a.Y = reinterpret_cast<__nv_bfloat16 *>(Y);
     a.part = reinterpret_cast<float *>(wsb + p.part_off);
     a.tickets = reinterpret_cast<unsigned *>(wsb);
@@ -679,14 +747,27 @@ mq_status launch_gemm_tc(const uint16_t *X, const mq_weights *w, int64_t M, uint
     a.P = p.P;
     a.maxc = p.maxc;
     a.plane_words = (int64_t)p.T * kTileN * (w->K / 32);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    if (w->zeros) {
+        // the asymmetric variant's sums of X, written before the GEMM reads them
+        cudaLaunchConfig_t pc = {};
+        const int64_t cells = (int64_t)p.G * a.Mpad;
+        pc.gridDim = dim3((unsigned)((cells + 255) / 256 < 1184 ? (cells + 255) / 256 : 1184));
+        pc.blockDim = dim3(256);
+        pc.stream = st;
+        pc.attrs = attr;
+        pc.numAttrs = 1;
+        e = cudaLaunchKernelEx(&pc, sumx_kernel, X, (int)M, (int64_t)w->K, a.Mpad,
+                               reinterpret_cast<float *>(wsb + p.sumx_off));
+        if (e != cudaSuccess) return cuda_fail(e, "sumx_kernel");
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)p.P);
     cfg.blockDim = dim3((unsigned)threads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, fn, a);

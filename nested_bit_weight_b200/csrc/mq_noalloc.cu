@@ -42,7 +42,7 @@ extern "C" mq_status mq_gemv_noalloc(const uint16_t *X, const mq_weights *w, int
     // its X operand and its arrival tickets)
     cudaStream_t st = (cudaStream_t)stream;
     if ((s = bind_device(st)) != MQ_OK) return s;
-    const bool gemv = small_m_uses_gemv(M, N, K, w->r);
+    const bool gemv = !w->zeros && small_m_uses_gemv(M, N, K, w->r);
     const size_t need = gemv ? gemv_tc_workspace_bytes(M, N, K, w->r)
                              : gemm_tc_workspace_bytes(M, N, K, w->r);
     if (need > kNoAllocBytes)

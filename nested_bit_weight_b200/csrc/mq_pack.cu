@@ -47,14 +47,17 @@ pack_kernel(const uint8_t *__restrict__ codes, int64_t N, int64_t K,
     }
 }
 
+// fp32 [N, G] -> fp16 RNE in the tiled block order; `signed_ok` admits
+// negative values (zero points) and refuses only NaN and fp16 overflow.
 __global__ void __launch_bounds__(256)
-scales_kernel(const float *__restrict__ s, int64_t N, int64_t G, __half *__restrict__ out) {
+scales_kernel(const float *__restrict__ s, int64_t N, int64_t G, __half *__restrict__ out,
+              bool signed_ok) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < N * G;
          i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t n = i / G, g = i - n * G;
         const float v = s[i];
         const __half h = __float2half_rn(v);
-        if (!(v >= 0.0f) || __hisinf(h)) atomicOr(&g_pack_bad, 1u);
+        if (!(signed_ok ? v == v : v >= 0.0f) || __hisinf(h)) atomicOr(&g_pack_bad, 1u);
         out[((n / 128) * G + g) * 128 + n % 128] = h;
     }
 }
@@ -128,7 +131,7 @@ extern "C" mq_status mq_pack(const uint8_t *codes, const float *scales, int64_t 
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "pack_kernel");
     const int64_t ns = N * (K / kGroup);
     scales_kernel<<<grid_for(ns, 256), 256, 0, st>>>(scales, N, K / kGroup,
-                                                     reinterpret_cast<__half *>(scales_out));
+                                                     reinterpret_cast<__half *>(scales_out), false);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "scales_kernel");
     unsigned bad = 0;
     e = cudaMemcpyFromSymbolAsync(&bad, g_pack_bad, sizeof(bad), 0,
@@ -137,6 +140,35 @@ extern "C" mq_status mq_pack(const uint8_t *codes, const float *scales, int64_t 
     if (e != cudaSuccess) return cuda_fail(e, "mq_pack");
     if (bad) return fail(MQ_ERR_UNSUPPORTED,
                          "a scale is negative, NaN, or overflows fp16");
+    return MQ_OK;
+}
+
+extern "C" mq_status mq_pack_zeros(const float *zeros, int64_t N, int64_t K, int group,
+                                   uint16_t *zeros_out, void *stream) {
+    if (!zeros || !zeros_out) return fail(MQ_ERR_INVALID_ARG, "NULL pointer passed to mq_pack_zeros");
+    if (N < 1 || K < kGroup || K % kGroup)
+        return fail(MQ_ERR_INVALID_ARG, "need N >= 1 and K a positive multiple of 128");
+    if (group != kGroup) return fail(MQ_ERR_INVALID_ARG, "group must be 128");
+    if (!aligned16(zeros) || !aligned16(zeros_out))
+        return fail(MQ_ERR_MISALIGNED, "mq_pack_zeros pointers must be 16-byte aligned");
+    cudaStream_t st = (cudaStream_t)stream;
+    mq_status bs = bind_device(st);
+    if (bs != MQ_OK) return bs;
+    const unsigned zero = 0;
+    cudaError_t e = cudaMemcpyToSymbolAsync(g_pack_bad, &zero, sizeof(zero), 0,
+                                            cudaMemcpyHostToDevice, st);
+    if (e != cudaSuccess) return cuda_fail(e, "mq_pack_zeros reset");
+    if (N % 128 && (e = cudaMemsetAsync(zeros_out, 0, mq_scale_bytes(N, K, kGroup), st)) != cudaSuccess)
+        return cuda_fail(e, "mq_pack_zeros padding");
+    const int64_t ns = N * (K / kGroup);
+    scales_kernel<<<grid_for(ns, 256), 256, 0, st>>>(zeros, N, K / kGroup,
+                                                     reinterpret_cast<__half *>(zeros_out), true);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "scales_kernel (zeros)");
+    unsigned bad = 0;
+    e = cudaMemcpyFromSymbolAsync(&bad, g_pack_bad, sizeof(bad), 0, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "mq_pack_zeros");
+    if (bad) return fail(MQ_ERR_UNSUPPORTED, "a zero point is NaN or overflows fp16");
     return MQ_OK;
 }
 

@@ -157,3 +157,15 @@ def test_chain_argument_errors_before_launch():
     assert mq.mq_gemm_workspace_bytes(16, 64, 256, 4) > 0
     assert mq.lib.mq_gemm_chain(arr(ok_call), 1, None, 0, None) == 6
     assert mq.lib.mq_gemm_chain(arr(ok_call), 1, FAKE * 8, 1024, None) == 6
+
+
+def test_pack_zeros_argument_errors():
+    f = mq.lib.mq_pack_zeros
+    assert f(None, 4, 256, 128, FAKE, None) == 1
+    assert f(FAKE, 4, 100, 128, FAKE, None) == 1          # K not a multiple of 128
+    assert f(FAKE, 4, 256, 64, FAKE, None) == 1           # group
+    assert f(FAKE + 4, 4, 256, 128, FAKE, None) == 3      # misaligned
+    # a view with a misaligned zero-point pointer is refused before any launch
+    w = mq.MqWeights(FAKE, FAKE * 2, 64, 256, 128, 4, FAKE + 8)
+    out = mq.MqWeights()
+    assert mq.lib.mq_slice(ctypes.byref(w), 4, ctypes.byref(out)) == 3

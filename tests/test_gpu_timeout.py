@@ -25,7 +25,8 @@ MQ_ERR_TIMEOUT = 5
 
 class _W(ctypes.Structure):
     _fields_ = [("planes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("N", ctypes.c_int64),
-                ("K", ctypes.c_int64), ("group", ctypes.c_int32), ("r", ctypes.c_int32)]
+                ("K", ctypes.c_int64), ("group", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("zeros", ctypes.c_void_p)]
 
 
 def _hooks_lib():
