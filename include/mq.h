@@ -201,6 +201,32 @@ typedef struct mq_call {
 MQ_API mq_status mq_gemm_chain(const mq_call *calls, int n, void *workspace,
                                size_t workspace_bytes, void *stream);
 
+/* One candidate bit width of one layer for mq_bitwidth_search. */
+typedef struct mq_choice {
+    int32_t r;              /* bit width (informational; returned through the index) */
+    uint64_t bytes;         /* storage the layer costs at this width (e.g. mq_plane_bytes) */
+    double error;           /* the layer's error at this width (e.g. its output error
+                               against the parent on calibration inputs), >= 0 */
+} mq_choice;
+
+/*
+ * Budget-aware per-layer bit-width search (MatGPTQ author page, abstract:
+ * "budget-aware search for heterogeneous per-layer bit-widths"): choose one
+ * candidate per layer so that the summed bytes stay within budget_bytes and
+ * the summed error is least (a multiple-choice knapsack, solved exactly by
+ * dynamic programming over the bytes in units of their greatest common
+ * divisor).  Host only, no device work.
+ *   choices     n_layers x n_choices candidates, layer-major
+ *   choice_out  n_layers indices into each layer's candidates
+ *   error_out   the summed error of the choice (may be NULL)
+ * Ties: least error, then fewest bytes, then the lowest candidate indices.
+ * Returns MQ_ERR_INVALID_ARG for bad sizes or a negative / non-finite error,
+ * MQ_ERR_UNSUPPORTED when no choice fits the budget or the dynamic program
+ * would need more than 2^26 (layer, budget unit) cells.
+ */
+MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int n_choices,
+                                    uint64_t budget_bytes, int *choice_out, double *error_out);
+
 /* Kernels for M <= 8 (both compute the same Y within the stated tolerance). */
 enum {
     MQ_GEMV_TC = 0,        /* default: 128 rows per tensor-core MMA, int8 operands,

@@ -19,6 +19,7 @@ __all__ = [
     "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
     "mq_device_status", "mq_gemm_kernel", "uses_gemv", "KERNEL_GEMV", "KERNEL_GEMM",
     "MqCall", "mq_gemm_chain", "gemm_chain", "pack_fused", "workspace_for", "mq_pack_zeros",
+    "MqChoice", "bitwidth_search", "layer_errors",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -42,6 +43,11 @@ class MqWeights(ctypes.Structure):
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64),
                 ("group", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("zeros", ctypes.c_void_p)]                # fp16 zero points or None (symmetric)
+
+
+class MqChoice(ctypes.Structure):
+    """One candidate of mq_bitwidth_search (mq_choice in include/mq.h)."""
+    _fields_ = [("r", ctypes.c_int32), ("bytes", ctypes.c_uint64), ("error", ctypes.c_double)]
 
 
 class MqCall(ctypes.Structure):
@@ -76,6 +82,8 @@ def _load() -> ctypes.CDLL:
         "mq_gemm_kernel": (I, [I64, I64, I64, I]),
         "mq_gemm_chain": (I, [ctypes.POINTER(MqCall), I, P, SZ, P]),
         "mq_pack_zeros": (I, [P, I64, I64, I, P, P]),
+        "mq_bitwidth_search": (I, [ctypes.POINTER(MqChoice), I, I, ctypes.c_uint64,
+                                   ctypes.POINTER(I), ctypes.POINTER(ctypes.c_double)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -265,6 +273,37 @@ def gemm_chain(calls, stream=None):
     ws = workspace_for(calls[0][0].device, need) if need else None
     mq_gemm_chain(views, ws, stream)
     return outs
+
+
+def bitwidth_search(table, budget_bytes: int):
+    """table[l] = [(r, bytes, error), ...] per layer -> (index chosen per
+    layer, summed error): the least summed error within the byte budget
+    (mq_bitwidth_search; exact)."""
+    L, C = len(table), len(table[0])
+    arr = (MqChoice * (L * C))()
+    for l, row in enumerate(table):
+        if len(row) != C:
+            raise ValueError("every layer needs the same number of candidates")
+        for j, (r, nbytes, err) in enumerate(row):
+            arr[l * C + j] = MqChoice(r, nbytes, err)
+    out = (ctypes.c_int * L)()
+    total = ctypes.c_double()
+    _check(lib.mq_bitwidth_search(arr, L, C, budget_bytes, out, ctypes.byref(total)))
+    return list(out), total.value
+
+
+def layer_errors(X, weights: NestedWeights, rs, stream=None):
+    """{r: ||X W_r^T - X W_8^T||^2 / ||X W_8^T||^2} for one layer, the outputs
+    computed by mq_gemm and reduced on the host in fp64 (the sensitivities a
+    bit-width search consumes)."""
+    import numpy as np
+    ref = gemm(X, weights, 8, stream=stream).float().cpu().numpy().astype(np.float64)
+    den = float(np.sum(ref * ref))
+    out = {}
+    for r in rs:
+        y = gemm(X, weights, r, stream=stream).float().cpu().numpy().astype(np.float64)
+        out[r] = float(np.sum((y - ref) ** 2)) / den
+    return out
 
 
 _ws_cache: dict = {}

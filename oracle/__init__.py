@@ -246,3 +246,32 @@ def violation_ratio(Y, Yref, rms: float | None = None) -> float:
     with np.errstate(divide="ignore", invalid="ignore"):
         ratio = np.where(tol > 0, err / tol, np.where(err > 0, np.inf, 0.0))
     return float(ratio.max())
+
+
+# ------------------------------------------------ per-layer bit-width search
+
+def bitwidth_search_exhaustive(errors, nbytes, budget):
+    """Every assignment of one candidate per layer (MatGPTQ author page,
+    abstract: budget-aware search for heterogeneous per-layer bit-widths):
+    returns (least summed error within the budget, its bytes, every optimal
+    assignment at that error and byte count), or None if nothing fits.  The
+    summed error is accumulated in layer order; assignments are compared by
+    (error, bytes).  Small instances only."""
+    import itertools
+    L = len(errors)
+    best = None
+    for pick in itertools.product(*[range(len(row)) for row in errors]):
+        b = sum(nbytes[l][pick[l]] for l in range(L))
+        if b > budget:
+            continue
+        e = 0.0
+        for l in range(L):
+            e += errors[l][pick[l]]
+        key = (e, b)
+        if best is None or key < best[0]:
+            best = (key, [pick])
+        elif key == best[0]:
+            best[1].append(pick)
+    if best is None:
+        return None
+    return best[0][0], best[0][1], best[1]
