@@ -141,9 +141,11 @@ def test_deterministic_and_workspace_reusable():
 @pytest.mark.parametrize("N,K,M,r", [(2048, 14336, 1, 4), (2048, 14336, 8, 8), (2048, 14336, 8, 2),
                                       (1024, 14336, 4, 3), (2000, 8192, 8, 6), (300, 28672, 3, 5)])
 def test_gemv_stage_ring_and_k_segments(N, K, M, r):
-    # more items per CTA than shared-memory stages (the ring wraps), and X
-    # operands too large for one CTA (K cut into segments, so every tile is
-    # combined across CTAs through the workspace); twice, bit-identical
+    # more items per CTA than shared-memory stages (the ring wraps), and long
+    # K (row tiles whose groups are split between CTAs: the GEMV sums them in
+    # a cluster through distributed shared memory, the GEMM through the
+    # workspace, both in a fixed order); twice, bit-identical (some of these
+    # shapes and batches take the GEMM under the small-batch dispatch)
     import torch
     import nested_bit_weight_b200 as mq
     codes, s, _ = wl.gen_weights(N, K, seed=N + K + M + r)
@@ -232,3 +234,31 @@ def test_qwen_chain_outlier_x(name, N, K, M):
     xbits, X = wl.gen_x(M, K, wl.layer_seed(3, 0) + M, outlier_channels=True)
     Y, _ = _run(codes, s, xbits, r)
     assert oracle.violation_ratio(Y, oracle.gemm(X, codes, s, r)) <= 1.0
+
+
+@pytest.mark.parametrize("M", [1, 3, 16])
+def test_weights_written_by_the_previous_kernel(M):
+    # stream order (programmatic dependent launch): a torch kernel writes the
+    # weights and mq_gemm follows at once on the same stream, no sync; torch's
+    # kernels do not let dependents start early, so the early weight reads of
+    # the GEMV and the GEMM see the new weights (the contract in mq.h)
+    import torch
+    import nested_bit_weight_b200 as mq
+    N, K = 2048, 4096
+    ca, sa, _ = wl.gen_weights(N, K, seed=501)
+    cb, sb, _ = wl.gen_weights(N, K, seed=502)
+    A = mq.pack_parent(torch.from_numpy(ca).cuda(), torch.from_numpy(sa).cuda())
+    B = mq.pack_parent(torch.from_numpy(cb).cuda(), torch.from_numpy(sb).cuda())
+    xbits, X = wl.gen_x(M, K, seed=503)
+    Xd = torch.from_numpy(xbits.view(np.int16)).cuda().view(torch.bfloat16)
+    ref_a, ref_b = oracle.gemm(X, ca, sa, 4), oracle.gemm(X, cb, sb, 4)
+    planes_a, scales_a = A.planes.clone(), A.scales16.clone()
+    outs = []
+    for src_p, src_s in ((B.planes, B.scales16), (planes_a, scales_a), (B.planes, B.scales16)):
+        A.planes.copy_(src_p)
+        A.scales16.copy_(src_s)
+        outs.append(mq.gemm(Xd, A, 4))            # no synchronisation in between
+    got = [o.float().cpu().numpy().astype(np.float64) for o in outs]
+    assert oracle.violation_ratio(got[0], ref_b) <= 1.0
+    assert oracle.violation_ratio(got[1], ref_a) <= 1.0
+    assert oracle.violation_ratio(got[2], ref_b) <= 1.0
