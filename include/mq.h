@@ -79,10 +79,21 @@ typedef struct {
                                  or NULL for the symmetric format (the zero point 128) */
 } mq_weights;
 
-/* Bytes of the first r planes: r * N128 * K / 8 (0 on invalid arguments). */
+/*
+ * Bytes of the first r planes: r * N128 * K / 8 (0 on invalid arguments),
+ * N128 = N rounded up to a multiple of 128.  An r-bit model reads exactly r
+ * bits per weight ("MatGPTQ: Efficient and Accurate Inference over Nested
+ * Quantized Models", abstract, and Table 1, "Exact r-bit loading"): these are
+ * the bytes one mq_gemm call at width r streams for its planes.
+ */
 MQ_API size_t mq_plane_bytes(int64_t N, int64_t K, int r);
 
-/* Bytes of the stored fp16 scales: 2 * N128 * (K / group) (0 on invalid arguments). */
+/*
+ * Bytes of the stored fp16 scales: 2 * N128 * (K / group) (0 on invalid
+ * arguments); one scale per row and 128-column group, shared by every r of
+ * the nested model (the single multi-precision checkpoint of the MatGPTQ
+ * abstract).  The zero points of the asymmetric variant take the same size.
+ */
 MQ_API size_t mq_scale_bytes(int64_t N, int64_t K, int group);
 
 /*
@@ -264,7 +275,10 @@ MQ_API int mq_gemm_kernel(int64_t M, int64_t N, int64_t K, int r);
 
 /*
  * Test helper: codes_out[n, k] = q_r[n, k] read back from the first r planes
- * (uint8 N x K row-major, device).  Same preconditions as mq_gemm on `w`.
+ * (uint8 N x K row-major, device): the r-bit model as the top r bits of the
+ * parent code ("MatGPTQ: Accurate and Efficient Post-Training Matryoshka
+ * Quantization", author-page abstract: the most significant bits are sliced
+ * at inference time).  Same preconditions as mq_gemm on `w`.
  */
 MQ_API mq_status mq_unpack(const mq_weights *w, uint8_t *codes_out, void *stream);
 

@@ -113,8 +113,15 @@ static void check_split(int64_t M, int64_t N, int64_t K, int sms) {
     }
     ++checked;
     if (prev != W) { ++bad; printf("ranges end at %ld, W=%ld\n", (long)prev, (long)W); }
+    // the regions of the workspace: tickets, partial sums, sums of X
+    ++checked;
+    if (p.part_off < kTicketBytes || p.sumx_off < p.part_off || p.sumx_off % 16 ||
+        p.sumx_off + (size_t)p.G * p.MB * p.BM * sizeof(float) > p.ws_bytes) {
+        ++bad;
+        printf("workspace regions M=%ld N=%ld K=%ld\n", (long)M, (long)N, (long)K);
+    }
     // tiles shared between CTAs: slots, partial-sum bounds
-    const size_t part_elems = (p.ws_bytes - p.part_off) / sizeof(float);
+    const size_t part_elems = (p.sumx_off - p.part_off) / sizeof(float);
     for (int64_t tu = 0; tu < (int64_t)p.MB * p.T; ++tu) {
         const int cf = cta_of(tu * p.G, W, p.P), cl = cta_of(tu * p.G + p.G - 1, W, p.P);
         const int cnt = cl - cf + 1;
