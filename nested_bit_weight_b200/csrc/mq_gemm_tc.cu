@@ -1,5 +1,6 @@
-// Batched path (M >= 9, and the M <= 8 fallback): tcgen05 tensor-core GEMM
-// over decoded r-bit tiles.
+// Batched path: tcgen05 tensor-core GEMM over decoded r-bit tiles (M >= 9,
+// the small batches the dispatch gives it, and asymmetric weights for every
+// M).
 //
 // The r-bit levels v_r = 2^(8-r) q_r + 2^(7-r) - 128 are exact in bf16 (at
 // most 8 significant bits), so the MMA operands are exact:
@@ -7,38 +8,45 @@
 //     Y[m, n]   = sum_g s[n, g] * D_g[n, m]                  (fp32 registers)
 // (the fp16 scale is applied per 128-column group in fp32: folding s * v
 // into one 16-bit operand rounds every weight, which the tolerance does not
-// allow on large layers).
+// allow on large layers).  Asymmetric variant (a zero point z per group):
+//     Y[m, n]   = sum_g s[n, g] * (D_g[n, m] + (128 - z[n, g]) * sum_{k in g} x[m, k])
+// with the sums of X written by a small kernel before the GEMM.
 //
 // Work: items (X block mb, 128-row tile t, group g) in that order, cut into
 // one contiguous range per CTA (about 148 CTAs, one per SM).  A tile whose
-// groups are spread over several CTAs is summed by the CTA that finishes it
-// last, from the fp32 partial sums the others leave in the workspace, in
-// CTA order (deterministic).
+// groups are spread over several CTAs is summed by the CTA that delivers its
+// last part, from the fp32 partial sums the others leave in the workspace,
+// in CTA order (deterministic), with all its threads after its own range.
 //
-// Roles (warp-specialised; every hand-off an mbarrier):
-//   decode warps    8 (two threads per weight row) or 4 (BM = 128): each
-//                   thread copies its share of the row's r plane words of the
-//                   items ahead into a ring of shared memory with cp.async
-//                   (up to 16 items, up to 96 KB in flight per SM), then
-//                   decodes the current group to bf16 levels in natural column
-//                   order and stores them to its TMEM lane in one of two A
-//                   stages (tcgen05.st; the MMA reads A from TMEM);
-//   X warp          one thread loads the group's BM x 128 block of X into one
-//                   of 2 or 4 B stages with one tensor-map (TMA) copy, in the
-//                   same layout; rows beyond M read as zeros;
-//   MMA warp        one thread issues eight 128 x BM x 16 MMAs per group into
-//                   the stage's TMEM accumulator and commits once: the
-//                   stage's A and B operands are free, its accumulator full;
+// Roles (warp-specialised; every hand-off an mbarrier; item i uses stage
+// i mod kS of the A operand, the X operand and the accumulator):
+//   decode warps    two groups of four taking alternate items (one group for
+//                   BM = 128); a thread per weight row copies exactly its
+//                   row's 16 bytes of each plane of the items ahead with
+//                   L1-bypassing cp.async (up to 16 items, 96 KB per SM in
+//                   flight), decodes each 32-column word to bf16 levels in
+//                   natural column order and stores them to its TMEM lane of
+//                   the A stage (tcgen05.st; the MMA reads A from TMEM);
+//   X warp          one thread loads the group's BM x 128 block of X into
+//                   the B stage with one 3-D tensor-map (TMA) copy in the
+//                   MMA's K-major layout; rows beyond M read as zeros;
+//   two MMA warps   one thread each (even / odd items) issues eight
+//                   128 x BM x 16 MMAs per group into the stage's TMEM
+//                   accumulator and commits once: the stage's A and B
+//                   operands are free, its accumulator full;
 //   fold warps      4 (BM <= 64) or 8 (BM = 128), one or two per TMEM lane
 //                   quarter: y += s[n, g] * D_g, the tile's fp32 sums kept in
-//                   registers until the tile ends.
+//                   registers until the tile ends; the scales (and zero
+//                   points) arrive by per-thread cp.async eight items ahead.
 // Launched with programmatic dependent launch: the decode warps stream the
 // weights before the previous kernel of the stream has completed; X is read
 // and Y and the workspace written only after griddepcontrol.wait.
 // Every wait is bounded (about a second); a wait that gives up sets a CTA
 // abort flag that ends the others at once, and a device flag read by
-// mq_device_status.  Arrival tickets always return to zero, also after a
-// timeout (the output is then unspecified).
+// mq_device_status.  The fold still runs every tile end, so arrival tickets
+// always return to zero, also after a timeout (the output is then
+// unspecified); copies, MMAs and barrier arrivals in flight land before the
+// CTA exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
