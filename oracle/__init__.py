@@ -275,3 +275,79 @@ def bitwidth_search_exhaustive(errors, nbytes, budget):
     if best is None:
         return None
     return best[0][0], best[0][1], best[1]
+
+
+# ------------------------------------------- one-shot multi-precision quantizer
+# "MatGPTQ: Efficient and Accurate Inference over Nested Quantized Models"
+# (abstract: a multi-precision objective with bit-slicing and cross-bit error
+# compensation; Tables 6-7: the lambda weighting of the bit widths) on top of
+# GPTQ's column loop.  The pages give prose only; the readings taken:
+#   * U = the upper Cholesky factor of (H + damp * mean(diag H) * I)^-1;
+#   * per 128-column group, when its first column is reached, the scale of a
+#     row is s = alpha * max|w| / 127.5 over the group's current weights,
+#     alpha searched over a small grid for the least lambda-weighted error of
+#     the group (the scale search);
+#   * each weight's 8-bit code minimises sum_r lambda_r (w - s v_r(q_r))^2 over
+#     the nested levels of every r (ties: the smallest code);
+#   * the error carried to the later columns is the lambda-weighted mean of
+#     the slice errors: w_k+1.. -= e / U[k, k] * U[k, k+1..].
+
+def matgptq_prepare(H: np.ndarray, damp: float = 0.01) -> np.ndarray:
+    """U upper triangular with U^T U = (H + damp * mean(diag H) * I)^-1."""
+    H = np.asarray(H, np.float64)
+    K = H.shape[0]
+    Hd = H + damp * float(np.mean(np.diag(H))) * np.eye(K)
+    return np.linalg.cholesky(np.linalg.inv(Hd)).T
+
+
+def _level_all(r: int) -> np.ndarray:
+    """The r-bit level of every 8-bit code 0..255 (v_r of its top r bits)."""
+    return level(np.arange(256) >> (8 - r), r)
+
+
+def matgptq_best_code(w: float, s: float, rs, lams) -> int:
+    """argmin over q in 0..255 of sum_r lambda_r (w - s v_r(q >> (8-r)))^2."""
+    cost = np.zeros(256)
+    for r, lam in zip(rs, lams):
+        d = w - s * _level_all(r)
+        cost += lam * d * d
+    return int(np.argmin(cost))
+
+
+def matgptq_quantize(W, U, rs=(3, 4, 8), lams=(1.0, 1.0, 1.0),
+                     alphas=(1.0, 0.95, 0.9, 0.85, 0.8)):
+    """codes uint8 [N, K], scales fp64 [N, K/128] by the column loop above."""
+    W = np.array(W, np.float64, copy=True)
+    U = np.asarray(U, np.float64)
+    N, K = W.shape
+    G = K // 128
+    lsum = float(sum(lams))
+    codes = np.zeros((N, K), np.uint8)
+    scales = np.zeros((N, G), np.float64)
+    for g in range(G):
+        cols = range(128 * g, 128 * g + 128)
+        for n in range(N):
+            base = float(np.max(np.abs(W[n, 128 * g:128 * g + 128]))) / 127.5
+            best_a, best_t = None, None
+            for a in alphas:
+                s = base * a
+                t = 0.0
+                for k in cols:
+                    q = matgptq_best_code(W[n, k], s, rs, lams)
+                    for r, lam in zip(rs, lams):
+                        d = W[n, k] - s * float(level(np.array(q >> (8 - r)), r))
+                        t += lam * d * d
+                if best_t is None or t < best_t:
+                    best_a, best_t = a, t
+            scales[n, g] = base * best_a
+        for k in cols:
+            for n in range(N):
+                s = scales[n, g]
+                q = matgptq_best_code(W[n, k], s, rs, lams)
+                codes[n, k] = q
+                e = 0.0
+                for r, lam in zip(rs, lams):
+                    e += lam * (W[n, k] - s * float(level(np.array(q >> (8 - r)), r)))
+                e /= lsum
+                W[n, k + 1:] -= (e / U[k, k]) * U[k, k + 1:]
+    return codes, scales
