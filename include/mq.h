@@ -238,6 +238,36 @@ typedef struct mq_choice {
 MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int n_choices,
                                     uint64_t budget_bytes, int *choice_out, double *error_out);
 
+/*
+ * One-shot multi-precision quantizer (host, offline): the parent codes and
+ * scales of the nested format from float weights W (N x K, row-major) and a
+ * layer's Hessian proxy H (K x K, e.g. X^T X of calibration inputs), by
+ * GPTQ's column loop with MatGPTQ's multi-precision objective ("MatGPTQ:
+ * Efficient and Accurate Inference over Nested Quantized Models", abstract:
+ * bit-slicing and cross-bit error compensation; Tables 6-7: the lambda
+ * weighting of the widths).  All pointers are host memory.
+ *   mq_matgptq_prepare: U_out (K x K) upper triangular with
+ *     U^T U = (H + damp * mean(diag H) * I)^-1.
+ *   mq_matgptq_quantize: per 128-column group, when its first column is
+ *     reached, a row's scale is alpha * max|w| / 127.5 over the group's
+ *     current weights (alpha from `alphas`, the least lambda-weighted group
+ *     error; ties: the first); each code minimises
+ *     sum_i lambdas[i] (w - s v_rs[i](q))^2 over the nested levels (ties: the
+ *     smallest code); the lambda-weighted mean of the slice errors e is
+ *     carried to the later columns of the row, w_j -= e / U[k][k] * U[k][j].
+ *     codes_out N x K uint8, scales_out N x (K/128) fp32 (inputs of mq_pack).
+ *     threads <= 0: one per hardware thread.  fp64 in a fixed order, so the
+ *     result does not depend on the thread count.
+ * Errors: MQ_ERR_INVALID_ARG for bad sizes, widths, lambdas (all zero, or
+ * negative) or alphas, or a zero on U's diagonal; MQ_ERR_UNSUPPORTED when the
+ * damped Hessian is not positive definite.
+ */
+MQ_API mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp, double *U_out);
+MQ_API mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const double *U,
+                                     const int32_t *rs, const double *lambdas, int n_r,
+                                     const double *alphas, int n_alpha, int threads,
+                                     uint8_t *codes_out, float *scales_out);
+
 /* Kernels for M <= 8 (both compute the same Y within the stated tolerance). */
 enum {
     MQ_GEMV_TC = 0,        /* default: 128 rows per tensor-core MMA, int8 operands,

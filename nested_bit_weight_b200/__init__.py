@@ -19,7 +19,7 @@ __all__ = [
     "mq_set_gemv_variant", "mq_get_gemv_variant", "GEMV_TC", "GEMV_VIA_GEMM",
     "mq_device_status", "mq_gemm_kernel", "uses_gemv", "KERNEL_GEMV", "KERNEL_GEMM",
     "MqCall", "mq_gemm_chain", "gemm_chain", "pack_fused", "workspace_for", "mq_pack_zeros",
-    "MqChoice", "bitwidth_search", "layer_errors",
+    "MqChoice", "bitwidth_search", "layer_errors", "matgptq_prepare", "matgptq_quantize",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -84,6 +84,8 @@ def _load() -> ctypes.CDLL:
         "mq_pack_zeros": (I, [P, I64, I64, I, P, P]),
         "mq_bitwidth_search": (I, [ctypes.POINTER(MqChoice), I, I, ctypes.c_uint64,
                                    ctypes.POINTER(I), ctypes.POINTER(ctypes.c_double)]),
+        "mq_matgptq_prepare": (I, [P, I64, ctypes.c_double, P]),
+        "mq_matgptq_quantize": (I, [P, I64, I64, P, P, P, I, P, I, I, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -290,6 +292,43 @@ def bitwidth_search(table, budget_bytes: int):
     total = ctypes.c_double()
     _check(lib.mq_bitwidth_search(arr, L, C, budget_bytes, out, ctypes.byref(total)))
     return list(out), total.value
+
+
+def matgptq_prepare(H, damp: float = 0.01):
+    """U (K x K, fp64, upper) with U^T U = (H + damp * mean(diag H) * I)^-1
+    (mq_matgptq_prepare, host)."""
+    import numpy as np
+    H = np.ascontiguousarray(H, np.float64)
+    if H.ndim != 2 or H.shape[0] != H.shape[1]:
+        raise ValueError("H must be a square matrix")
+    K = H.shape[0]
+    U = np.empty((K, K), np.float64)
+    _check(lib.mq_matgptq_prepare(H.ctypes.data, K, float(damp), U.ctypes.data))
+    return U
+
+
+def matgptq_quantize(W, U, rs=(3, 4, 8), lambdas=(1.0, 1.0, 1.0),
+                     alphas=(1.0, 0.95, 0.9, 0.85, 0.8), threads: int = 0):
+    """(codes uint8 N x K, scales fp32 N x K/128): the parent codes of the
+    nested format from float weights W by the multi-precision column loop
+    (mq_matgptq_quantize, host; the inputs of pack_parent)."""
+    import numpy as np
+    W = np.ascontiguousarray(W, np.float32)
+    U = np.ascontiguousarray(U, np.float64)
+    if W.ndim != 2 or U.shape != (W.shape[1], W.shape[1]):
+        raise ValueError("need W of N x K and U of K x K")
+    if len(rs) != len(lambdas):
+        raise ValueError("one lambda per bit width")
+    N, K = W.shape
+    rs_a = np.ascontiguousarray(rs, np.int32)
+    lam_a = np.ascontiguousarray(lambdas, np.float64)
+    al_a = np.ascontiguousarray(alphas, np.float64)
+    codes = np.empty((N, K), np.uint8)
+    scales = np.empty((N, max(K // 128, 1)), np.float32)
+    _check(lib.mq_matgptq_quantize(W.ctypes.data, N, K, U.ctypes.data, rs_a.ctypes.data,
+                                   lam_a.ctypes.data, len(rs_a), al_a.ctypes.data, len(al_a),
+                                   int(threads), codes.ctypes.data, scales.ctypes.data))
+    return codes, scales
 
 
 def layer_errors(X, weights: NestedWeights, rs, stream=None):

@@ -17,13 +17,14 @@ OBJ = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmq.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden",
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2,-fvisibility=hidden,-ffp-contract=off",
          "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include")]
 
 
 def _headers_mtime() -> float:
+    # this script too: a change of its flags rebuilds every object
     hs = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(ROOT, "include", "*.h"))
-    return max([os.path.getmtime(h) for h in hs] + [0.0])
+    return max([os.path.getmtime(h) for h in hs] + [os.path.getmtime(os.path.abspath(__file__))])
 
 
 def _compile(src: str, hdr_mtime: float, verbose: bool, obj_dir: str = OBJ, extra=()) -> str:

@@ -1,0 +1,106 @@
+"""The library's one-shot multi-precision quantizer (host) against the
+oracle: given the same U, the codes and the scales must be identical (both
+sides take every decision in fp64 in the same order), the prepare step must
+agree with the oracle's within rounding, and bad arguments must be refused."""
+import numpy as np
+import pytest
+
+import oracle
+import nested_bit_weight_b200 as mq
+
+
+def _H(K, seed, corr=0.9):
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((4 * K, K))
+    X = z.copy()
+    for k in range(1, K):                       # AR(1) columns: correlated inputs
+        X[:, k] = corr * X[:, k - 1] + np.sqrt(1 - corr * corr) * z[:, k]
+    return X.T @ X / X.shape[0]
+
+
+def _W(N, K, seed):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((N, K)) * 0.02
+    W[:, rng.integers(K, size=3)] *= 8.0        # a few outlier columns
+    return W.astype(np.float32)
+
+
+@pytest.mark.parametrize("rs,lams,alphas", [
+    ((3, 4, 8), (1.0, 1.0, 1.0), (1.0, 0.95, 0.9, 0.85, 0.8)),
+    ((2, 4, 6, 8), (4.0, 2.0, 1.0, 1.0), (1.0, 0.9, 0.8)),
+    ((8,), (1.0,), (1.0,)),
+    ((1, 3), (1.0, 0.5), (1.0, 0.7)),
+])
+def test_codes_and_scales_identical_to_the_oracle(rs, lams, alphas):
+    N, K = 5, 256
+    U = oracle.matgptq_prepare(_H(K, 11))
+    W = _W(N, K, 12)
+    c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U, rs=rs, lams=lams, alphas=alphas)
+    codes, scales = mq.matgptq_quantize(W, U, rs=rs, lambdas=lams, alphas=alphas)
+    assert codes.shape == (N, K) and scales.shape == (N, K // 128)
+    assert np.array_equal(codes, c_ref)
+    assert np.array_equal(scales, s_ref.astype(np.float32))
+
+
+def test_thread_count_does_not_change_the_result():
+    N, K = 9, 384
+    U = oracle.matgptq_prepare(_H(K, 21))
+    W = _W(N, K, 22)
+    a = mq.matgptq_quantize(W, U, threads=1)
+    for t in (2, 4, 0, 64):
+        b = mq.matgptq_quantize(W, U, threads=t)
+        assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("K", [1, 7, 128, 300])
+def test_prepare_agrees_with_the_oracle(K):
+    H = _H(K, 31 + K)
+    U = mq.matgptq_prepare(H, damp=0.01)
+    ref = oracle.matgptq_prepare(H, damp=0.01)
+    assert np.array_equal(U, np.triu(U))
+    assert np.allclose(U, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(K)
+    assert np.allclose(U.T @ U @ Hd, np.eye(K), atol=1e-8)
+
+
+def test_prepare_then_quantize_is_the_oracle_pipeline():
+    N, K = 4, 256
+    H = _H(K, 41)
+    W = _W(N, K, 42)
+    codes, scales = mq.matgptq_quantize(W, mq.matgptq_prepare(H))
+    c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), oracle.matgptq_prepare(H))
+    # U agrees to ~1e-13 relative, so a code may differ only where two codes
+    # tie to within that; none do on this input
+    assert np.array_equal(codes, c_ref)
+    assert np.allclose(scales, s_ref, rtol=1e-6)
+
+
+def test_argument_errors():
+    K = 128
+    U = np.eye(K)
+    W = _W(2, K, 51)
+    bad = [
+        dict(W=_W(2, 100, 1), U=np.eye(100)),               # K not a multiple of 128
+        dict(rs=(3, 9), lambdas=(1.0, 1.0)),                 # width above 8
+        dict(rs=(0,), lambdas=(1.0,)),                       # width below 1
+        dict(rs=(3, 4), lambdas=(0.0, 0.0)),                 # all lambdas zero
+        dict(rs=(3, 4), lambdas=(1.0, -1.0)),                # a negative lambda
+        dict(alphas=(1.0, 0.0)),                             # a zero alpha
+        dict(alphas=()),                                     # no alpha
+        dict(U=np.diag(np.r_[np.ones(K - 1), 0.0])),         # zero on U's diagonal
+    ]
+    for kw in bad:
+        args = dict(W=W, U=U)
+        args.update(kw)
+        with pytest.raises(mq.MQError):
+            mq.matgptq_quantize(**args)
+    with pytest.raises(ValueError):
+        mq.matgptq_quantize(W, np.eye(64))
+    with pytest.raises(ValueError):
+        mq.matgptq_quantize(W, U, rs=(3, 4), lambdas=(1.0,))
+    with pytest.raises(mq.MQError):
+        mq.matgptq_prepare(-np.eye(8))                       # not positive definite
+    with pytest.raises(mq.MQError):
+        mq.matgptq_prepare(np.eye(8), damp=-1.0)
+    with pytest.raises(ValueError):
+        mq.matgptq_prepare(np.eye(8)[:4])
