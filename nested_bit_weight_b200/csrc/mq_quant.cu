@@ -18,6 +18,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <atomic>
 #include <thread>
 #include <vector>
 
@@ -45,24 +46,56 @@ struct Objective {
         for (int i = 0; i < nr; ++i)
             for (int q = 0; q < 256; ++q) levels[(size_t)i * 256 + q] = level_of(q, rs[i]);
     }
-    // argmin over q of sum_r lambda_r (w - s v_r(q))^2, the first minimum
+    // argmin over q of sum_r lambda_r (w - s v_r(q))^2, the first minimum;
+    // each cost sums its terms in the order of the widths (the loop over q
+    // is the vectorised one, which leaves every cost's own sum unchanged)
     int best_code(double w, double s) const {
-        int best = 0;
-        double best_c = 0.0;
-        for (int q = 0; q < 256; ++q) {
-            double c = 0.0;
-            for (int i = 0; i < nr; ++i) {
-                const double d = w - s * levels[(size_t)i * 256 + q];
-                c += lams[i] * d * d;
-            }
-            if (q == 0 || c < best_c) {
-                best = q;
-                best_c = c;
+        alignas(64) double c[256];
+        for (int q = 0; q < 256; ++q) c[q] = 0.0;
+        for (int i = 0; i < nr; ++i) {
+            const double lam = lams[i];
+            const double *lv = levels.data() + (size_t)i * 256;
+            for (int q = 0; q < 256; ++q) {
+                const double d = w - s * lv[q];
+                c[q] += lam * d * d;
             }
         }
+        int best = 0;
+        for (int q = 1; q < 256; ++q)
+            if (c[q] < c[best]) best = q;
         return best;
     }
 };
+
+// sum a[i] b[i], four interleaved partial sums
+inline double dot(const double *a, const double *b, int64_t m) {
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    int64_t i = 0;
+    for (; i + 4 <= m; i += 4) {
+        s0 += a[i] * b[i];
+        s1 += a[i + 1] * b[i + 1];
+        s2 += a[i + 2] * b[i + 2];
+        s3 += a[i + 3] * b[i + 3];
+    }
+    for (; i < m; ++i) s0 += a[i] * b[i];
+    return (s0 + s1) + (s2 + s3);
+}
+
+// f(i) for i in [i0, i1), spread over up to nt threads by a shared counter
+// (rows of unequal cost balance themselves)
+template <class F>
+void parallel_rows(int64_t i0, int64_t i1, int nt, F &&f) {
+    if (i1 <= i0) return;
+    std::atomic<int64_t> next{i0};
+    auto work = [&]() {
+        for (int64_t i; (i = next.fetch_add(1)) < i1;) f(i);
+    };
+    const int m = (int)std::min<int64_t>(nt, i1 - i0);
+    std::vector<std::thread> pool;
+    for (int t = 1; t < m; ++t) pool.emplace_back(work);
+    work();
+    for (auto &th : pool) th.join();
+}
 
 void quantize_rows(const float *W, int64_t K, const double *U, const Objective &obj, const double *alphas,
                    int na, double lsum, int64_t n0, int64_t n1, uint8_t *codes, float *scales) {
@@ -112,59 +145,54 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
     if (!H || !U_out) return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_matgptq_prepare");
     if (K < 1 || K > 65536) return fail(MQ_ERR_INVALID_ARG, "need 1 <= K <= 65536");
     if (!(damp >= 0.0)) return fail(MQ_ERR_INVALID_ARG, "damp must be >= 0");
-    const size_t n = (size_t)K;
+    // A = H + damp * mean(diag H) * I and J the reversal (J A J reverses
+    // rows and columns).  With J A J = L L^T (lower Cholesky), A = R R^T for
+    // the upper R = J L J, so A^-1 = R^-T R^-1 and U = R^-1 = J L^-1 J is the
+    // upper factor with U^T U = A^-1 (unique for a positive diagonal).
+    const int64_t n = K;
     double mean = 0.0;
-    for (size_t i = 0; i < n; ++i) mean += H[i * n + i];
+    for (int64_t i = 0; i < n; ++i) mean += H[i * n + i];
     mean /= (double)K;
-    // L L^T = H + damp * mean * I (lower Cholesky)
-    std::vector<double> L(n * n, 0.0);
-    for (size_t j = 0; j < n; ++j) {
-        double d = H[j * n + j] + damp * mean;
-        for (size_t p = 0; p < j; ++p) d -= L[j * n + p] * L[j * n + p];
-        if (!(d > 0.0)) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is not positive definite");
-        const double ljj = sqrt(d);
-        L[j * n + j] = ljj;
-        for (size_t i = j + 1; i < n; ++i) {
-            double v = H[i * n + j];
-            for (size_t p = 0; p < j; ++p) v -= L[i * n + p] * L[j * n + p];
-            L[i * n + j] = v / ljj;
-        }
+    const double add = damp * mean;
+    auto P = [&](int64_t i, int64_t j) {
+        return H[(n - 1 - i) * n + (n - 1 - j)] + (i == j ? add : 0.0);
+    };
+    const int nt = std::max(1, std::min<int>(64, (int)std::thread::hardware_concurrency()));
+    std::vector<double> L((size_t)n * n, 0.0);
+    double *Lp = L.data();
+    // Cholesky by panels of kPanel columns: the panel's diagonal rows in
+    // order, then every row below it (independent of one another) in threads
+    constexpr int64_t kPanel = 64;
+    for (int64_t j0 = 0; j0 < n; j0 += kPanel) {
+        const int64_t j1 = std::min(n, j0 + kPanel);
+        for (int64_t i = j0; i < j1; ++i)
+            for (int64_t j = j0; j <= i; ++j) {
+                const double v = P(i, j) - dot(Lp + i * n, Lp + j * n, j);
+                if (i == j) {
+                    if (!(v > 0.0) || !isfinite(v))
+                        return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is not positive definite");
+                    Lp[i * n + i] = sqrt(v);
+                } else {
+                    Lp[i * n + j] = v / Lp[j * n + j];
+                }
+            }
+        parallel_rows(j1, n, nt, [&](int64_t i) {
+            for (int64_t j = j0; j < j1; ++j)
+                Lp[i * n + j] = (P(i, j) - dot(Lp + i * n, Lp + j * n, j)) / Lp[j * n + j];
+        });
     }
-    // M = L^-1 (lower), then Hinv = M^T M
-    std::vector<double> Mi(n * n, 0.0);
-    for (size_t j = 0; j < n; ++j) {
-        Mi[j * n + j] = 1.0 / L[j * n + j];
-        for (size_t i = j + 1; i < n; ++i) {
-            double v = 0.0;
-            for (size_t p = j; p < i; ++p) v -= L[i * n + p] * Mi[p * n + j];
-            Mi[i * n + j] = v / L[i * n + i];
-        }
-    }
-    std::vector<double> Hinv(n * n, 0.0);
-    for (size_t i = 0; i < n; ++i)
-        for (size_t j = 0; j <= i; ++j) {
-            double v = 0.0;
-            for (size_t p = i; p < n; ++p) v += Mi[p * n + i] * Mi[p * n + j];
-            Hinv[i * n + j] = v;
-            Hinv[j * n + i] = v;
-        }
-    // U upper with U^T U = Hinv: U = R^T, R R^T = Hinv the lower Cholesky
-    std::fill(U_out, U_out + n * n, 0.0);
-    std::vector<double> R(n * n, 0.0);
-    for (size_t j = 0; j < n; ++j) {
-        double d = Hinv[j * n + j];
-        for (size_t p = 0; p < j; ++p) d -= R[j * n + p] * R[j * n + p];
-        if (!(d > 0.0)) return fail(MQ_ERR_UNSUPPORTED, "the inverse Hessian is not positive definite");
-        const double rjj = sqrt(d);
-        R[j * n + j] = rjj;
-        for (size_t i = j + 1; i < n; ++i) {
-            double v = Hinv[i * n + j];
-            for (size_t p = 0; p < j; ++p) v -= R[i * n + p] * R[j * n + p];
-            R[i * n + j] = v / rjj;
-        }
-    }
-    for (size_t i = 0; i < n; ++i)
-        for (size_t j = i; j < n; ++j) U_out[i * n + j] = R[j * n + i];
+    // column c of L^-1 by forward substitution (columns independent), written
+    // reversed into U: U[n-1-i][n-1-c] = (L^-1)[i][c]
+    std::fill(U_out, U_out + (size_t)n * n, 0.0);
+    parallel_rows(0, n, nt, [&](int64_t c) {
+        std::vector<double> x((size_t)(n - c));
+        x[0] = 1.0 / Lp[c * n + c];
+        for (int64_t i = c + 1; i < n; ++i)
+            x[(size_t)(i - c)] = -dot(Lp + i * n + c, x.data(), i - c) / Lp[i * n + i];
+        for (int64_t i = c; i < n; ++i) U_out[(n - 1 - i) * n + (n - 1 - c)] = x[(size_t)(i - c)];
+    });
+    for (int64_t i = 0; i < n; ++i)
+        if (!(U_out[i * n + i] > 0.0) || !isfinite(U_out[i * n + i])) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is too ill-conditioned to invert");
     return MQ_OK;
 }
 
