@@ -104,3 +104,40 @@ def test_argument_errors():
         mq.matgptq_prepare(np.eye(8), damp=-1.0)
     with pytest.raises(ValueError):
         mq.matgptq_prepare(np.eye(8)[:4])
+
+
+def test_degenerate_rows_and_exact_ties_match_the_oracle():
+    # row 0: all zero (s = 0, every code ties: code 0); row 1: its first group
+    # zero; row 2: values exactly halfway between two 8-bit levels with
+    # s = 2^-7 exactly (ties to the smaller code); row 3: one nonzero weight
+    K = 256
+    W = np.zeros((4, K), np.float32)
+    W[1, 128:] = np.linspace(-0.03, 0.05, 128, dtype=np.float32)
+    q = np.arange(128) % 255
+    W[2, :128] = ((q - 127.0) / 128.0).astype(np.float32)     # (q - 127) * 2^-7
+    W[2, 0] = np.float32(127.5 / 128.0)                       # max |w| = 127.5 * 2^-7
+    W[2, 128:] = W[2, :128]
+    W[3, 200] = 0.01
+    U = oracle.matgptq_prepare(_H(K, 61))
+    for U_ in (np.eye(K), U):
+        for rs, lams in (((8,), (1.0,)), ((3, 4, 8), (1.0, 1.0, 1.0))):
+            c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U_, rs=rs, lams=lams, alphas=(1.0,))
+            codes, scales = mq.matgptq_quantize(W, U_, rs=rs, lambdas=lams, alphas=(1.0,))
+            assert np.array_equal(codes, c_ref), rs
+            assert np.array_equal(scales, s_ref.astype(np.float32)), rs
+    codes, scales = mq.matgptq_quantize(W, np.eye(K), rs=(8,), lambdas=(1.0,), alphas=(1.0,))
+    assert np.all(codes[0] == 0) and np.all(scales[0] == 0)
+    assert np.all(codes[1, :128] == 0) and scales[1, 0] == 0 and scales[1, 1] > 0
+    assert scales[2, 0] == 2.0 ** -7
+    # w / s = q - 127 lies halfway between the levels q - 127.5 and q - 126.5
+    # of codes q and q + 1: the smaller code wins
+    assert codes[2, 0] == 255
+    assert np.array_equal(codes[2, 1:128], q[1:].astype(np.uint8))
+
+
+def test_single_row_single_group():
+    W = _W(1, 128, 71)
+    U = oracle.matgptq_prepare(_H(128, 72))
+    c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U)
+    codes, scales = mq.matgptq_quantize(W, U)
+    assert np.array_equal(codes, c_ref) and np.array_equal(scales, s_ref.astype(np.float32))
