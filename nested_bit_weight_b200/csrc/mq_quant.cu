@@ -46,23 +46,57 @@ struct Objective {
         for (int i = 0; i < nr; ++i)
             for (int q = 0; q < 256; ++q) levels[(size_t)i * 256 + q] = level_of(q, rs[i]);
     }
-    // argmin over q of sum_r lambda_r (w - s v_r(q))^2, the first minimum;
-    // each cost sums its terms in the order of the widths (the loop over q
-    // is the vectorised one, which leaves every cost's own sum unchanged)
-    int best_code(double w, double s) const {
-        alignas(64) double c[256];
-        for (int q = 0; q < 256; ++q) c[q] = 0.0;
+
+    // sv[i][q] = s * v_i(q) for one scale s (non-decreasing in q for s >= 0)
+    void products(double s, double *sv) const {
+        for (int i = 0; i < nr * 256; ++i) sv[i] = s * levels[(size_t)i];
+    }
+
+    // the objective at code q, its terms summed in the order of the widths
+    double cost(double w, const double *sv, int q) const {
+        double c = 0.0;
         for (int i = 0; i < nr; ++i) {
-            const double lam = lams[i];
-            const double *lv = levels.data() + (size_t)i * 256;
-            for (int q = 0; q < 256; ++q) {
-                const double d = w - s * lv[q];
-                c[q] += lam * d * d;
+            const double d = w - sv[i * 256 + q];
+            c += lams[i] * d * d;
+        }
+        return c;
+    }
+
+    // The first q in 0..255 of least cost(w, sv, q), found exactly without
+    // evaluating every code.  Each term lambda (w - s v_i(q))^2, rounded, is
+    // non-increasing in q up to A_i, the last code with s v_i(q) <= w, and
+    // non-decreasing from B_i, the first code with s v_i(q) >= w (rounding is
+    // monotone and keeps the sign of w - s v_i(q)); so is their rounded sum
+    // (addition is monotone in each operand).  Hence the cost cannot fall
+    // below its value on [min(a, b), max(a, b)], a = min A_i, b = max B_i,
+    // outside it, and the first minimum lies inside it or, when the cost is
+    // flat at the window's left end, further left by equal steps.
+    int best_code(double w, const double *sv) const {
+        int a = 256, b = -1;
+        for (int i = 0; i < nr; ++i) {
+            if (!(lams[i] > 0.0)) continue;          // a zero term is flat everywhere
+            const double *p = sv + i * 256;
+            a = std::min(a, (int)(std::upper_bound(p, p + 256, w) - p) - 1);
+            b = std::max(b, (int)(std::lower_bound(p, p + 256, w) - p));
+        }
+        const int q0 = std::max(0, std::min(a, b)), q1 = std::min(255, std::max(a, b));
+        int best = q0;
+        double bc = cost(w, sv, q0);
+        for (int q = q0 + 1; q <= q1; ++q) {
+            const double c = cost(w, sv, q);
+            if (c < bc) {
+                best = q;
+                bc = c;
             }
         }
-        int best = 0;
-        for (int q = 1; q < 256; ++q)
-            if (c[q] < c[best]) best = q;
+        if (best == q0) {
+            while (best > 0) {
+                const double c = cost(w, sv, best - 1);
+                if (!(c <= bc)) break;
+                bc = c;
+                --best;
+            }
+        }
         return best;
     }
 };
@@ -81,6 +115,34 @@ inline double dot(const double *a, const double *b, int64_t m) {
     return (s0 + s1) + (s2 + s3);
 }
 
+// out[r] = sum_p a[r * lda + p] b[p] for r < 4, p < m: four rows against one
+inline void dot4(const double *a, int64_t lda, const double *b, int64_t m, double *out) {
+    const double *a0 = a, *a1 = a + lda, *a2 = a + 2 * lda, *a3 = a + 3 * lda;
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0, t0 = 0.0, t1 = 0.0, t2 = 0.0, t3 = 0.0;
+    int64_t p = 0;
+    for (; p + 2 <= m; p += 2) {
+        const double b0 = b[p], b1 = b[p + 1];
+        s0 += a0[p] * b0;
+        t0 += a0[p + 1] * b1;
+        s1 += a1[p] * b0;
+        t1 += a1[p + 1] * b1;
+        s2 += a2[p] * b0;
+        t2 += a2[p + 1] * b1;
+        s3 += a3[p] * b0;
+        t3 += a3[p + 1] * b1;
+    }
+    if (p < m) {
+        s0 += a0[p] * b[p];
+        s1 += a1[p] * b[p];
+        s2 += a2[p] * b[p];
+        s3 += a3[p] * b[p];
+    }
+    out[0] = s0 + t0;
+    out[1] = s1 + t1;
+    out[2] = s2 + t2;
+    out[3] = s3 + t3;
+}
+
 // f(i) for i in [i0, i1), spread over up to nt threads by a shared counter
 // (rows of unequal cost balance themselves)
 template <class F>
@@ -97,24 +159,36 @@ void parallel_rows(int64_t i0, int64_t i1, int nt, F &&f) {
     for (auto &th : pool) th.join();
 }
 
+// Rows n0..n1-1 (at most kRowBlock), column by column together: each row of
+// U is then read once per block of rows rather than once per row (the
+// feedback streams U's upper triangle for every column).  Every row still
+// takes exactly the operations, in the order, of quantizing it alone.
+constexpr int64_t kRowBlock = 16;
+
 void quantize_rows(const float *W, int64_t K, const double *U, const Objective &obj, const double *alphas,
                    int na, double lsum, int64_t n0, int64_t n1, uint8_t *codes, float *scales) {
-    const int64_t G = K / 128;
-    std::vector<double> w((size_t)K);
-    for (int64_t n = n0; n < n1; ++n) {
-        for (int64_t k = 0; k < K; ++k) w[(size_t)k] = (double)W[n * K + k];
-        for (int64_t g = 0; g < G; ++g) {
+    const int64_t G = K / 128, nb = n1 - n0;
+    const size_t nsv = (size_t)obj.nr * 256;
+    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)nb);
+    for (int64_t b = 0; b < nb; ++b)
+        for (int64_t k = 0; k < K; ++k) w[(size_t)(b * K + k)] = (double)W[(n0 + b) * K + k];
+    for (int64_t g = 0; g < G; ++g) {
+        // each row's scale, from its group's current weights
+        for (int64_t b = 0; b < nb; ++b) {
+            const double *wb = w.data() + b * K;
+            double *svb = sv.data() + nsv * (size_t)b;
             double mx = 0.0;
-            for (int64_t k = 128 * g; k < 128 * g + 128; ++k) mx = std::max(mx, fabs(w[(size_t)k]));
+            for (int64_t k = 128 * g; k < 128 * g + 128; ++k) mx = std::max(mx, fabs(wb[k]));
             const double base = mx / 127.5;
             double best_a = 0.0, best_t = 0.0;
             for (int ia = 0; ia < na; ++ia) {
-                const double s = base * alphas[ia];
+                obj.products(base * alphas[ia], svb);
                 double t = 0.0;
                 for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
-                    const int q = obj.best_code(w[(size_t)k], s);
+                    const double x = wb[k];
+                    const int q = obj.best_code(x, svb);
                     for (int i = 0; i < obj.nr; ++i) {
-                        const double d = w[(size_t)k] - s * obj.levels[(size_t)i * 256 + q];
+                        const double d = x - svb[(size_t)i * 256 + q];
                         t += obj.lams[i] * d * d;
                     }
                 }
@@ -124,16 +198,25 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
                 }
             }
             const double s = base * best_a;
-            scales[n * G + g] = (float)s;
-            for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
-                const int q = obj.best_code(w[(size_t)k], s);
-                codes[n * K + k] = (uint8_t)q;
+            scales[(n0 + b) * G + g] = (float)s;
+            obj.products(s, svb);
+        }
+        for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
+            for (int64_t b = 0; b < nb; ++b) {
+                const double *svb = sv.data() + nsv * (size_t)b;
+                const double x = w[(size_t)(b * K + k)];
+                const int q = obj.best_code(x, svb);
+                codes[(n0 + b) * K + k] = (uint8_t)q;
                 double e = 0.0;
-                for (int i = 0; i < obj.nr; ++i) e += obj.lams[i] * (w[(size_t)k] - s * obj.levels[(size_t)i * 256 + q]);
+                for (int i = 0; i < obj.nr; ++i) e += obj.lams[i] * (x - svb[(size_t)i * 256 + q]);
                 e /= lsum;
-                const double f = e / U[k * K + k];
-                const double *urow = U + k * K;
-                for (int64_t j = k + 1; j < K; ++j) w[(size_t)j] -= f * urow[j];
+                f[(size_t)b] = e / U[k * K + k];
+            }
+            const double *urow = U + k * K;
+            for (int64_t b = 0; b < nb; ++b) {
+                double *wb = w.data() + b * K;
+                const double fb = f[(size_t)b];
+                for (int64_t j = k + 1; j < K; ++j) wb[j] -= fb * urow[j];
             }
         }
     }
@@ -176,20 +259,48 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
                     Lp[i * n + j] = v / Lp[j * n + j];
                 }
             }
-        parallel_rows(j1, n, nt, [&](int64_t i) {
-            for (int64_t j = j0; j < j1; ++j)
-                Lp[i * n + j] = (P(i, j) - dot(Lp + i * n, Lp + j * n, j)) / Lp[j * n + j];
+        // rows below the panel, four at a time (each panel row read once for four)
+        parallel_rows(0, (n - j1 + 3) / 4, nt, [&](int64_t t) {
+            const int64_t i0 = j1 + 4 * t;
+            const int m = (int)std::min<int64_t>(4, n - i0);
+            for (int64_t j = j0; j < j1; ++j) {
+                double acc[4];
+                if (m == 4) {
+                    dot4(Lp + i0 * n, n, Lp + j * n, j, acc);
+                } else {
+                    for (int r = 0; r < m; ++r) acc[r] = dot(Lp + (i0 + r) * n, Lp + j * n, j);
+                }
+                for (int r = 0; r < m; ++r) Lp[(i0 + r) * n + j] = (P(i0 + r, j) - acc[r]) / Lp[j * n + j];
+            }
         });
     }
-    // column c of L^-1 by forward substitution (columns independent), written
-    // reversed into U: U[n-1-i][n-1-c] = (L^-1)[i][c]
+    // columns c0..c0+kCols-1 of L^-1 together by forward substitution (each
+    // row of L read once for kCols columns; x_t[p] = 0 above the diagonal),
+    // written reversed into U: U[n-1-i][n-1-c] = (L^-1)[i][c]
+    constexpr int kCols = 4;
     std::fill(U_out, U_out + (size_t)n * n, 0.0);
-    parallel_rows(0, n, nt, [&](int64_t c) {
-        std::vector<double> x((size_t)(n - c));
-        x[0] = 1.0 / Lp[c * n + c];
-        for (int64_t i = c + 1; i < n; ++i)
-            x[(size_t)(i - c)] = -dot(Lp + i * n + c, x.data(), i - c) / Lp[i * n + i];
-        for (int64_t i = c; i < n; ++i) U_out[(n - 1 - i) * n + (n - 1 - c)] = x[(size_t)(i - c)];
+    parallel_rows(0, (n + kCols - 1) / kCols, nt, [&](int64_t blk) {
+        const int64_t c0 = blk * kCols;
+        const int mc = (int)std::min<int64_t>(kCols, n - c0);
+        std::vector<double> x((size_t)(n - c0) * kCols, 0.0);
+        for (int64_t i = c0; i < n; ++i) {
+            double acc[kCols] = {};
+            const double *li = Lp + i * n;
+            for (int64_t p = c0; p < i; ++p) {
+                const double l = li[p];
+                const double *xp = x.data() + (p - c0) * kCols;
+                for (int t = 0; t < kCols; ++t) acc[t] += l * xp[t];
+            }
+            double *xi = x.data() + (i - c0) * kCols;
+            for (int t = 0; t < mc; ++t) {
+                const int64_t c = c0 + t;
+                xi[t] = i < c ? 0.0 : i == c ? 1.0 / li[i] : -acc[t] / li[i];
+            }
+        }
+        for (int t = 0; t < mc; ++t) {
+            const int64_t c = c0 + t;
+            for (int64_t i = c; i < n; ++i) U_out[(n - 1 - i) * n + (n - 1 - c)] = x[(size_t)((i - c0) * kCols + t)];
+        }
     });
     for (int64_t i = 0; i < n; ++i)
         if (!(U_out[i * n + i] > 0.0) || !isfinite(U_out[i * n + i])) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is too ill-conditioned to invert");
@@ -215,16 +326,14 @@ extern "C" mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, c
         if (!(alphas[i] > 0.0) || !isfinite(alphas[i])) return fail(MQ_ERR_INVALID_ARG, "alphas must be finite and > 0");
     for (int64_t k = 0; k < K; ++k)
         if (!(U[k * K + k] != 0.0)) return fail(MQ_ERR_INVALID_ARG, "U has a zero on its diagonal");
+    for (int64_t i = 0; i < N * K; ++i)
+        if (!isfinite(W[i])) return fail(MQ_ERR_INVALID_ARG, "W holds a non-finite value");
     const Objective obj(rs, lambdas, n_r);
-    int nt = threads > 0 ? threads : (int)std::max(1u, std::thread::hardware_concurrency());
-    nt = (int)std::min<int64_t>(nt, N);
-    std::vector<std::thread> pool;
-    const int64_t per = (N + nt - 1) / nt;
-    for (int t = 0; t < nt; ++t) {
-        const int64_t n0 = t * per, n1 = std::min<int64_t>(N, n0 + per);
-        if (n0 >= n1) break;
-        pool.emplace_back(quantize_rows, W, K, U, std::cref(obj), alphas, n_alpha, lsum, n0, n1, codes_out, scales_out);
-    }
-    for (auto &th : pool) th.join();
+    const int nt = threads > 0 ? threads : (int)std::max(1u, std::thread::hardware_concurrency());
+    const int64_t nblocks = (N + kRowBlock - 1) / kRowBlock;
+    parallel_rows(0, nblocks, nt, [&](int64_t blk) {
+        quantize_rows(W, K, U, obj, alphas, n_alpha, lsum, blk * kRowBlock,
+                      std::min<int64_t>(N, (blk + 1) * kRowBlock), codes_out, scales_out);
+    });
     return MQ_OK;
 }

@@ -141,3 +141,38 @@ def test_single_row_single_group():
     c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U)
     codes, scales = mq.matgptq_quantize(W, U)
     assert np.array_equal(codes, c_ref) and np.array_equal(scales, s_ref.astype(np.float32))
+
+
+def _stress_cases():
+    rng = np.random.default_rng(81)
+    widths = [(1,), (2,), (1, 2), (1, 3), (2, 4), (3, 4, 8), (2, 3, 6), (1, 8), (4, 4), (5, 7, 8)]
+    for i, rs in enumerate(widths):
+        lams = tuple(float(x) for x in rng.choice([0.0, 0.25, 1.0, 3.0], size=len(rs)))
+        if sum(lams) == 0.0:
+            lams = (1.0,) + lams[1:]
+        yield pytest.param(rs, lams, i, id=f"r{'-'.join(map(str, rs))}")
+
+
+@pytest.mark.parametrize("rs,lams,seed", list(_stress_cases()))
+def test_code_search_matches_the_oracle_on_coarse_and_mixed_widths(rs, lams, seed):
+    # half the weights sit on the 2^-7 grid with s = 2^-7 (exact ties between
+    # levels and between whole blocks of codes), half are random
+    K = 256
+    rng = np.random.default_rng(90 + seed)
+    W = (rng.standard_normal((4, K)) * 0.02).astype(np.float32)
+    W[:2] = (rng.integers(-127, 128, size=(2, K)) / 128.0).astype(np.float32)
+    W[:2, 0] = W[:2, 128] = np.float32(127.5 / 128.0)
+    U = np.eye(K) if seed % 2 else oracle.matgptq_prepare(_H(K, 91 + seed))
+    c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U, rs=rs, lams=lams, alphas=(1.0, 0.9))
+    codes, scales = mq.matgptq_quantize(W, U, rs=rs, lambdas=lams, alphas=(1.0, 0.9))
+    assert np.array_equal(codes, c_ref)
+    assert np.array_equal(scales, s_ref.astype(np.float32))
+
+
+def test_non_finite_weights_are_refused():
+    W = _W(2, 128, 95)
+    for bad in (np.nan, np.inf, -np.inf):
+        W2 = W.copy()
+        W2[1, 17] = bad
+        with pytest.raises(mq.MQError):
+            mq.matgptq_quantize(W2, np.eye(128))
