@@ -259,8 +259,10 @@ MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int 
  *     threads <= 0: one per hardware thread.  fp64 in a fixed order, so the
  *     result does not depend on the thread count.
  * Errors: MQ_ERR_INVALID_ARG for bad sizes, widths, lambdas (all zero, or
- * negative) or alphas, or a zero on U's diagonal; MQ_ERR_UNSUPPORTED when the
- * damped Hessian is not positive definite.
+ * negative) or alphas, a non-finite weight, or a zero on U's diagonal;
+ * MQ_ERR_UNSUPPORTED when the damped Hessian is not positive definite (or
+ * too ill-conditioned to invert).  The caller owns every buffer; nothing is
+ * written to codes_out or scales_out on an argument error.
  */
 MQ_API mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp, double *U_out);
 MQ_API mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const double *U,
