@@ -94,6 +94,19 @@ def test_lambda3_lowers_the_3bit_slice_error(q=oracle):
     assert _proxy_loss(W, cm, sm, H, 3) < _proxy_loss(W, c8, s8, H, 3)
 
 
+def test_lambda8_lowers_the_8bit_slice_error(q=oracle):
+    # the other end of the same trade-off: weighting the 8-bit slice up moves
+    # the shared feedback towards the parent's own errors
+    K = 256
+    H = _H(K, seed=8)
+    rng = np.random.default_rng(9)
+    W = rng.standard_normal((4, K)) * 0.02
+    U = q.matgptq_prepare(H)
+    c1, s1 = q.matgptq_quantize(W, U, rs=(3, 4, 8), lams=(1.0, 1.0, 1.0), alphas=(1.0,))
+    c16, s16 = q.matgptq_quantize(W, U, rs=(3, 4, 8), lams=(1.0, 1.0, 16.0), alphas=(1.0,))
+    assert _proxy_loss(W, c16, s16, H, 8) < 0.5 * _proxy_loss(W, c1, s1, H, 8)
+
+
 def test_prepare_factor(q=oracle):
     H = _H(128, seed=7)
     U = q.matgptq_prepare(H, damp=0.01)
@@ -120,7 +133,7 @@ def test_planted_mistakes_fail_a_pin(name):
     exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
     pins = [test_r8_without_feedback_is_round_to_nearest, test_r3_only_uses_the_top_three_bits,
             test_two_column_feedback_worked_example, test_feedback_beats_round_to_nearest_on_correlated_inputs,
-            test_lambda3_lowers_the_3bit_slice_error]
+            test_lambda3_lowers_the_3bit_slice_error, test_lambda8_lowers_the_8bit_slice_error]
     failed = 0
     for pin in pins:
         try:
