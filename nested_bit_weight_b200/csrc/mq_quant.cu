@@ -12,10 +12,14 @@
 //   * each weight's 8-bit code q minimises sum_r lambda_r (w - s v_r(q_r))^2
 //     over the nested levels v_r of every width r (ties: the smallest code);
 //   * the error carried to the later columns of the row is the
-//     lambda-weighted mean of the slice errors e:  w_j -= e / U[k,k] * U[k,j].
-// Rows are independent given U, so threads take rows; every operation is
-// fp64 in a fixed order.
+//     lambda-weighted mean of the slice errors e:  w_j -= e / U[k,k] * U[k,j]
+//     (the update of the row's shared remainder that minimises the
+//     lambda-weighted sum of the widths' quadratic losses).
+// Rows are independent given U, so threads take blocks of rows; every
+// operation is fp64 in a fixed order, the same whatever the thread count.
+#include <immintrin.h>
 #include <math.h>
+#include <stdlib.h>
 
 #include <algorithm>
 #include <atomic>
@@ -159,6 +163,92 @@ void parallel_rows(int64_t i0, int64_t i1, int nt, F &&f) {
     for (auto &th : pool) th.join();
 }
 
+// acc[4 r + t] = sum_{p0 <= p < p1} L[i0 + r][p] x[p - p0][t], r, t < 4 (x
+// holds rows of four)
+inline void acc4x4(const double *L, int64_t n, int64_t i0, int64_t p0, int64_t p1, const double *x,
+                   double *acc) {
+    for (int r = 0; r < 16; ++r) acc[r] = 0.0;
+    for (int64_t p = p0; p < p1; ++p) {
+        const double *xp = x + (p - p0) * 4;
+        for (int r = 0; r < 4; ++r) {
+            const double l = L[(i0 + r) * n + p];
+            for (int t = 0; t < 4; ++t) acc[4 * r + t] += l * xp[t];
+        }
+    }
+}
+
+// The same three kernels with AVX2 and FMA, used by the prepare step when
+// the CPU has both (rounding differs from the portable loops within the
+// prepare step's own error; the code search never uses them).
+// (MQ_PORTABLE_HOST=1 in the environment selects the portable loops.)
+bool have_avx2_fma() {
+    static const bool ok = __builtin_cpu_supports("avx2") && __builtin_cpu_supports("fma") &&
+                           !(getenv("MQ_PORTABLE_HOST") && getenv("MQ_PORTABLE_HOST")[0] == '1');
+    return ok;
+}
+
+__attribute__((target("avx2,fma"))) inline double hsum(__m256d v) {
+    alignas(32) double t[4];
+    _mm256_store_pd(t, v);
+    return (t[0] + t[1]) + (t[2] + t[3]);
+}
+
+__attribute__((target("avx2,fma"))) double dot_avx2(const double *a, const double *b, int64_t m) {
+    __m256d s0 = _mm256_setzero_pd(), s1 = _mm256_setzero_pd();
+    int64_t i = 0;
+    for (; i + 8 <= m; i += 8) {
+        s0 = _mm256_fmadd_pd(_mm256_loadu_pd(a + i), _mm256_loadu_pd(b + i), s0);
+        s1 = _mm256_fmadd_pd(_mm256_loadu_pd(a + i + 4), _mm256_loadu_pd(b + i + 4), s1);
+    }
+    for (; i + 4 <= m; i += 4) s0 = _mm256_fmadd_pd(_mm256_loadu_pd(a + i), _mm256_loadu_pd(b + i), s0);
+    double r = hsum(_mm256_add_pd(s0, s1));
+    for (; i < m; ++i) r += a[i] * b[i];
+    return r;
+}
+
+__attribute__((target("avx2,fma"))) void dot4_avx2(const double *a, int64_t lda, const double *b, int64_t m,
+                                                   double *out) {
+    const double *a0 = a, *a1 = a + lda, *a2 = a + 2 * lda, *a3 = a + 3 * lda;
+    __m256d s0 = _mm256_setzero_pd(), s1 = _mm256_setzero_pd(), s2 = _mm256_setzero_pd(),
+            s3 = _mm256_setzero_pd();
+    int64_t p = 0;
+    for (; p + 4 <= m; p += 4) {
+        const __m256d bv = _mm256_loadu_pd(b + p);
+        s0 = _mm256_fmadd_pd(_mm256_loadu_pd(a0 + p), bv, s0);
+        s1 = _mm256_fmadd_pd(_mm256_loadu_pd(a1 + p), bv, s1);
+        s2 = _mm256_fmadd_pd(_mm256_loadu_pd(a2 + p), bv, s2);
+        s3 = _mm256_fmadd_pd(_mm256_loadu_pd(a3 + p), bv, s3);
+    }
+    out[0] = hsum(s0);
+    out[1] = hsum(s1);
+    out[2] = hsum(s2);
+    out[3] = hsum(s3);
+    for (; p < m; ++p) {
+        out[0] += a0[p] * b[p];
+        out[1] += a1[p] * b[p];
+        out[2] += a2[p] * b[p];
+        out[3] += a3[p] * b[p];
+    }
+}
+
+__attribute__((target("avx2,fma"))) void acc4x4_avx2(const double *L, int64_t n, int64_t i0, int64_t p0,
+                                                     int64_t p1, const double *x, double *acc) {
+    const double *l0 = L + i0 * n, *l1 = l0 + n, *l2 = l1 + n, *l3 = l2 + n;
+    __m256d a0 = _mm256_setzero_pd(), a1 = _mm256_setzero_pd(), a2 = _mm256_setzero_pd(),
+            a3 = _mm256_setzero_pd();
+    for (int64_t p = p0; p < p1; ++p) {
+        const __m256d xv = _mm256_loadu_pd(x + (p - p0) * 4);
+        a0 = _mm256_fmadd_pd(_mm256_broadcast_sd(l0 + p), xv, a0);
+        a1 = _mm256_fmadd_pd(_mm256_broadcast_sd(l1 + p), xv, a1);
+        a2 = _mm256_fmadd_pd(_mm256_broadcast_sd(l2 + p), xv, a2);
+        a3 = _mm256_fmadd_pd(_mm256_broadcast_sd(l3 + p), xv, a3);
+    }
+    _mm256_storeu_pd(acc, a0);
+    _mm256_storeu_pd(acc + 4, a1);
+    _mm256_storeu_pd(acc + 8, a2);
+    _mm256_storeu_pd(acc + 12, a3);
+}
+
 // Rows n0..n1-1 (at most kRowBlock), column by column together: each row of
 // U is then read once per block of rows rather than once per row (the
 // feedback streams U's upper triangle for every column).  Every row still
@@ -246,11 +336,15 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
     // Cholesky by panels of kPanel columns: the panel's diagonal rows in
     // order, then every row below it (independent of one another) in threads
     constexpr int64_t kPanel = 64;
+    const bool avx = have_avx2_fma();
+    auto dotv = [avx](const double *a, const double *b, int64_t m) {
+        return avx ? dot_avx2(a, b, m) : dot(a, b, m);
+    };
     for (int64_t j0 = 0; j0 < n; j0 += kPanel) {
         const int64_t j1 = std::min(n, j0 + kPanel);
         for (int64_t i = j0; i < j1; ++i)
             for (int64_t j = j0; j <= i; ++j) {
-                const double v = P(i, j) - dot(Lp + i * n, Lp + j * n, j);
+                const double v = P(i, j) - dotv(Lp + i * n, Lp + j * n, j);
                 if (i == j) {
                     if (!(v > 0.0) || !isfinite(v))
                         return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is not positive definite");
@@ -266,40 +360,51 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
             for (int64_t j = j0; j < j1; ++j) {
                 double acc[4];
                 if (m == 4) {
-                    dot4(Lp + i0 * n, n, Lp + j * n, j, acc);
+                    if (avx) dot4_avx2(Lp + i0 * n, n, Lp + j * n, j, acc);
+                    else dot4(Lp + i0 * n, n, Lp + j * n, j, acc);
                 } else {
-                    for (int r = 0; r < m; ++r) acc[r] = dot(Lp + (i0 + r) * n, Lp + j * n, j);
+                    for (int r = 0; r < m; ++r) acc[r] = dotv(Lp + (i0 + r) * n, Lp + j * n, j);
                 }
                 for (int r = 0; r < m; ++r) Lp[(i0 + r) * n + j] = (P(i0 + r, j) - acc[r]) / Lp[j * n + j];
             }
         });
     }
-    // columns c0..c0+kCols-1 of L^-1 together by forward substitution (each
-    // row of L read once for kCols columns; x_t[p] = 0 above the diagonal),
-    // written reversed into U: U[n-1-i][n-1-c] = (L^-1)[i][c]
-    constexpr int kCols = 4;
+    // columns c0..c0+3 of L^-1 together by forward substitution, rows four
+    // at a time (each row of L read once for four columns; x_t[p] = 0 above
+    // the diagonal), written reversed into U: U[n-1-i][n-1-c] = (L^-1)[i][c]
     std::fill(U_out, U_out + (size_t)n * n, 0.0);
-    parallel_rows(0, (n + kCols - 1) / kCols, nt, [&](int64_t blk) {
-        const int64_t c0 = blk * kCols;
-        const int mc = (int)std::min<int64_t>(kCols, n - c0);
-        std::vector<double> x((size_t)(n - c0) * kCols, 0.0);
-        for (int64_t i = c0; i < n; ++i) {
-            double acc[kCols] = {};
-            const double *li = Lp + i * n;
-            for (int64_t p = c0; p < i; ++p) {
-                const double l = li[p];
-                const double *xp = x.data() + (p - c0) * kCols;
-                for (int t = 0; t < kCols; ++t) acc[t] += l * xp[t];
+    parallel_rows(0, (n + 3) / 4, nt, [&](int64_t blk) {
+        const int64_t c0 = blk * 4;
+        const int mc = (int)std::min<int64_t>(4, n - c0);
+        std::vector<double> x((size_t)(n - c0) * 4, 0.0);
+        double acc[16];
+        for (int64_t i0 = c0; i0 < n; i0 += 4) {
+            const int m = (int)std::min<int64_t>(4, n - i0);
+            if (m == 4) {
+                if (avx) acc4x4_avx2(Lp, n, i0, c0, i0, x.data(), acc);
+                else acc4x4(Lp, n, i0, c0, i0, x.data(), acc);
+            } else {
+                for (int r = 0; r < 16; ++r) acc[r] = 0.0;
+                for (int r = 0; r < m; ++r)
+                    for (int64_t p = c0; p < i0; ++p)
+                        for (int t = 0; t < 4; ++t) acc[4 * r + t] += Lp[(i0 + r) * n + p] * x[(size_t)((p - c0) * 4 + t)];
             }
-            double *xi = x.data() + (i - c0) * kCols;
-            for (int t = 0; t < mc; ++t) {
-                const int64_t c = c0 + t;
-                xi[t] = i < c ? 0.0 : i == c ? 1.0 / li[i] : -acc[t] / li[i];
+            for (int r = 0; r < m; ++r) {
+                const int64_t i = i0 + r;
+                const double *li = Lp + i * n;
+                double *a = acc + 4 * r;
+                for (int64_t p = i0; p < i; ++p)
+                    for (int t = 0; t < 4; ++t) a[t] += li[p] * x[(size_t)((p - c0) * 4 + t)];
+                double *xi = x.data() + (i - c0) * 4;
+                for (int t = 0; t < mc; ++t) {
+                    const int64_t c = c0 + t;
+                    xi[t] = i < c ? 0.0 : i == c ? 1.0 / li[i] : -a[t] / li[i];
+                }
             }
         }
         for (int t = 0; t < mc; ++t) {
             const int64_t c = c0 + t;
-            for (int64_t i = c; i < n; ++i) U_out[(n - 1 - i) * n + (n - 1 - c)] = x[(size_t)((i - c0) * kCols + t)];
+            for (int64_t i = c; i < n; ++i) U_out[(n - 1 - i) * n + (n - 1 - c)] = x[(size_t)((i - c0) * 4 + t)];
         }
     });
     for (int64_t i = 0; i < n; ++i)

@@ -176,3 +176,23 @@ def test_non_finite_weights_are_refused():
         W2[1, 17] = bad
         with pytest.raises(mq.MQError):
             mq.matgptq_quantize(W2, np.eye(128))
+
+
+def test_prepare_portable_loops_agree_with_the_oracle():
+    # the prepare step's portable loops (selected by MQ_PORTABLE_HOST=1; the
+    # default takes AVX2 and FMA when the CPU has them), in a fresh process
+    import os
+    import subprocess
+    import sys
+    code = (
+        "import numpy as np, sys; sys.path[:0] = %r\n"
+        "import oracle, nested_bit_weight_b200 as mq\n"
+        "rng = np.random.default_rng(5)\n"
+        "for K in (3, 130, 257):\n"
+        "    X = rng.standard_normal((2 * K, K)); H = X.T @ X / (2 * K)\n"
+        "    U = mq.matgptq_prepare(H); ref = oracle.matgptq_prepare(H)\n"
+        "    assert np.allclose(U, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max()), K\n"
+        "print('ok')\n" % (sys.path,))
+    env = dict(os.environ, MQ_PORTABLE_HOST="1")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stderr
