@@ -182,7 +182,7 @@ inline void acc4x4(const double *L, int64_t n, int64_t i0, int64_t p0, int64_t p
 // prepare step's own error; the code search never uses them).
 // (MQ_PORTABLE_HOST=1 in the environment selects the portable loops.)
 bool have_avx2_fma() {
-    static const bool ok = __builtin_cpu_supports("avx2") && __builtin_cpu_supports("fma") &&
+    static const bool ok = (__builtin_cpu_init(), __builtin_cpu_supports("avx2")) && __builtin_cpu_supports("fma") &&
                            !(getenv("MQ_PORTABLE_HOST") && getenv("MQ_PORTABLE_HOST")[0] == '1');
     return ok;
 }
