@@ -63,9 +63,9 @@ def gen_layers():
 
 
 # DRAM traffic of one step (dram__bytes_read.sum + dram__bytes_write.sum
-# summed over the 21 launches) from the ncu capture summarised in
-# profiles/gemv_llama8b_m1_step_traffic.md, valid for the kernel source it was
-# taken with (sha256 of csrc/mq_gemv_tc.cu); None once that source changes.
+# summed over the 21 launches) from one ncu capture of this step (its summary
+# is kept with the other profiles), valid for the kernel source it was taken
+# with (sha256 of csrc/mq_gemv_tc.cu); None once that source changes.
 STEP_TRAFFIC = {"bytes": 257207552, "sha256": "41bd2a91ec1688de3deb334ffff1423e930c225992e283b1b9f4b2ec9c043d84"}
 
 
