@@ -255,8 +255,26 @@ __attribute__((target("avx2,fma"))) void acc4x4_avx2(const double *L, int64_t n,
 // takes exactly the operations, in the order, of quantizing it alone.
 constexpr int64_t kRowBlock = 16;
 
+// w[j] -= f u[j] for j0 <= j < j1: one rounded product and one rounded
+// difference per element (no fused multiply-add), as the oracle computes it
+inline void feedback(double *w, const double *u, double f, int64_t j0, int64_t j1) {
+    for (int64_t j = j0; j < j1; ++j) w[j] -= f * u[j];
+}
+
+// the same, four lanes at a time (AVX2 without FMA: each lane rounds exactly
+// as the scalar loop does)
+__attribute__((target("avx2"))) void feedback_avx2(double *w, const double *u, double f, int64_t j0,
+                                                  int64_t j1) {
+    const __m256d fv = _mm256_set1_pd(f);
+    int64_t j = j0;
+    for (; j + 4 <= j1; j += 4)
+        _mm256_storeu_pd(w + j, _mm256_sub_pd(_mm256_loadu_pd(w + j), _mm256_mul_pd(fv, _mm256_loadu_pd(u + j))));
+    for (; j < j1; ++j) w[j] -= f * u[j];
+}
+
 void quantize_rows(const float *W, int64_t K, const double *U, const Objective &obj, const double *alphas,
                    int na, double lsum, int64_t n0, int64_t n1, uint8_t *codes, float *scales) {
+    const bool avx = have_avx2_fma();
     const int64_t G = K / 128, nb = n1 - n0;
     const size_t nsv = (size_t)obj.nr * 256;
     std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)nb);
@@ -304,9 +322,8 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
             }
             const double *urow = U + k * K;
             for (int64_t b = 0; b < nb; ++b) {
-                double *wb = w.data() + b * K;
-                const double fb = f[(size_t)b];
-                for (int64_t j = k + 1; j < K; ++j) wb[j] -= fb * urow[j];
+                if (avx) feedback_avx2(w.data() + b * K, urow, f[(size_t)b], k + 1, K);
+                else feedback(w.data() + b * K, urow, f[(size_t)b], k + 1, K);
             }
         }
     }
