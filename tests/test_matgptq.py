@@ -178,9 +178,10 @@ def test_non_finite_weights_are_refused():
             mq.matgptq_quantize(W2, np.eye(128))
 
 
-def test_prepare_portable_loops_agree_with_the_oracle():
-    # the prepare step's portable loops (selected by MQ_PORTABLE_HOST=1; the
-    # default takes AVX2 and FMA when the CPU has them), in a fresh process
+def test_portable_loops_agree_with_the_oracle():
+    # the portable host loops (selected by MQ_PORTABLE_HOST=1; the default
+    # takes AVX2, and FMA in the prepare step, when the CPU has them), in a
+    # fresh process: prepare within rounding, quantize bit for bit
     import os
     import subprocess
     import sys
@@ -192,6 +193,10 @@ def test_prepare_portable_loops_agree_with_the_oracle():
         "    X = rng.standard_normal((2 * K, K)); H = X.T @ X / (2 * K)\n"
         "    U = mq.matgptq_prepare(H); ref = oracle.matgptq_prepare(H)\n"
         "    assert np.allclose(U, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max()), K\n"
+        "W = (rng.standard_normal((3, 256)) * 0.02).astype(np.float32)\n"
+        "U = oracle.matgptq_prepare(W.T.astype(np.float64) @ W + np.eye(256))\n"
+        "c, s = mq.matgptq_quantize(W, U); cr, sr = oracle.matgptq_quantize(W.astype(np.float64), U)\n"
+        "assert np.array_equal(c, cr) and np.array_equal(s, sr.astype(np.float32))\n"
         "print('ok')\n" % (sys.path,))
     env = dict(os.environ, MQ_PORTABLE_HOST="1")
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
