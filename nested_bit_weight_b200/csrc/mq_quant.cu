@@ -23,6 +23,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <memory>
 #include <thread>
 #include <vector>
 
@@ -119,34 +120,6 @@ inline double dot(const double *a, const double *b, int64_t m) {
     return (s0 + s1) + (s2 + s3);
 }
 
-// out[r] = sum_p a[r * lda + p] b[p] for r < 4, p < m: four rows against one
-inline void dot4(const double *a, int64_t lda, const double *b, int64_t m, double *out) {
-    const double *a0 = a, *a1 = a + lda, *a2 = a + 2 * lda, *a3 = a + 3 * lda;
-    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0, t0 = 0.0, t1 = 0.0, t2 = 0.0, t3 = 0.0;
-    int64_t p = 0;
-    for (; p + 2 <= m; p += 2) {
-        const double b0 = b[p], b1 = b[p + 1];
-        s0 += a0[p] * b0;
-        t0 += a0[p + 1] * b1;
-        s1 += a1[p] * b0;
-        t1 += a1[p + 1] * b1;
-        s2 += a2[p] * b0;
-        t2 += a2[p + 1] * b1;
-        s3 += a3[p] * b0;
-        t3 += a3[p + 1] * b1;
-    }
-    if (p < m) {
-        s0 += a0[p] * b[p];
-        s1 += a1[p] * b[p];
-        s2 += a2[p] * b[p];
-        s3 += a3[p] * b[p];
-    }
-    out[0] = s0 + t0;
-    out[1] = s1 + t1;
-    out[2] = s2 + t2;
-    out[3] = s3 + t3;
-}
-
 // f(i) for i in [i0, i1), spread over up to nt threads by a shared counter
 // (rows of unequal cost balance themselves)
 template <class F>
@@ -163,21 +136,26 @@ void parallel_rows(int64_t i0, int64_t i1, int nt, F &&f) {
     for (auto &th : pool) th.join();
 }
 
-// acc[4 r + t] = sum_{p0 <= p < p1} L[i0 + r][p] x[p - p0][t], r, t < 4 (x
-// holds rows of four)
-inline void acc4x4(const double *L, int64_t n, int64_t i0, int64_t p0, int64_t p1, const double *x,
-                   double *acc) {
-    for (int r = 0; r < 16; ++r) acc[r] = 0.0;
+// T[r][c] += sum_{p0 <= p < p1} A[r][p] B[p][c] for r < 4, c < 8 (rows of
+// A, B and T at strides lda, ldb, ldt): the inner block of the triangular
+// inverse
+inline void gemm4x8(const double *A, int64_t lda, const double *B, int64_t ldb, int64_t p0, int64_t p1,
+                    double *T, int64_t ldt) {
+    double acc[4][8];
+    for (int r = 0; r < 4; ++r)
+        for (int c = 0; c < 8; ++c) acc[r][c] = T[r * ldt + c];
     for (int64_t p = p0; p < p1; ++p) {
-        const double *xp = x + (p - p0) * 4;
+        const double *bp = B + p * ldb;
         for (int r = 0; r < 4; ++r) {
-            const double l = L[(i0 + r) * n + p];
-            for (int t = 0; t < 4; ++t) acc[4 * r + t] += l * xp[t];
+            const double a = A[r * lda + p];
+            for (int c = 0; c < 8; ++c) acc[r][c] += a * bp[c];
         }
     }
+    for (int r = 0; r < 4; ++r)
+        for (int c = 0; c < 8; ++c) T[r * ldt + c] = acc[r][c];
 }
 
-// The same three kernels with AVX2 and FMA, used by the prepare step when
+// The same kernels with AVX2 and FMA, used by the prepare step when
 // the CPU has both (rounding differs from the portable loops within the
 // prepare step's own error; the code search never uses them).
 // (MQ_PORTABLE_HOST=1 in the environment selects the portable loops.)
@@ -206,47 +184,103 @@ __attribute__((target("avx2,fma"))) double dot_avx2(const double *a, const doubl
     return r;
 }
 
-__attribute__((target("avx2,fma"))) void dot4_avx2(const double *a, int64_t lda, const double *b, int64_t m,
-                                                   double *out) {
-    const double *a0 = a, *a1 = a + lda, *a2 = a + 2 * lda, *a3 = a + 3 * lda;
-    __m256d s0 = _mm256_setzero_pd(), s1 = _mm256_setzero_pd(), s2 = _mm256_setzero_pd(),
-            s3 = _mm256_setzero_pd();
-    int64_t p = 0;
-    for (; p + 4 <= m; p += 4) {
-        const __m256d bv = _mm256_loadu_pd(b + p);
-        s0 = _mm256_fmadd_pd(_mm256_loadu_pd(a0 + p), bv, s0);
-        s1 = _mm256_fmadd_pd(_mm256_loadu_pd(a1 + p), bv, s1);
-        s2 = _mm256_fmadd_pd(_mm256_loadu_pd(a2 + p), bv, s2);
-        s3 = _mm256_fmadd_pd(_mm256_loadu_pd(a3 + p), bv, s3);
+__attribute__((target("avx2,fma"))) void gemm4x8_avx2(const double *A, int64_t lda, const double *B,
+                                                      int64_t ldb, int64_t p0, int64_t p1, double *T,
+                                                      int64_t ldt) {
+    const double *a0 = A, *a1 = A + lda, *a2 = A + 2 * lda, *a3 = A + 3 * lda;
+    __m256d t00 = _mm256_loadu_pd(T), t01 = _mm256_loadu_pd(T + 4);
+    __m256d t10 = _mm256_loadu_pd(T + ldt), t11 = _mm256_loadu_pd(T + ldt + 4);
+    __m256d t20 = _mm256_loadu_pd(T + 2 * ldt), t21 = _mm256_loadu_pd(T + 2 * ldt + 4);
+    __m256d t30 = _mm256_loadu_pd(T + 3 * ldt), t31 = _mm256_loadu_pd(T + 3 * ldt + 4);
+    for (int64_t p = p0; p < p1; ++p) {
+        const double *bp = B + p * ldb;
+        const __m256d b0 = _mm256_loadu_pd(bp), b1 = _mm256_loadu_pd(bp + 4);
+        __m256d a = _mm256_broadcast_sd(a0 + p);
+        t00 = _mm256_fmadd_pd(a, b0, t00);
+        t01 = _mm256_fmadd_pd(a, b1, t01);
+        a = _mm256_broadcast_sd(a1 + p);
+        t10 = _mm256_fmadd_pd(a, b0, t10);
+        t11 = _mm256_fmadd_pd(a, b1, t11);
+        a = _mm256_broadcast_sd(a2 + p);
+        t20 = _mm256_fmadd_pd(a, b0, t20);
+        t21 = _mm256_fmadd_pd(a, b1, t21);
+        a = _mm256_broadcast_sd(a3 + p);
+        t30 = _mm256_fmadd_pd(a, b0, t30);
+        t31 = _mm256_fmadd_pd(a, b1, t31);
     }
-    out[0] = hsum(s0);
-    out[1] = hsum(s1);
-    out[2] = hsum(s2);
-    out[3] = hsum(s3);
-    for (; p < m; ++p) {
-        out[0] += a0[p] * b[p];
-        out[1] += a1[p] * b[p];
-        out[2] += a2[p] * b[p];
-        out[3] += a3[p] * b[p];
-    }
+    _mm256_storeu_pd(T, t00);
+    _mm256_storeu_pd(T + 4, t01);
+    _mm256_storeu_pd(T + ldt, t10);
+    _mm256_storeu_pd(T + ldt + 4, t11);
+    _mm256_storeu_pd(T + 2 * ldt, t20);
+    _mm256_storeu_pd(T + 2 * ldt + 4, t21);
+    _mm256_storeu_pd(T + 3 * ldt, t30);
+    _mm256_storeu_pd(T + 3 * ldt + 4, t31);
 }
 
-__attribute__((target("avx2,fma"))) void acc4x4_avx2(const double *L, int64_t n, int64_t i0, int64_t p0,
-                                                     int64_t p1, const double *x, double *acc) {
-    const double *l0 = L + i0 * n, *l1 = l0 + n, *l2 = l1 + n, *l3 = l2 + n;
-    __m256d a0 = _mm256_setzero_pd(), a1 = _mm256_setzero_pd(), a2 = _mm256_setzero_pd(),
-            a3 = _mm256_setzero_pd();
-    for (int64_t p = p0; p < p1; ++p) {
-        const __m256d xv = _mm256_loadu_pd(x + (p - p0) * 4);
-        a0 = _mm256_fmadd_pd(_mm256_broadcast_sd(l0 + p), xv, a0);
-        a1 = _mm256_fmadd_pd(_mm256_broadcast_sd(l1 + p), xv, a1);
-        a2 = _mm256_fmadd_pd(_mm256_broadcast_sd(l2 + p), xv, a2);
-        a3 = _mm256_fmadd_pd(_mm256_broadcast_sd(l3 + p), xv, a3);
+// M = L^-1 (both n x n row-major, lower triangular; M zero on entry above
+// the diagonal and written everywhere on and below it), by blocks of kRB
+// rows, each after the ones above it:
+//   M[I, J] = -L[I, I]^-1 (L[I, 0:i0] M[0:i0, J])  for the columns J < i0,
+//   M[I, I] = L[I, I]^-1,
+// the product taken kCW columns per task and kPB terms at a time so that
+// its operands stay in cache.
+void invert_lower(const double *L, int64_t n, double *M, int nt, bool avx) {
+    constexpr int64_t kRB = 128, kCW = 64, kPB = 256;
+    for (int64_t i0 = 0; i0 < n; i0 += kRB) {
+        const int64_t b = std::min(kRB, n - i0);
+        parallel_rows(0, (i0 + kCW - 1) / kCW, nt, [&](int64_t task) {
+            const int64_t j0 = task * kCW, w = std::min(kCW, i0 - j0);
+            std::vector<double> T((size_t)(kRB * kCW), 0.0), Bp((size_t)(kPB * kCW), 0.0);
+            // T = L[I, j0:i0] M[j0:i0, j0:j0+w]  (M[p][j] = 0 for p < j), each
+            // kPB x kCW block of M first copied to a contiguous buffer
+            for (int64_t pp = j0; pp < i0; pp += kPB) {
+                const int64_t pe = std::min(i0, pp + kPB);
+                for (int64_t p = pp; p < pe; ++p)
+                    std::copy(M + p * n + j0, M + p * n + j0 + w, Bp.data() + (p - pp) * kCW);
+                const double *B = Bp.data() - pp * kCW;   // row p of the block at B + p * kCW
+                for (int64_t r0 = 0; r0 < b; r0 += 4) {
+                    const double *A = L + (i0 + r0) * n;
+                    for (int64_t c0 = 0; c0 < w; c0 += 8) {
+                        double *Tt = T.data() + r0 * kCW + c0;
+                        if (r0 + 4 <= b && c0 + 8 <= w) {
+                            if (avx) gemm4x8_avx2(A, n, B + c0, kCW, pp, pe, Tt, kCW);
+                            else gemm4x8(A, n, B + c0, kCW, pp, pe, Tt, kCW);
+                        } else {
+                            for (int64_t r = 0; r < std::min<int64_t>(4, b - r0); ++r)
+                                for (int64_t c = 0; c < std::min<int64_t>(8, w - c0); ++c) {
+                                    double v = Tt[r * kCW + c];
+                                    for (int64_t p = pp; p < pe; ++p) v += A[r * n + p] * B[p * kCW + c0 + c];
+                                    Tt[r * kCW + c] = v;
+                                }
+                        }
+                    }
+                }
+            }
+            // M[I, j0:j0+w] = -L[I, I]^-1 T, down the block's rows
+            double v[kCW];
+            for (int64_t r = 0; r < b; ++r) {
+                const double *li = L + (i0 + r) * n + i0;
+                for (int64_t c = 0; c < w; ++c) v[c] = -T[(size_t)(r * kCW + c)];
+                for (int64_t q = 0; q < r; ++q) {
+                    const double lq = li[q];
+                    const double *mq = M + (i0 + q) * n + j0;
+                    for (int64_t c = 0; c < w; ++c) v[c] -= lq * mq[c];
+                }
+                double *mi = M + (i0 + r) * n + j0;
+                for (int64_t c = 0; c < w; ++c) mi[c] = v[c] / li[r];
+            }
+        });
+        // M[I, I] = L[I, I]^-1
+        for (int64_t c = 0; c < b; ++c) {
+            M[(i0 + c) * n + i0 + c] = 1.0 / L[(i0 + c) * n + i0 + c];
+            for (int64_t r = c + 1; r < b; ++r) {
+                double v = 0.0;
+                for (int64_t q = c; q < r; ++q) v += L[(i0 + r) * n + i0 + q] * M[(i0 + q) * n + i0 + c];
+                M[(i0 + r) * n + i0 + c] = -v / L[(i0 + r) * n + i0 + r];
+            }
+        }
     }
-    _mm256_storeu_pd(acc, a0);
-    _mm256_storeu_pd(acc + 4, a1);
-    _mm256_storeu_pd(acc + 8, a2);
-    _mm256_storeu_pd(acc + 12, a3);
 }
 
 // Rows n0..n1-1 (at most kRowBlock), column by column together: each row of
@@ -348,20 +382,31 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
         return H[(n - 1 - i) * n + (n - 1 - j)] + (i == j ? add : 0.0);
     };
     const int nt = std::max(1, std::min<int>(64, (int)std::thread::hardware_concurrency()));
-    std::vector<double> L((size_t)n * n, 0.0);
-    double *Lp = L.data();
-    // Cholesky by panels of kPanel columns: the panel's diagonal rows in
-    // order, then every row below it (independent of one another) in threads
-    constexpr int64_t kPanel = 64;
+    // L starts as the lower triangle of J A J and is factorised in place;
+    // its upper triangle is never read, so the buffer is not initialised
+    // (its pages are first touched by the threads that copy the rows)
+    std::unique_ptr<double[]> L(new double[(size_t)n * n]);
+    double *Lp = L.get();
+    parallel_rows(0, n, nt, [&](int64_t i) {
+        for (int64_t j = 0; j <= i; ++j) Lp[i * n + j] = P(i, j);
+    });
     const bool avx = have_avx2_fma();
     auto dotv = [avx](const double *a, const double *b, int64_t m) {
         return avx ? dot_avx2(a, b, m) : dot(a, b, m);
     };
-    for (int64_t j0 = 0; j0 < n; j0 += kPanel) {
-        const int64_t j1 = std::min(n, j0 + kPanel);
+    // Right-looking blocked Cholesky, kNB columns per panel: factor the
+    // panel's diagonal block, solve the rows below it against that block,
+    // then subtract the panel's product from the trailing lower triangle
+    // (4 x 8 tiles by the same kernel as the inverse, against the panel
+    // transposed and negated, kGR rows per task so that each 8-column tile
+    // of it is reused from cache).
+    constexpr int64_t kNB = 128, kGR = 32;
+    std::vector<double> Pt;
+    for (int64_t j0 = 0; j0 < n; j0 += kNB) {
+        const int64_t j1 = std::min(n, j0 + kNB), nb = j1 - j0;
         for (int64_t i = j0; i < j1; ++i)
             for (int64_t j = j0; j <= i; ++j) {
-                const double v = P(i, j) - dotv(Lp + i * n, Lp + j * n, j);
+                const double v = Lp[i * n + j] - dotv(Lp + i * n + j0, Lp + j * n + j0, j - j0);
                 if (i == j) {
                     if (!(v > 0.0) || !isfinite(v))
                         return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is not positive definite");
@@ -370,60 +415,57 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
                     Lp[i * n + j] = v / Lp[j * n + j];
                 }
             }
-        // rows below the panel, four at a time (each panel row read once for four)
-        parallel_rows(0, (n - j1 + 3) / 4, nt, [&](int64_t t) {
-            const int64_t i0 = j1 + 4 * t;
-            const int m = (int)std::min<int64_t>(4, n - i0);
-            for (int64_t j = j0; j < j1; ++j) {
-                double acc[4];
-                if (m == 4) {
-                    if (avx) dot4_avx2(Lp + i0 * n, n, Lp + j * n, j, acc);
-                    else dot4(Lp + i0 * n, n, Lp + j * n, j, acc);
-                } else {
-                    for (int r = 0; r < m; ++r) acc[r] = dotv(Lp + (i0 + r) * n, Lp + j * n, j);
+        const int64_t m = n - j1;
+        if (m == 0) break;
+        parallel_rows(j1, n, nt, [&](int64_t i) {
+            double *li = Lp + i * n;
+            for (int64_t j = j0; j < j1; ++j)
+                li[j] = (li[j] - dotv(li + j0, Lp + j * n + j0, j - j0)) / Lp[j * n + j];
+        });
+        // Pt: the panel's rows below j1, negated and transposed, in tiles of 8
+        // columns each contiguous (tile t, term p, column c at (t nb + p) 8 + c;
+        // the last tile padded with zeros)
+        const int64_t m8 = (m + 7) / 8 * 8;
+        Pt.resize((size_t)(nb * m8));
+        parallel_rows(0, m8, nt, [&](int64_t jj) {
+            double *dst = Pt.data() + (jj / 8) * nb * 8 + jj % 8;
+            if (jj >= m) {
+                for (int64_t p = 0; p < nb; ++p) dst[p * 8] = 0.0;
+                return;
+            }
+            const double *lj = Lp + (j1 + jj) * n + j0;
+            for (int64_t p = 0; p < nb; ++p) dst[p * 8] = -lj[p];
+        });
+        const int64_t ng = (m + kGR - 1) / kGR;
+        parallel_rows(0, ng, nt, [&](int64_t t) {
+            const int64_t g0 = j1 + (ng - 1 - t) * kGR;          // largest groups first
+            const int64_t g1 = std::min(n, g0 + kGR);
+            for (int64_t jt = j1; jt < g1; jt += 8) {
+                const double *B = Pt.data() + (jt - j1) * nb;        // tile (jt - j1) / 8
+                for (int64_t i = g0; i < g1; i += 4) {
+                    if (jt > i + 3) continue;                     // tile above the diagonal
+                    if (i + 4 <= g1 && jt + 8 <= n) {
+                        // writes of the tile's entries above the diagonal
+                        // land in L's unread upper triangle
+                        if (avx) gemm4x8_avx2(Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
+                        else gemm4x8(Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
+                    } else {
+                        for (int64_t r = i; r < std::min(i + 4, g1); ++r)
+                            for (int64_t c = jt; c < std::min(jt + 8, r + 1); ++c) {
+                                double v = 0.0;
+                                for (int64_t p = 0; p < nb; ++p) v += Lp[r * n + j0 + p] * B[p * 8 + (c - jt)];
+                                Lp[r * n + c] += v;
+                            }
+                    }
                 }
-                for (int r = 0; r < m; ++r) Lp[(i0 + r) * n + j] = (P(i0 + r, j) - acc[r]) / Lp[j * n + j];
             }
         });
     }
-    // columns c0..c0+3 of L^-1 together by forward substitution, rows four
-    // at a time (each row of L read once for four columns; x_t[p] = 0 above
-    // the diagonal), written reversed into U: U[n-1-i][n-1-c] = (L^-1)[i][c]
-    std::fill(U_out, U_out + (size_t)n * n, 0.0);
-    parallel_rows(0, (n + 3) / 4, nt, [&](int64_t blk) {
-        const int64_t c0 = blk * 4;
-        const int mc = (int)std::min<int64_t>(4, n - c0);
-        std::vector<double> x((size_t)(n - c0) * 4, 0.0);
-        double acc[16];
-        for (int64_t i0 = c0; i0 < n; i0 += 4) {
-            const int m = (int)std::min<int64_t>(4, n - i0);
-            if (m == 4) {
-                if (avx) acc4x4_avx2(Lp, n, i0, c0, i0, x.data(), acc);
-                else acc4x4(Lp, n, i0, c0, i0, x.data(), acc);
-            } else {
-                for (int r = 0; r < 16; ++r) acc[r] = 0.0;
-                for (int r = 0; r < m; ++r)
-                    for (int64_t p = c0; p < i0; ++p)
-                        for (int t = 0; t < 4; ++t) acc[4 * r + t] += Lp[(i0 + r) * n + p] * x[(size_t)((p - c0) * 4 + t)];
-            }
-            for (int r = 0; r < m; ++r) {
-                const int64_t i = i0 + r;
-                const double *li = Lp + i * n;
-                double *a = acc + 4 * r;
-                for (int64_t p = i0; p < i; ++p)
-                    for (int t = 0; t < 4; ++t) a[t] += li[p] * x[(size_t)((p - c0) * 4 + t)];
-                double *xi = x.data() + (i - c0) * 4;
-                for (int t = 0; t < mc; ++t) {
-                    const int64_t c = c0 + t;
-                    xi[t] = i < c ? 0.0 : i == c ? 1.0 / li[i] : -a[t] / li[i];
-                }
-            }
-        }
-        for (int t = 0; t < mc; ++t) {
-            const int64_t c = c0 + t;
-            for (int64_t i = c; i < n; ++i) U_out[(n - 1 - i) * n + (n - 1 - c)] = x[(size_t)((i - c0) * 4 + t)];
-        }
-    });
+    // M = L^-1 into U_out, then U = J M J: the 180-degree rotation of the
+    // matrix, i.e. the flat array reversed
+    parallel_rows(0, n, nt, [&](int64_t i) { std::fill(U_out + i * n, U_out + (i + 1) * n, 0.0); });
+    invert_lower(Lp, n, U_out, nt, avx);
+    std::reverse(U_out, U_out + (size_t)n * n);
     for (int64_t i = 0; i < n; ++i)
         if (!(U_out[i * n + i] > 0.0) || !isfinite(U_out[i * n + i])) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is too ill-conditioned to invert");
     return MQ_OK;

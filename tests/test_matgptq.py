@@ -52,7 +52,7 @@ def test_thread_count_does_not_change_the_result():
         assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
 
 
-@pytest.mark.parametrize("K", [1, 7, 128, 300])
+@pytest.mark.parametrize("K", [1, 7, 128, 300, 700])
 def test_prepare_agrees_with_the_oracle(K):
     H = _H(K, 31 + K)
     U = mq.matgptq_prepare(H, damp=0.01)
@@ -189,7 +189,7 @@ def test_portable_loops_agree_with_the_oracle():
         "import numpy as np, sys; sys.path[:0] = %r\n"
         "import oracle, nested_bit_weight_b200 as mq\n"
         "rng = np.random.default_rng(5)\n"
-        "for K in (3, 130, 257):\n"
+        "for K in (3, 130, 257, 521):\n"
         "    X = rng.standard_normal((2 * K, K)); H = X.T @ X / (2 * K)\n"
         "    U = mq.matgptq_prepare(H); ref = oracle.matgptq_prepare(H)\n"
         "    assert np.allclose(U, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max()), K\n"
