@@ -52,6 +52,22 @@ struct Objective {
             for (int q = 0; q < 256; ++q) levels[(size_t)i * 256 + q] = level_of(q, rs[i]);
     }
 
+    // (codes with s v_i(q) <= w, codes with s v_i(q) < w) for s > 0: the
+    // count of width r's levels (blocks of 2^(8-r) equal codes) below w
+    // estimated from w / s and then settled by exact comparisons with the
+    // rounded products, so the counts are those a search over sv would give
+    void counts(int i, const double *svi, double w, double inv_s, int &le, int &lt) const {
+        const int r = rs[i], step = 1 << (8 - r), nblk = 1 << r;
+        const double x = (w * inv_s - levels[(size_t)i * 256]) / step + 1.0;
+        int j = x > 0.0 ? (x < nblk ? (int)x : nblk) : 0;   // NaN -> 0
+        while (j < nblk && svi[j * step] <= w) ++j;
+        while (j > 0 && svi[(j - 1) * step] > w) --j;
+        int k = j;
+        while (k > 0 && svi[(k - 1) * step] >= w) --k;
+        le = j * step;
+        lt = k * step;
+    }
+
     // sv[i][q] = s * v_i(q) for one scale s (non-decreasing in q for s >= 0)
     void products(double s, double *sv) const {
         for (int i = 0; i < nr * 256; ++i) sv[i] = s * levels[(size_t)i];
@@ -76,13 +92,21 @@ struct Objective {
     // below its value on [min(a, b), max(a, b)], a = min A_i, b = max B_i,
     // outside it, and the first minimum lies inside it or, when the cost is
     // flat at the window's left end, further left by equal steps.
-    int best_code(double w, const double *sv) const {
+    // inv_s = 1 / s when s > 0 (a hint for locating A_i and B_i), else 0.
+    int best_code(double w, const double *sv, double inv_s) const {
         int a = 256, b = -1;
         for (int i = 0; i < nr; ++i) {
             if (!(lams[i] > 0.0)) continue;          // a zero term is flat everywhere
             const double *p = sv + i * 256;
-            a = std::min(a, (int)(std::upper_bound(p, p + 256, w) - p) - 1);
-            b = std::max(b, (int)(std::lower_bound(p, p + 256, w) - p));
+            int le, lt;
+            if (inv_s > 0.0) {
+                counts(i, p, w, inv_s, le, lt);
+            } else {
+                le = (int)(std::upper_bound(p, p + 256, w) - p);
+                lt = (int)(std::lower_bound(p, p + 256, w) - p);
+            }
+            a = std::min(a, le - 1);
+            b = std::max(b, lt);
         }
         const int q0 = std::max(0, std::min(a, b)), q1 = std::min(255, std::max(a, b));
         int best = q0;
@@ -311,7 +335,7 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
     const bool avx = have_avx2_fma();
     const int64_t G = K / 128, nb = n1 - n0;
     const size_t nsv = (size_t)obj.nr * 256;
-    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)nb);
+    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)nb), inv_s((size_t)nb);
     for (int64_t b = 0; b < nb; ++b)
         for (int64_t k = 0; k < K; ++k) w[(size_t)(b * K + k)] = (double)W[(n0 + b) * K + k];
     for (int64_t g = 0; g < G; ++g) {
@@ -324,11 +348,12 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
             const double base = mx / 127.5;
             double best_a = 0.0, best_t = 0.0;
             for (int ia = 0; ia < na; ++ia) {
-                obj.products(base * alphas[ia], svb);
+                const double st = base * alphas[ia], inv = st > 0.0 ? 1.0 / st : 0.0;
+                obj.products(st, svb);
                 double t = 0.0;
                 for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
                     const double x = wb[k];
-                    const int q = obj.best_code(x, svb);
+                    const int q = obj.best_code(x, svb, inv);
                     for (int i = 0; i < obj.nr; ++i) {
                         const double d = x - svb[(size_t)i * 256 + q];
                         t += obj.lams[i] * d * d;
@@ -342,12 +367,13 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
             const double s = base * best_a;
             scales[(n0 + b) * G + g] = (float)s;
             obj.products(s, svb);
+            inv_s[(size_t)b] = s > 0.0 ? 1.0 / s : 0.0;
         }
         for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
             for (int64_t b = 0; b < nb; ++b) {
                 const double *svb = sv.data() + nsv * (size_t)b;
                 const double x = w[(size_t)(b * K + k)];
-                const int q = obj.best_code(x, svb);
+                const int q = obj.best_code(x, svb, inv_s[(size_t)b]);
                 codes[(n0 + b) * K + k] = (uint8_t)q;
                 double e = 0.0;
                 for (int i = 0; i < obj.nr; ++i) e += obj.lams[i] * (x - svb[(size_t)i * 256 + q]);
