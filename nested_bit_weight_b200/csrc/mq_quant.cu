@@ -330,12 +330,70 @@ __attribute__((target("avx2"))) void feedback_avx2(double *w, const double *u, d
     for (; j < j1; ++j) w[j] -= f * u[j];
 }
 
+// The feedback of one group's 128 columns (factors F[b][k], U's rows of the
+// group from Ug, row stride K) to the columns j0..K-1 of nb rows of w:
+// w[b][j] -= F[b][k] U[k][j] for k = 0..127 in order, each a rounded product
+// and a rounded difference.  By tiles of 16 columns, all rows against the
+// same tile of U (held in the L1 cache).
+constexpr int64_t kFbTile = 16;
+
+inline void feedback_group(double *w, int64_t nb, int64_t K, const double *Ug, const double *F, int64_t j0) {
+    for (int64_t jt = j0; jt < K; jt += kFbTile) {
+        const int64_t je = std::min(K, jt + kFbTile);
+        for (int64_t b = 0; b < nb; ++b) {
+            double *wb = w + b * K;
+            for (int64_t k = 0; k < 128; ++k) {
+                const double fk = F[b * 128 + k];
+                const double *u = Ug + k * K;
+                for (int64_t j = jt; j < je; ++j) wb[j] -= fk * u[j];
+            }
+        }
+    }
+}
+
+__attribute__((target("avx2"))) void feedback_group_avx2(double *w, int64_t nb, int64_t K, const double *Ug,
+                                                        const double *F, int64_t j0) {
+    static_assert(kFbTile == 16, "four vectors of four per row");
+    alignas(32) double ut[128 * kFbTile];     // the tile of U, contiguous (one page walk per row of U)
+    int64_t jt = j0;
+    for (; jt + kFbTile <= K; jt += kFbTile) {
+        for (int64_t k = 0; k < 128; ++k)
+            for (int64_t c = 0; c < kFbTile; ++c) ut[k * kFbTile + c] = Ug[k * K + jt + c];
+        for (int64_t b = 0; b < nb; ++b) {
+            double *wb = w + b * K + jt;
+            __m256d w0 = _mm256_loadu_pd(wb), w1 = _mm256_loadu_pd(wb + 4), w2 = _mm256_loadu_pd(wb + 8),
+                    w3 = _mm256_loadu_pd(wb + 12);
+            const double *Fb = F + b * 128;
+            for (int64_t k = 0; k < 128; ++k) {
+                const __m256d fk = _mm256_set1_pd(Fb[k]);
+                const double *u = ut + k * kFbTile;
+                w0 = _mm256_sub_pd(w0, _mm256_mul_pd(fk, _mm256_loadu_pd(u)));
+                w1 = _mm256_sub_pd(w1, _mm256_mul_pd(fk, _mm256_loadu_pd(u + 4)));
+                w2 = _mm256_sub_pd(w2, _mm256_mul_pd(fk, _mm256_loadu_pd(u + 8)));
+                w3 = _mm256_sub_pd(w3, _mm256_mul_pd(fk, _mm256_loadu_pd(u + 12)));
+            }
+            _mm256_storeu_pd(wb, w0);
+            _mm256_storeu_pd(wb + 4, w1);
+            _mm256_storeu_pd(wb + 8, w2);
+            _mm256_storeu_pd(wb + 12, w3);
+        }
+    }
+    if (jt < K) {
+        for (int64_t b = 0; b < nb; ++b)
+            for (int64_t k = 0; k < 128; ++k) {
+                const double fk = F[b * 128 + k];
+                const double *u = Ug + k * K;
+                for (int64_t j = jt; j < K; ++j) w[b * K + j] -= fk * u[j];
+            }
+    }
+}
+
 void quantize_rows(const float *W, int64_t K, const double *U, const Objective &obj, const double *alphas,
                    int na, double lsum, int64_t n0, int64_t n1, uint8_t *codes, float *scales) {
     const bool avx = have_avx2_fma();
     const int64_t G = K / 128, nb = n1 - n0;
     const size_t nsv = (size_t)obj.nr * 256;
-    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)nb), inv_s((size_t)nb);
+    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)(nb * 128)), inv_s((size_t)nb);
     for (int64_t b = 0; b < nb; ++b)
         for (int64_t k = 0; k < K; ++k) w[(size_t)(b * K + k)] = (double)W[(n0 + b) * K + k];
     for (int64_t g = 0; g < G; ++g) {
@@ -369,7 +427,12 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
             obj.products(s, svb);
             inv_s[(size_t)b] = s > 0.0 ? 1.0 / s : 0.0;
         }
-        for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
+        // the group's columns in order; each column's feedback reaches the
+        // rest of the group at once and the later groups' columns after the
+        // group (below): every weight still takes the updates of all earlier
+        // columns one at a time in column order, before anything reads it
+        const int64_t ge = 128 * g + 128;
+        for (int64_t k = 128 * g; k < ge; ++k) {
             for (int64_t b = 0; b < nb; ++b) {
                 const double *svb = sv.data() + nsv * (size_t)b;
                 const double x = w[(size_t)(b * K + k)];
@@ -378,13 +441,18 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
                 double e = 0.0;
                 for (int i = 0; i < obj.nr; ++i) e += obj.lams[i] * (x - svb[(size_t)i * 256 + q]);
                 e /= lsum;
-                f[(size_t)b] = e / U[k * K + k];
+                f[(size_t)(b * 128 + (k - 128 * g))] = e / U[k * K + k];
             }
             const double *urow = U + k * K;
             for (int64_t b = 0; b < nb; ++b) {
-                if (avx) feedback_avx2(w.data() + b * K, urow, f[(size_t)b], k + 1, K);
-                else feedback(w.data() + b * K, urow, f[(size_t)b], k + 1, K);
+                const double fb = f[(size_t)(b * 128 + (k - 128 * g))];
+                if (avx) feedback_avx2(w.data() + b * K, urow, fb, k + 1, ge);
+                else feedback(w.data() + b * K, urow, fb, k + 1, ge);
             }
+        }
+        if (ge < K) {
+            if (avx) feedback_group_avx2(w.data(), nb, K, U + 128 * g * K, f.data(), ge);
+            else feedback_group(w.data(), nb, K, U + 128 * g * K, f.data(), ge);
         }
     }
 }
