@@ -201,3 +201,15 @@ def test_portable_loops_agree_with_the_oracle():
     env = dict(os.environ, MQ_PORTABLE_HOST="1")
     out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stderr
+
+
+def test_many_groups_and_a_ragged_row_block_match_the_oracle():
+    # five groups (each group's feedback reaches the later groups after it)
+    # and 17 rows (a full block of 16 plus one)
+    N, K = 17, 640
+    U = oracle.matgptq_prepare(_H(K, 101))
+    W = _W(N, K, 102)
+    c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U, alphas=(1.0, 0.85))
+    codes, scales = mq.matgptq_quantize(W, U, alphas=(1.0, 0.85))
+    assert np.array_equal(codes, c_ref)
+    assert np.array_equal(scales, s_ref.astype(np.float32))
