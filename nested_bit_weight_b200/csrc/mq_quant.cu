@@ -307,10 +307,10 @@ void invert_lower(const double *L, int64_t n, double *M, int nt, bool avx) {
     }
 }
 
-// Rows n0..n1-1 (at most kRowBlock), column by column together: each row of
-// U is then read once per block of rows rather than once per row (the
-// feedback streams U's upper triangle for every column).  Every row still
-// takes exactly the operations, in the order, of quantizing it alone.
+// Rows n0..n1-1 (at most kRowBlock), column by column together: each tile of
+// U that the feedback reads then serves a block of rows rather than one row.
+// Every row still takes exactly the operations, in the order, of quantizing
+// it alone.
 constexpr int64_t kRowBlock = 16;
 
 // w[j] -= f u[j] for j0 <= j < j1: one rounded product and one rounded
@@ -333,8 +333,9 @@ __attribute__((target("avx2"))) void feedback_avx2(double *w, const double *u, d
 // The feedback of one group's 128 columns (factors F[b][k], U's rows of the
 // group from Ug, row stride K) to the columns j0..K-1 of nb rows of w:
 // w[b][j] -= F[b][k] U[k][j] for k = 0..127 in order, each a rounded product
-// and a rounded difference.  By tiles of 16 columns, all rows against the
-// same tile of U (held in the L1 cache).
+// and a rounded difference.  By tiles of 16 columns: the tile of U copied to
+// a contiguous buffer (its 128 rows lie a row of U apart), then each row's
+// 16 weights held in registers through the 128 updates.
 constexpr int64_t kFbTile = 16;
 
 inline void feedback_group(double *w, int64_t nb, int64_t K, const double *Ug, const double *F, int64_t j0) {
