@@ -360,7 +360,38 @@ __attribute__((target("avx2"))) void feedback_group_avx2(double *w, int64_t nb, 
     for (; jt + kFbTile <= K; jt += kFbTile) {
         for (int64_t k = 0; k < 128; ++k)
             for (int64_t c = 0; c < kFbTile; ++c) ut[k * kFbTile + c] = Ug[k * K + jt + c];
-        for (int64_t b = 0; b < nb; ++b) {
+        int64_t b = 0;
+        for (; b + 2 <= nb; b += 2) {                 // two rows: eight independent chains
+            double *wa = w + b * K + jt, *wc = wa + K;
+            __m256d a0 = _mm256_loadu_pd(wa), a1 = _mm256_loadu_pd(wa + 4), a2 = _mm256_loadu_pd(wa + 8),
+                    a3 = _mm256_loadu_pd(wa + 12);
+            __m256d c0 = _mm256_loadu_pd(wc), c1 = _mm256_loadu_pd(wc + 4), c2 = _mm256_loadu_pd(wc + 8),
+                    c3 = _mm256_loadu_pd(wc + 12);
+            const double *Fa = F + b * 128, *Fc = Fa + 128;
+            for (int64_t k = 0; k < 128; ++k) {
+                const __m256d fa = _mm256_set1_pd(Fa[k]), fc = _mm256_set1_pd(Fc[k]);
+                const double *u = ut + k * kFbTile;
+                const __m256d u0 = _mm256_load_pd(u), u1 = _mm256_load_pd(u + 4), u2 = _mm256_load_pd(u + 8),
+                              u3 = _mm256_load_pd(u + 12);
+                a0 = _mm256_sub_pd(a0, _mm256_mul_pd(fa, u0));
+                c0 = _mm256_sub_pd(c0, _mm256_mul_pd(fc, u0));
+                a1 = _mm256_sub_pd(a1, _mm256_mul_pd(fa, u1));
+                c1 = _mm256_sub_pd(c1, _mm256_mul_pd(fc, u1));
+                a2 = _mm256_sub_pd(a2, _mm256_mul_pd(fa, u2));
+                c2 = _mm256_sub_pd(c2, _mm256_mul_pd(fc, u2));
+                a3 = _mm256_sub_pd(a3, _mm256_mul_pd(fa, u3));
+                c3 = _mm256_sub_pd(c3, _mm256_mul_pd(fc, u3));
+            }
+            _mm256_storeu_pd(wa, a0);
+            _mm256_storeu_pd(wa + 4, a1);
+            _mm256_storeu_pd(wa + 8, a2);
+            _mm256_storeu_pd(wa + 12, a3);
+            _mm256_storeu_pd(wc, c0);
+            _mm256_storeu_pd(wc + 4, c1);
+            _mm256_storeu_pd(wc + 8, c2);
+            _mm256_storeu_pd(wc + 12, c3);
+        }
+        for (; b < nb; ++b) {
             double *wb = w + b * K + jt;
             __m256d w0 = _mm256_loadu_pd(wb), w1 = _mm256_loadu_pd(wb + 4), w2 = _mm256_loadu_pd(wb + 8),
                     w3 = _mm256_loadu_pd(wb + 12);
