@@ -660,7 +660,12 @@ def main():
     ap.add_argument("--case", default=None, help="N,K,M,r: one layer, eager launches (for ncu)")
     ap.add_argument("--sweep", default=None, help="config indices (e.g. 0,1,2) or 'all': "
                                                   "per-(layer, M, r) isolated timings")
+    ap.add_argument("--quantizer", action="store_true",
+                    help="host only: time the one-shot quantizer on the Llama-3.1-8B shapes")
     args = ap.parse_args()
+    if args.quantizer:
+        run_quantizer()
+        return
     if args.case:
         run_case(args)
         return
@@ -680,6 +685,34 @@ def main():
     if ws_n > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+# The pages' complete MatGPTQ passes over the Llama-3.1-8B shapes (seconds;
+# "MatGPTQ: Efficient and Accurate Inference over Nested Quantized Models",
+# appendix Table 3; their machine is not stated): context for the host times.
+PAGES_MATGPTQ_PASS_S = {"k_proj": 3.59, "q_proj": 3.59, "gate_proj": 6.58, "down_proj": 12.45}
+
+
+def run_quantizer():
+    """One JSON line per shape: the one-shot quantizer (r = 3, 4, 8, lambda =
+    1, 1, 1, five scale multipliers) on a synthetic AR(1) Hessian, timed on
+    the host around the library calls."""
+    import nested_bit_weight_b200 as mq
+    for i, name in enumerate(("k_proj", "q_proj", "gate_proj", "down_proj")):
+        l = next(x for x in wl.LLAMA8B if x.name == name)
+        H = wl.gen_hessian(l.K, 7000 + i)
+        W = wl.gen_float_weights(l.N, l.K, 7100 + i)
+        t0 = time.perf_counter()
+        U = mq.matgptq_prepare(H)
+        t1 = time.perf_counter()
+        mq.matgptq_quantize(W, U)
+        t2 = time.perf_counter()
+        print(json.dumps({"metric": "quantizer_pass_s", "layer": name, "N": l.N, "K": l.K,
+                          "prepare_s": round(t1 - t0, 2), "quantize_s": round(t2 - t1, 2),
+                          "total_s": round(t2 - t0, 2), "threads": os.cpu_count(),
+                          "pages_matgptq_pass_s": PAGES_MATGPTQ_PASS_S[name],
+                          "higher_is_better": False, "data": "synthetic"}), flush=True)
+        del H, U, W
 
 
 def run_reference(args):

@@ -191,3 +191,32 @@ def gen_scales(N: int, K: int, seed: int, zero_groups: int = 0) -> np.ndarray:
         idx = rng.choice(s.size, size=min(zero_groups, s.size), replace=False)
         s.reshape(-1)[idx] = 0.0
     return s
+
+
+def gen_hessian(K: int, seed: int, corr: float = 0.9, samples: int | None = None) -> np.ndarray:
+    """A layer's Hessian proxy H = X^T X / n (fp64, K x K) from synthetic
+    calibration inputs: n = samples (default K + 1024) rows whose K columns
+    follow an AR(1) process with coefficient `corr` (neighbouring input
+    channels correlated, as activations are), unit variance.  Inputs only:
+    the quantizer's own arithmetic starts from H."""
+    n = samples if samples is not None else K + 1024
+    rng = np.random.default_rng(seed)
+    z = rng.standard_normal((n, K), dtype=np.float32)
+    X = np.empty_like(z)
+    X[:, 0] = z[:, 0]
+    c, d = np.float32(corr), np.float32(np.sqrt(1.0 - corr * corr))
+    for k in range(1, K):
+        X[:, k] = c * X[:, k - 1] + d * z[:, k]
+    X64 = X.astype(np.float64)
+    return X64.T @ X64 / n
+
+
+def gen_float_weights(N: int, K: int, seed: int) -> np.ndarray:
+    """Float weights to quantize (fp32, N x K): N(0, 0.02^2) with the same
+    outlier recipe as gen_weights (1 % of entries x10)."""
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    n_out = int(0.01 * N * K)
+    idx = rng.choice(N * K, size=n_out, replace=False)
+    W.reshape(-1)[idx] *= np.float32(10.0)
+    return W
