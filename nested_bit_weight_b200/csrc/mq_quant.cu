@@ -566,10 +566,14 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
         parallel_rows(0, ng, nt, [&](int64_t t) {
             const int64_t g0 = j1 + (ng - 1 - t) * kGR;          // largest groups first
             const int64_t g1 = std::min(n, g0 + kGR);
-            for (int64_t jt = j1; jt < g1; jt += 8) {
-                const double *B = Pt.data() + (jt - j1) * nb;        // tile (jt - j1) / 8
-                for (int64_t i = g0; i < g1; i += 4) {
-                    if (jt > i + 3) continue;                     // tile above the diagonal
+            // chunks of kCC columns (their panel tiles stay in cache), each
+            // row tile of the group running along the chunk
+            constexpr int64_t kCC = 64;
+            for (int64_t jc = j1; jc < g1; jc += kCC)
+            for (int64_t i = g0; i < g1; i += 4) {
+                for (int64_t jt = jc; jt < std::min(g1, jc + kCC); jt += 8) {
+                    if (jt > i + 3) break;                        // the rest lies above the diagonal
+                    const double *B = Pt.data() + (jt - j1) * nb;    // tile (jt - j1) / 8
                     if (i + 4 <= g1 && jt + 8 <= n) {
                         // writes of the tile's entries above the diagonal
                         // land in L's unread upper triangle
