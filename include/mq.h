@@ -248,9 +248,10 @@ MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int 
  * weighting of the widths).  All pointers are host memory.
  *   mq_matgptq_prepare: U_out (K x K) upper triangular with
  *     U^T U = (H + damp * mean(diag H) * I)^-1, by one blocked Cholesky
- *     factorisation and one blocked triangular inverse (threads; AVX2 and
- *     FMA when the CPU has them, else portable loops, or always with
- *     MQ_PORTABLE_HOST=1 in the environment: the two round differently, within
+ *     factorisation and one blocked triangular inverse (threads; AVX-512 or
+ *     AVX2 with FMA when the CPU has them, else portable loops; in the
+ *     environment MQ_PORTABLE_HOST=1 forces the portable loops and
+ *     MQ_NO_AVX512=1 stops at AVX2: the paths round differently, within
  *     ~1e-15 relative).  Holds one K x K work buffer besides U_out.
  *   mq_matgptq_quantize: per 128-column group, when its first column is
  *     reached, a row's scale is alpha * max|w| / 127.5 over the group's

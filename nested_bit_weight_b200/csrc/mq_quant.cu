@@ -179,15 +179,33 @@ inline void gemm4x8(const double *A, int64_t lda, const double *B, int64_t ldb, 
         for (int c = 0; c < 8; ++c) T[r * ldt + c] = acc[r][c];
 }
 
-// The same kernels with AVX2 and FMA, used by the prepare step when
-// the CPU has both (rounding differs from the portable loops within the
-// prepare step's own error; the code search never uses them).
-// (MQ_PORTABLE_HOST=1 in the environment selects the portable loops.)
-bool have_avx2_fma() {
-    static const bool ok = (__builtin_cpu_init(), __builtin_cpu_supports("avx2")) && __builtin_cpu_supports("fma") &&
-                           !(getenv("MQ_PORTABLE_HOST") && getenv("MQ_PORTABLE_HOST")[0] == '1');
-    return ok;
+// The same kernels with AVX2 and FMA (and the tile product with AVX-512),
+// used by the prepare step when the CPU has them (rounding differs from the
+// portable loops within the prepare step's own error; the code search never
+// uses them).  MQ_PORTABLE_HOST=1 in the environment selects the portable
+// loops, MQ_NO_AVX512=1 stops at AVX2.
+enum class Simd { portable, avx2, avx512 };
+
+bool env_set(const char *name) {
+    const char *v = getenv(name);
+    return v && v[0] == '1';
 }
+
+Simd host_simd() {
+    static const Simd s = [] {
+        __builtin_cpu_init();
+        if (env_set("MQ_PORTABLE_HOST") || !__builtin_cpu_supports("avx2") || !__builtin_cpu_supports("fma"))
+            return Simd::portable;
+        if (!env_set("MQ_NO_AVX512") && __builtin_cpu_supports("avx512f")) return Simd::avx512;
+        return Simd::avx2;
+    }();
+    return s;
+}
+
+bool have_avx2_fma() { return host_simd() != Simd::portable; }
+
+// rows of A (and of T) per call of the tile product: 8 with AVX-512, else 4
+inline int64_t tile_rows(Simd s) { return s == Simd::avx512 ? 8 : 4; }
 
 __attribute__((target("avx2,fma"))) inline double hsum(__m256d v) {
     alignas(32) double t[4];
@@ -242,6 +260,42 @@ __attribute__((target("avx2,fma"))) void gemm4x8_avx2(const double *A, int64_t l
     _mm256_storeu_pd(T + 3 * ldt + 4, t31);
 }
 
+__attribute__((target("avx512f"))) void gemm8x8_avx512(const double *A, int64_t lda, const double *B,
+                                                       int64_t ldb, int64_t p0, int64_t p1, double *T,
+                                                       int64_t ldt) {
+    __m512d t0 = _mm512_loadu_pd(T), t1 = _mm512_loadu_pd(T + ldt), t2 = _mm512_loadu_pd(T + 2 * ldt),
+            t3 = _mm512_loadu_pd(T + 3 * ldt), t4 = _mm512_loadu_pd(T + 4 * ldt),
+            t5 = _mm512_loadu_pd(T + 5 * ldt), t6 = _mm512_loadu_pd(T + 6 * ldt),
+            t7 = _mm512_loadu_pd(T + 7 * ldt);
+    for (int64_t p = p0; p < p1; ++p) {
+        const __m512d b = _mm512_loadu_pd(B + p * ldb);
+        t0 = _mm512_fmadd_pd(_mm512_set1_pd(A[p]), b, t0);
+        t1 = _mm512_fmadd_pd(_mm512_set1_pd(A[lda + p]), b, t1);
+        t2 = _mm512_fmadd_pd(_mm512_set1_pd(A[2 * lda + p]), b, t2);
+        t3 = _mm512_fmadd_pd(_mm512_set1_pd(A[3 * lda + p]), b, t3);
+        t4 = _mm512_fmadd_pd(_mm512_set1_pd(A[4 * lda + p]), b, t4);
+        t5 = _mm512_fmadd_pd(_mm512_set1_pd(A[5 * lda + p]), b, t5);
+        t6 = _mm512_fmadd_pd(_mm512_set1_pd(A[6 * lda + p]), b, t6);
+        t7 = _mm512_fmadd_pd(_mm512_set1_pd(A[7 * lda + p]), b, t7);
+    }
+    _mm512_storeu_pd(T, t0);
+    _mm512_storeu_pd(T + ldt, t1);
+    _mm512_storeu_pd(T + 2 * ldt, t2);
+    _mm512_storeu_pd(T + 3 * ldt, t3);
+    _mm512_storeu_pd(T + 4 * ldt, t4);
+    _mm512_storeu_pd(T + 5 * ldt, t5);
+    _mm512_storeu_pd(T + 6 * ldt, t6);
+    _mm512_storeu_pd(T + 7 * ldt, t7);
+}
+
+// T[r][c] += sum_{p0 <= p < p1} A[r][p] B[p][c], r < tile_rows(s), c < 8
+inline void gemm_tile(Simd s, const double *A, int64_t lda, const double *B, int64_t ldb, int64_t p0,
+                      int64_t p1, double *T, int64_t ldt) {
+    if (s == Simd::avx512) gemm8x8_avx512(A, lda, B, ldb, p0, p1, T, ldt);
+    else if (s == Simd::avx2) gemm4x8_avx2(A, lda, B, ldb, p0, p1, T, ldt);
+    else gemm4x8(A, lda, B, ldb, p0, p1, T, ldt);
+}
+
 // M = L^-1 (both n x n row-major, lower triangular; M zero on entry above
 // the diagonal and written everywhere on and below it), by blocks of kRB
 // rows, each after the ones above it:
@@ -249,8 +303,9 @@ __attribute__((target("avx2,fma"))) void gemm4x8_avx2(const double *A, int64_t l
 //   M[I, I] = L[I, I]^-1,
 // the product taken kCW columns per task and kPB terms at a time so that
 // its operands stay in cache.
-void invert_lower(const double *L, int64_t n, double *M, int nt, bool avx) {
+void invert_lower(const double *L, int64_t n, double *M, int nt, Simd simd) {
     constexpr int64_t kRB = 128, kCW = 64, kPB = 256;
+    const int64_t R = tile_rows(simd);
     for (int64_t i0 = 0; i0 < n; i0 += kRB) {
         const int64_t b = std::min(kRB, n - i0);
         parallel_rows(0, (i0 + kCW - 1) / kCW, nt, [&](int64_t task) {
@@ -263,15 +318,14 @@ void invert_lower(const double *L, int64_t n, double *M, int nt, bool avx) {
                 for (int64_t p = pp; p < pe; ++p)
                     std::copy(M + p * n + j0, M + p * n + j0 + w, Bp.data() + (p - pp) * kCW);
                 const double *B = Bp.data() - pp * kCW;   // row p of the block at B + p * kCW
-                for (int64_t r0 = 0; r0 < b; r0 += 4) {
+                for (int64_t r0 = 0; r0 < b; r0 += R) {
                     const double *A = L + (i0 + r0) * n;
                     for (int64_t c0 = 0; c0 < w; c0 += 8) {
                         double *Tt = T.data() + r0 * kCW + c0;
-                        if (r0 + 4 <= b && c0 + 8 <= w) {
-                            if (avx) gemm4x8_avx2(A, n, B + c0, kCW, pp, pe, Tt, kCW);
-                            else gemm4x8(A, n, B + c0, kCW, pp, pe, Tt, kCW);
+                        if (r0 + R <= b && c0 + 8 <= w) {
+                            gemm_tile(simd, A, n, B + c0, kCW, pp, pe, Tt, kCW);
                         } else {
-                            for (int64_t r = 0; r < std::min<int64_t>(4, b - r0); ++r)
+                            for (int64_t r = 0; r < std::min<int64_t>(R, b - r0); ++r)
                                 for (int64_t c = 0; c < std::min<int64_t>(8, w - c0); ++c) {
                                     double v = Tt[r * kCW + c];
                                     for (int64_t p = pp; p < pe; ++p) v += A[r * n + p] * B[p * kCW + c0 + c];
@@ -516,7 +570,9 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
     parallel_rows(0, n, nt, [&](int64_t i) {
         for (int64_t j = 0; j <= i; ++j) Lp[i * n + j] = P(i, j);
     });
-    const bool avx = have_avx2_fma();
+    const Simd simd = host_simd();
+    const bool avx = simd != Simd::portable;
+    const int64_t R = tile_rows(simd);
     auto dotv = [avx](const double *a, const double *b, int64_t m) {
         return avx ? dot_avx2(a, b, m) : dot(a, b, m);
     };
@@ -570,17 +626,16 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
             // row tile of the group running along the chunk
             constexpr int64_t kCC = 64;
             for (int64_t jc = j1; jc < g1; jc += kCC)
-            for (int64_t i = g0; i < g1; i += 4) {
+            for (int64_t i = g0; i < g1; i += R) {
                 for (int64_t jt = jc; jt < std::min(g1, jc + kCC); jt += 8) {
-                    if (jt > i + 3) break;                        // the rest lies above the diagonal
+                    if (jt > i + R - 1) break;                    // the rest lies above the diagonal
                     const double *B = Pt.data() + (jt - j1) * nb;    // tile (jt - j1) / 8
-                    if (i + 4 <= g1 && jt + 8 <= n) {
+                    if (i + R <= g1 && jt + 8 <= n) {
                         // writes of the tile's entries above the diagonal
                         // land in L's unread upper triangle
-                        if (avx) gemm4x8_avx2(Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
-                        else gemm4x8(Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
+                        gemm_tile(simd, Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
                     } else {
-                        for (int64_t r = i; r < std::min(i + 4, g1); ++r)
+                        for (int64_t r = i; r < std::min(i + R, g1); ++r)
                             for (int64_t c = jt; c < std::min(jt + 8, r + 1); ++c) {
                                 double v = 0.0;
                                 for (int64_t p = 0; p < nb; ++p) v += Lp[r * n + j0 + p] * B[p * 8 + (c - jt)];
@@ -594,7 +649,7 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
     // M = L^-1 into U_out, then U = J M J: the 180-degree rotation of the
     // matrix, i.e. the flat array reversed
     parallel_rows(0, n, nt, [&](int64_t i) { std::fill(U_out + i * n, U_out + (i + 1) * n, 0.0); });
-    invert_lower(Lp, n, U_out, nt, avx);
+    invert_lower(Lp, n, U_out, nt, simd);
     std::reverse(U_out, U_out + (size_t)n * n);
     for (int64_t i = 0; i < n; ++i)
         if (!(U_out[i * n + i] > 0.0) || !isfinite(U_out[i * n + i])) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is too ill-conditioned to invert");

@@ -178,10 +178,12 @@ def test_non_finite_weights_are_refused():
             mq.matgptq_quantize(W2, np.eye(128))
 
 
-def test_portable_loops_agree_with_the_oracle():
-    # the portable host loops (selected by MQ_PORTABLE_HOST=1; the default
-    # takes AVX2, and FMA in the prepare step, when the CPU has them), in a
-    # fresh process: prepare within rounding, quantize bit for bit
+@pytest.mark.parametrize("env", ["MQ_PORTABLE_HOST", "MQ_NO_AVX512"])
+def test_other_host_code_paths_agree_with_the_oracle(env):
+    # the portable host loops (MQ_PORTABLE_HOST=1) and the AVX2 ones
+    # (MQ_NO_AVX512=1; the default takes AVX-512 for the prepare step's tile
+    # product where the CPU has it), each in a fresh process: prepare within
+    # rounding, quantize bit for bit
     import os
     import subprocess
     import sys
@@ -198,8 +200,8 @@ def test_portable_loops_agree_with_the_oracle():
         "c, s = mq.matgptq_quantize(W, U); cr, sr = oracle.matgptq_quantize(W.astype(np.float64), U)\n"
         "assert np.array_equal(c, cr) and np.array_equal(s, sr.astype(np.float32))\n"
         "print('ok')\n" % (sys.path,))
-    env = dict(os.environ, MQ_PORTABLE_HOST="1")
-    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=300)
+    out = subprocess.run([sys.executable, "-c", code], env=dict(os.environ, **{env: "1"}),
+                         capture_output=True, text=True, timeout=300)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stderr
 
 
