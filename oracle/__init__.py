@@ -351,3 +351,87 @@ def matgptq_quantize(W, U, rs=(3, 4, 8), lams=(1.0, 1.0, 1.0),
                 e /= lsum
                 W[n, k + 1:] -= (e / U[k, k]) * U[k, k + 1:]
     return codes, scales
+
+
+# ----------------------------- one-shot quantizer, asymmetric variant (R16)
+# The same column loop with the asymmetric levels u_r = 2^(8-r) q_r +
+# 2^(7-r) - z ("MatGPTQ: Efficient and Accurate Inference over Nested
+# Quantized Models", captions of Tables 5-7: the evaluated models are
+# asymmetric MatGPTQ).  Readings: per group and alpha, the grid spans
+# alpha times the group's current range and is centred on it,
+# s = alpha (hi - lo) / 255 and z = 128 - (hi + lo) / (2 s), z taken as
+# stored (fp32, then fp16, RNE); s stays fp64 as in the symmetric loop.  A
+# group whose range is zero, or whose z is not a finite fp16, takes the
+# symmetric grid (s = alpha max|w| / 127.5, z = 128).
+
+def matgptq_asym_grid(lo: float, hi: float, alpha: float):
+    """(s, z16) of one group for one multiplier (fp64; z16 the stored value)."""
+    if hi > lo:
+        s = alpha * (hi - lo) / 255.0
+        z = float(zeros_f16(np.array(128.0 - (hi + lo) / (2.0 * s))))
+        if np.isfinite(z):
+            return s, z
+    return alpha * max(abs(lo), abs(hi)) / 127.5, 128.0
+
+
+def _level_all_asym(r: int, z: float) -> np.ndarray:
+    """The asymmetric r-bit level of every 8-bit code 0..255."""
+    return level_asym(np.arange(256) >> (8 - r), r, z)
+
+
+def matgptq_best_code_asym(w: float, s: float, z: float, rs, lams) -> int:
+    """argmin over q of sum_r lambda_r (w - s u_r(q >> (8-r), z))^2."""
+    cost = np.zeros(256)
+    for r, lam in zip(rs, lams):
+        d = w - s * _level_all_asym(r, z)
+        cost += lam * d * d
+    return int(np.argmin(cost))
+
+
+def matgptq_quantize_asym(W, U, rs=(3, 4, 8), lams=(1.0, 1.0, 1.0),
+                          alphas=(1.0, 0.95, 0.9, 0.85, 0.8)):
+    """codes uint8 [N, K], scales fp64 [N, K/128], zero points [N, K/128]
+    (the stored fp16 values, as fp64) by the column loop with asymmetric
+    levels."""
+    W = np.array(W, np.float64, copy=True)
+    U = np.asarray(U, np.float64)
+    N, K = W.shape
+    G = K // 128
+    lsum = float(sum(lams))
+    codes = np.zeros((N, K), np.uint8)
+    scales = np.zeros((N, G), np.float64)
+    zeros = np.zeros((N, G), np.float64)
+
+    def slice_err(w, s, z, q):
+        out = []
+        for r in rs:
+            out.append(w - s * float(level_asym(np.array(q >> (8 - r)), r, z)))
+        return out
+
+    for g in range(G):
+        cols = range(128 * g, 128 * g + 128)
+        for n in range(N):
+            seg = W[n, 128 * g:128 * g + 128]
+            lo, hi = float(np.min(seg)), float(np.max(seg))
+            best = None
+            for a in alphas:
+                s, z = matgptq_asym_grid(lo, hi, a)
+                t = 0.0
+                for k in cols:
+                    q = matgptq_best_code_asym(W[n, k], s, z, rs, lams)
+                    for lam, d in zip(lams, slice_err(W[n, k], s, z, q)):
+                        t += lam * d * d
+                if best is None or t < best[0]:
+                    best = (t, s, z)
+            scales[n, g], zeros[n, g] = best[1], best[2]
+        for k in cols:
+            for n in range(N):
+                s, z = scales[n, g], zeros[n, g]
+                q = matgptq_best_code_asym(W[n, k], s, z, rs, lams)
+                codes[n, k] = q
+                e = 0.0
+                for lam, d in zip(lams, slice_err(W[n, k], s, z, q)):
+                    e += lam * d
+                e /= lsum
+                W[n, k + 1:] -= (e / U[k, k]) * U[k, k + 1:]
+    return codes, scales, zeros
