@@ -275,6 +275,22 @@ MQ_API mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const
                                      const double *alphas, int n_alpha, int threads,
                                      uint8_t *codes_out, float *scales_out);
 
+/*
+ * The same with the asymmetric levels u_r = 2^(8-r) q_r + 2^(7-r) - z (the
+ * variant the pages evaluate: "MatGPTQ: Efficient and Accurate Inference over
+ * Nested Quantized Models", captions of Tables 5-7).  Per group and alpha the
+ * grid spans alpha times the group's current range [lo, hi], centred on it:
+ * s = alpha (hi - lo) / 255, z = 128 - (hi + lo) / (2 s), z rounded as stored
+ * (to fp32, then fp16, nearest-even); a group of zero range, or whose z is no
+ * finite fp16, takes the symmetric grid (s = alpha max|w| / 127.5, z = 128).
+ * zeros_out N x (K/128) fp32 holds those fp16 values (the input of
+ * mq_pack_zeros); the rest as mq_matgptq_quantize.
+ */
+MQ_API mq_status mq_matgptq_quantize_asym(const float *W, int64_t N, int64_t K, const double *U,
+                                          const int32_t *rs, const double *lambdas, int n_r,
+                                          const double *alphas, int n_alpha, int threads,
+                                          uint8_t *codes_out, float *scales_out, float *zeros_out);
+
 /* Kernels for M <= 8 (both compute the same Y within the stated tolerance). */
 enum {
     MQ_GEMV_TC = 0,        /* default: 128 rows per tensor-core MMA, int8 operands,

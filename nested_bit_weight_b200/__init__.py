@@ -86,6 +86,7 @@ def _load() -> ctypes.CDLL:
                                    ctypes.POINTER(I), ctypes.POINTER(ctypes.c_double)]),
         "mq_matgptq_prepare": (I, [P, I64, ctypes.c_double, P]),
         "mq_matgptq_quantize": (I, [P, I64, I64, P, P, P, I, P, I, I, P, P]),
+        "mq_matgptq_quantize_asym": (I, [P, I64, I64, P, P, P, I, P, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -308,10 +309,12 @@ def matgptq_prepare(H, damp: float = 0.01):
 
 
 def matgptq_quantize(W, U, rs=(3, 4, 8), lambdas=(1.0, 1.0, 1.0),
-                     alphas=(1.0, 0.95, 0.9, 0.85, 0.8), threads: int = 0):
+                     alphas=(1.0, 0.95, 0.9, 0.85, 0.8), threads: int = 0, asymmetric: bool = False):
     """(codes uint8 N x K, scales fp32 N x K/128): the parent codes of the
     nested format from float weights W by the multi-precision column loop
-    (mq_matgptq_quantize, host; the inputs of pack_parent)."""
+    (mq_matgptq_quantize, host; the inputs of pack_parent).  asymmetric=True:
+    (codes, scales, zeros) by mq_matgptq_quantize_asym (zeros: the input of
+    pack_parent's `zeros`)."""
     import numpy as np
     W = np.ascontiguousarray(W, np.float32)
     U = np.ascontiguousarray(U, np.float64)
@@ -325,9 +328,13 @@ def matgptq_quantize(W, U, rs=(3, 4, 8), lambdas=(1.0, 1.0, 1.0),
     al_a = np.ascontiguousarray(alphas, np.float64)
     codes = np.empty((N, K), np.uint8)
     scales = np.empty((N, max(K // 128, 1)), np.float32)
-    _check(lib.mq_matgptq_quantize(W.ctypes.data, N, K, U.ctypes.data, rs_a.ctypes.data,
-                                   lam_a.ctypes.data, len(rs_a), al_a.ctypes.data, len(al_a),
-                                   int(threads), codes.ctypes.data, scales.ctypes.data))
+    args = (W.ctypes.data, N, K, U.ctypes.data, rs_a.ctypes.data, lam_a.ctypes.data, len(rs_a),
+            al_a.ctypes.data, len(al_a), int(threads), codes.ctypes.data, scales.ctypes.data)
+    if asymmetric:
+        zeros = np.empty_like(scales)
+        _check(lib.mq_matgptq_quantize_asym(*args, zeros.ctypes.data))
+        return codes, scales, zeros
+    _check(lib.mq_matgptq_quantize(*args))
     return codes, scales
 
 

@@ -22,6 +22,7 @@
 #include <stdlib.h>
 
 #include <algorithm>
+#include <cmath>
 #include <atomic>
 #include <memory>
 #include <thread>
@@ -56,9 +57,9 @@ struct Objective {
     // count of width r's levels (blocks of 2^(8-r) equal codes) below w
     // estimated from w / s and then settled by exact comparisons with the
     // rounded products, so the counts are those a search over sv would give
-    void counts(int i, const double *svi, double w, double inv_s, int &le, int &lt) const {
+    void counts(int i, const double *svi, double w, double inv_s, double off, int &le, int &lt) const {
         const int r = rs[i], step = 1 << (8 - r), nblk = 1 << r;
-        const double x = (w * inv_s - levels[(size_t)i * 256]) / step + 1.0;
+        const double x = (w * inv_s - (levels[(size_t)i * 256] + off)) / step + 1.0;
         int j = x > 0.0 ? (x < nblk ? (int)x : nblk) : 0;   // NaN -> 0
         while (j < nblk && svi[j * step] <= w) ++j;
         while (j > 0 && svi[(j - 1) * step] > w) --j;
@@ -69,8 +70,11 @@ struct Objective {
     }
 
     // sv[i][q] = s * v_i(q) for one scale s (non-decreasing in q for s >= 0)
-    void products(double s, double *sv) const {
-        for (int i = 0; i < nr * 256; ++i) sv[i] = s * levels[(size_t)i];
+    // sv[i][q] = s * (v_i(q) + off) for one scale s >= 0 and level offset
+    // off = 128 - z (0 for the symmetric levels; v_i(q) + off is exact, so
+    // each product is the level's one rounding), non-decreasing in q
+    void products(double s, double off, double *sv) const {
+        for (int i = 0; i < nr * 256; ++i) sv[i] = s * (levels[(size_t)i] + off);
     }
 
     // the objective at code q, its terms summed in the order of the widths
@@ -92,15 +96,16 @@ struct Objective {
     // below its value on [min(a, b), max(a, b)], a = min A_i, b = max B_i,
     // outside it, and the first minimum lies inside it or, when the cost is
     // flat at the window's left end, further left by equal steps.
-    // inv_s = 1 / s when s > 0 (a hint for locating A_i and B_i), else 0.
-    int best_code(double w, const double *sv, double inv_s) const {
+    // inv_s = 1 / s when s > 0 and off (as in products) are hints for
+    // locating A_i and B_i; inv_s = 0 searches instead.
+    int best_code(double w, const double *sv, double inv_s, double off) const {
         int a = 256, b = -1;
         for (int i = 0; i < nr; ++i) {
             if (!(lams[i] > 0.0)) continue;          // a zero term is flat everywhere
             const double *p = sv + i * 256;
             int le, lt;
             if (inv_s > 0.0) {
-                counts(i, p, w, inv_s, le, lt);
+                counts(i, p, w, inv_s, off, le, lt);
             } else {
                 le = (int)(std::upper_bound(p, p + 256, w) - p);
                 lt = (int)(std::lower_bound(p, p + 256, w) - p);
@@ -367,6 +372,35 @@ void invert_lower(const double *L, int64_t n, double *M, int nt, Simd simd) {
 // it alone.
 constexpr int64_t kRowBlock = 16;
 
+// x (fp32) rounded to the nearest fp16 value, ties to even, as a double
+// (infinite past the largest finite fp16, 65504): IEEE binary16 has 11
+// significant bits down to 2^-14 and a fixed step of 2^-24 below
+double fp16_value(float x) {
+    const double v = x;
+    if (!std::isfinite(v)) return v;
+    const double a = fabs(v);
+    int e;
+    frexp(a, &e);                                  // a = m 2^e, 0.5 <= m < 1
+    const double step = a < 0x1p-14 ? 0x1p-24 : ldexp(1.0, e - 11);
+    const double r = nearbyint(v / step) * step;   // the default rounding: to nearest, ties to even
+    return fabs(r) > 65504.0 ? copysign(INFINITY, v) : r;
+}
+
+// The asymmetric grid of one group for one multiplier: it spans alpha times
+// the group's range [lo, hi] and is centred on it, s = alpha (hi - lo) / 255
+// and z = 128 - (hi + lo) / (2 s), z as stored (fp32, then fp16); a group of
+// zero range, or one whose z is no finite fp16, takes the symmetric grid
+// (s = alpha max|w| / 127.5, z = 128).
+void asym_grid(double lo, double hi, double alpha, double &s, double &z) {
+    if (hi > lo) {
+        s = alpha * (hi - lo) / 255.0;
+        z = fp16_value((float)(128.0 - (hi + lo) / (2.0 * s)));
+        if (std::isfinite(z)) return;
+    }
+    s = alpha * std::max(fabs(lo), fabs(hi)) / 127.5;
+    z = 128.0;
+}
+
 // w[j] -= f u[j] for j0 <= j < j1: one rounded product and one rounded
 // difference per element (no fused multiply-add), as the oracle computes it
 inline void feedback(double *w, const double *u, double f, int64_t j0, int64_t j1) {
@@ -475,43 +509,52 @@ __attribute__((target("avx2"))) void feedback_group_avx2(double *w, int64_t nb, 
 }
 
 void quantize_rows(const float *W, int64_t K, const double *U, const Objective &obj, const double *alphas,
-                   int na, double lsum, int64_t n0, int64_t n1, uint8_t *codes, float *scales) {
+                   int na, double lsum, int64_t n0, int64_t n1, uint8_t *codes, float *scales, float *zeros) {
     const bool avx = have_avx2_fma();
     const int64_t G = K / 128, nb = n1 - n0;
     const size_t nsv = (size_t)obj.nr * 256;
-    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)(nb * 128)), inv_s((size_t)nb);
+    std::vector<double> w((size_t)(nb * K)), sv(nsv * (size_t)nb), f((size_t)(nb * 128)), inv_s((size_t)nb),
+        off((size_t)nb, 0.0);
     for (int64_t b = 0; b < nb; ++b)
         for (int64_t k = 0; k < K; ++k) w[(size_t)(b * K + k)] = (double)W[(n0 + b) * K + k];
     for (int64_t g = 0; g < G; ++g) {
-        // each row's scale, from its group's current weights
+        // each row's scale (and zero point), from its group's current weights
         for (int64_t b = 0; b < nb; ++b) {
             const double *wb = w.data() + b * K;
             double *svb = sv.data() + nsv * (size_t)b;
-            double mx = 0.0;
-            for (int64_t k = 128 * g; k < 128 * g + 128; ++k) mx = std::max(mx, fabs(wb[k]));
+            double mx = 0.0, lo = wb[128 * g], hi = wb[128 * g];
+            for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
+                mx = std::max(mx, fabs(wb[k]));
+                lo = std::min(lo, wb[k]);
+                hi = std::max(hi, wb[k]);
+            }
             const double base = mx / 127.5;
-            double best_a = 0.0, best_t = 0.0;
+            double best_s = 0.0, best_z = 128.0, best_t = 0.0;
             for (int ia = 0; ia < na; ++ia) {
-                const double st = base * alphas[ia], inv = st > 0.0 ? 1.0 / st : 0.0;
-                obj.products(st, svb);
+                double st = base * alphas[ia], zt = 128.0;
+                if (zeros) asym_grid(lo, hi, alphas[ia], st, zt);
+                const double inv = st > 0.0 ? 1.0 / st : 0.0;
+                obj.products(st, 128.0 - zt, svb);
                 double t = 0.0;
                 for (int64_t k = 128 * g; k < 128 * g + 128; ++k) {
                     const double x = wb[k];
-                    const int q = obj.best_code(x, svb, inv);
+                    const int q = obj.best_code(x, svb, inv, 128.0 - zt);
                     for (int i = 0; i < obj.nr; ++i) {
                         const double d = x - svb[(size_t)i * 256 + q];
                         t += obj.lams[i] * d * d;
                     }
                 }
                 if (ia == 0 || t < best_t) {
-                    best_a = alphas[ia];
+                    best_s = st;
+                    best_z = zt;
                     best_t = t;
                 }
             }
-            const double s = base * best_a;
-            scales[(n0 + b) * G + g] = (float)s;
-            obj.products(s, svb);
-            inv_s[(size_t)b] = s > 0.0 ? 1.0 / s : 0.0;
+            scales[(n0 + b) * G + g] = (float)best_s;
+            if (zeros) zeros[(n0 + b) * G + g] = (float)best_z;
+            off[(size_t)b] = 128.0 - best_z;
+            obj.products(best_s, off[(size_t)b], svb);
+            inv_s[(size_t)b] = best_s > 0.0 ? 1.0 / best_s : 0.0;
         }
         // the group's columns in order; each column's feedback reaches the
         // rest of the group at once and the later groups' columns after the
@@ -522,7 +565,7 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
             for (int64_t b = 0; b < nb; ++b) {
                 const double *svb = sv.data() + nsv * (size_t)b;
                 const double x = w[(size_t)(b * K + k)];
-                const int q = obj.best_code(x, svb, inv_s[(size_t)b]);
+                const int q = obj.best_code(x, svb, inv_s[(size_t)b], off[(size_t)b]);
                 codes[(n0 + b) * K + k] = (uint8_t)q;
                 double e = 0.0;
                 for (int i = 0; i < obj.nr; ++i) e += obj.lams[i] * (x - svb[(size_t)i * 256 + q]);
@@ -656,10 +699,9 @@ extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp,
     return MQ_OK;
 }
 
-extern "C" mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const double *U,
-                                         const int32_t *rs, const double *lambdas, int n_r,
-                                         const double *alphas, int n_alpha, int threads,
-                                         uint8_t *codes_out, float *scales_out) {
+static mq_status quantize_common(const float *W, int64_t N, int64_t K, const double *U, const int32_t *rs,
+                                 const double *lambdas, int n_r, const double *alphas, int n_alpha,
+                                 int threads, uint8_t *codes_out, float *scales_out, float *zeros_out) {
     if (!W || !U || !rs || !lambdas || !alphas || !codes_out || !scales_out)
         return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_matgptq_quantize");
     if (N < 1 || K < kGroup || K % kGroup) return fail(MQ_ERR_INVALID_ARG, "need N >= 1 and K a positive multiple of 128");
@@ -682,7 +724,24 @@ extern "C" mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, c
     const int64_t nblocks = (N + kRowBlock - 1) / kRowBlock;
     parallel_rows(0, nblocks, nt, [&](int64_t blk) {
         quantize_rows(W, K, U, obj, alphas, n_alpha, lsum, blk * kRowBlock,
-                      std::min<int64_t>(N, (blk + 1) * kRowBlock), codes_out, scales_out);
+                      std::min<int64_t>(N, (blk + 1) * kRowBlock), codes_out, scales_out, zeros_out);
     });
     return MQ_OK;
+}
+
+extern "C" mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const double *U,
+                                         const int32_t *rs, const double *lambdas, int n_r,
+                                         const double *alphas, int n_alpha, int threads,
+                                         uint8_t *codes_out, float *scales_out) {
+    return quantize_common(W, N, K, U, rs, lambdas, n_r, alphas, n_alpha, threads, codes_out, scales_out,
+                           nullptr);
+}
+
+extern "C" mq_status mq_matgptq_quantize_asym(const float *W, int64_t N, int64_t K, const double *U,
+                                              const int32_t *rs, const double *lambdas, int n_r,
+                                              const double *alphas, int n_alpha, int threads,
+                                              uint8_t *codes_out, float *scales_out, float *zeros_out) {
+    if (!zeros_out) return fail(MQ_ERR_INVALID_ARG, "NULL zeros_out");
+    return quantize_common(W, N, K, U, rs, lambdas, n_r, alphas, n_alpha, threads, codes_out, scales_out,
+                           zeros_out);
 }
