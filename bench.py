@@ -696,7 +696,8 @@ PAGES_MATGPTQ_PASS_S = {"k_proj": 3.59, "q_proj": 3.59, "gate_proj": 6.58, "down
 def run_quantizer():
     """One JSON line per shape: the one-shot quantizer (r = 3, 4, 8, lambda =
     1, 1, 1, five scale multipliers) on a synthetic AR(1) Hessian, timed on
-    the host around the library calls."""
+    the host around the library calls; total_s is prepare plus the symmetric
+    quantize, quantize_asym_s the asymmetric variant on the same U."""
     import nested_bit_weight_b200 as mq
     for i, name in enumerate(("k_proj", "q_proj", "gate_proj", "down_proj")):
         l = next(x for x in wl.LLAMA8B if x.name == name)
@@ -707,9 +708,12 @@ def run_quantizer():
         t1 = time.perf_counter()
         mq.matgptq_quantize(W, U)
         t2 = time.perf_counter()
+        mq.matgptq_quantize(W, U, asymmetric=True)
+        t3 = time.perf_counter()
         print(json.dumps({"metric": "quantizer_pass_s", "layer": name, "N": l.N, "K": l.K,
                           "prepare_s": round(t1 - t0, 2), "quantize_s": round(t2 - t1, 2),
-                          "total_s": round(t2 - t0, 2), "threads": os.cpu_count(),
+                          "total_s": round(t2 - t0, 2), "quantize_asym_s": round(t3 - t2, 2),
+                          "threads": os.cpu_count(),
                           "pages_matgptq_pass_s": PAGES_MATGPTQ_PASS_S[name],
                           "higher_is_better": False, "data": "synthetic"}), flush=True)
         del H, U, W
