@@ -15,6 +15,9 @@
 //     lambda-weighted mean of the slice errors e:  w_j -= e / U[k,k] * U[k,j]
 //     (the update of the row's shared remainder that minimises the
 //     lambda-weighted sum of the widths' quadratic losses).
+// The asymmetric variant (mq_matgptq_quantize_asym; captions of Tables 5-7)
+// takes the levels u_r = 2^(8-r) q_r + 2^(7-r) - z on a grid that spans each
+// group's range, centred on it (asym_grid below); the rest is the same loop.
 // Rows are independent given U, so threads take blocks of rows; every
 // operation is fp64 in a fixed order, the same whatever the thread count.
 #include <immintrin.h>
@@ -69,7 +72,6 @@ struct Objective {
         lt = k * step;
     }
 
-    // sv[i][q] = s * v_i(q) for one scale s (non-decreasing in q for s >= 0)
     // sv[i][q] = s * (v_i(q) + off) for one scale s >= 0 and level offset
     // off = 128 - z (0 for the symmetric levels; v_i(q) + off is exact, so
     // each product is the level's one rounding), non-decreasing in q
