@@ -232,8 +232,9 @@ typedef struct mq_choice {
  *   error_out   the summed error of the choice (may be NULL)
  * Ties: least error, then fewest bytes, then the lowest candidate indices.
  * Returns MQ_ERR_INVALID_ARG for bad sizes or a negative / non-finite error,
- * MQ_ERR_UNSUPPORTED when no choice fits the budget or the dynamic program
- * would need more than 2^26 (layer, budget unit) cells.
+ * MQ_ERR_UNSUPPORTED when no choice fits the budget, the dynamic program
+ * would need more than 2^26 (layer, budget unit) cells, or host memory runs
+ * out.
  */
 MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int n_choices,
                                     uint64_t budget_bytes, int *choice_out, double *error_out);
@@ -266,8 +267,9 @@ MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int 
  * Errors: MQ_ERR_INVALID_ARG for bad sizes, widths, lambdas (all zero, or
  * negative) or alphas, a non-finite weight, or a zero on U's diagonal;
  * MQ_ERR_UNSUPPORTED when the damped Hessian is not positive definite (or
- * too ill-conditioned to invert).  The caller owns every buffer; nothing is
- * written to codes_out or scales_out on an argument error.
+ * too ill-conditioned to invert), or when host memory or threads run out (no
+ * C++ exception leaves the library).  The caller owns every buffer; nothing
+ * is written to codes_out or scales_out on an argument error.
  */
 MQ_API mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp, double *U_out);
 MQ_API mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const double *U,

@@ -7,6 +7,9 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <exception>
+#include <new>
+
 #include "../../include/mq.h"
 
 namespace mq {
@@ -24,6 +27,22 @@ inline mq_status fail(mq_status s, const char *what) {
     return s;
 }
 mq_status cuda_fail(cudaError_t e, const char *where);
+
+// f() for the host-only entry points that allocate or start threads: no C++
+// exception crosses the C ABI (host memory exhausted, or threads refused,
+// returns MQ_ERR_UNSUPPORTED with the reason).
+template <class F>
+mq_status host_guarded(F &&f) {
+    try {
+        return f();
+    } catch (const std::bad_alloc &) {
+        return fail(MQ_ERR_UNSUPPORTED, "out of host memory");
+    } catch (const std::exception &e) {
+        return fail(MQ_ERR_UNSUPPORTED, e.what());
+    } catch (...) {
+        return fail(MQ_ERR_UNSUPPORTED, "host error");
+    }
+}
 
 inline bool aligned16(const void *p) {
     return (reinterpret_cast<uintptr_t>(p) & 15u) == 0;

@@ -28,6 +28,7 @@
 #include <cmath>
 #include <atomic>
 #include <memory>
+#include <mutex>
 #include <thread>
 #include <vector>
 
@@ -152,19 +153,36 @@ inline double dot(const double *a, const double *b, int64_t m) {
 }
 
 // f(i) for i in [i0, i1), spread over up to nt threads by a shared counter
-// (rows of unequal cost balance themselves)
+// (rows of unequal cost balance themselves); an exception in any thread is
+// rethrown here after all have joined
 template <class F>
 void parallel_rows(int64_t i0, int64_t i1, int nt, F &&f) {
     if (i1 <= i0) return;
     std::atomic<int64_t> next{i0};
+    std::exception_ptr err;
+    std::mutex mu;
     auto work = [&]() {
-        for (int64_t i; (i = next.fetch_add(1)) < i1;) f(i);
+        try {
+            for (int64_t i; (i = next.fetch_add(1)) < i1;) f(i);
+        } catch (...) {                        // first failure wins; the others stop taking rows
+            std::lock_guard<std::mutex> g(mu);
+            if (!err) err = std::current_exception();
+            next.store(i1);
+        }
     };
     const int m = (int)std::min<int64_t>(nt, i1 - i0);
     std::vector<std::thread> pool;
-    for (int t = 1; t < m; ++t) pool.emplace_back(work);
+    pool.reserve((size_t)m);
+    for (int t = 1; t < m; ++t) {
+        try {
+            pool.emplace_back(work);
+        } catch (...) {                        // fewer threads: the rest of the rows run here
+            break;
+        }
+    }
     work();
     for (auto &th : pool) th.join();
+    if (err) std::rethrow_exception(err);
 }
 
 // T[r][c] += sum_{p0 <= p < p1} A[r][p] B[p][c] for r < 4, c < 8 (rows of
@@ -591,144 +609,148 @@ void quantize_rows(const float *W, int64_t K, const double *U, const Objective &
 }  // namespace
 
 extern "C" mq_status mq_matgptq_prepare(const double *H, int64_t K, double damp, double *U_out) {
-    if (!H || !U_out) return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_matgptq_prepare");
-    if (K < 1 || K > 65536) return fail(MQ_ERR_INVALID_ARG, "need 1 <= K <= 65536");
-    if (!(damp >= 0.0)) return fail(MQ_ERR_INVALID_ARG, "damp must be >= 0");
-    // A = H + damp * mean(diag H) * I and J the reversal (J A J reverses
-    // rows and columns).  With J A J = L L^T (lower Cholesky), A = R R^T for
-    // the upper R = J L J, so A^-1 = R^-T R^-1 and U = R^-1 = J L^-1 J is the
-    // upper factor with U^T U = A^-1 (unique for a positive diagonal).
-    const int64_t n = K;
-    double mean = 0.0;
-    for (int64_t i = 0; i < n; ++i) mean += H[i * n + i];
-    mean /= (double)K;
-    const double add = damp * mean;
-    auto P = [&](int64_t i, int64_t j) {
-        return H[(n - 1 - i) * n + (n - 1 - j)] + (i == j ? add : 0.0);
-    };
-    const int nt = std::max(1, std::min<int>(64, (int)std::thread::hardware_concurrency()));
-    // L starts as the lower triangle of J A J and is factorised in place;
-    // its upper triangle is never read, so the buffer is not initialised
-    // (its pages are first touched by the threads that copy the rows)
-    std::unique_ptr<double[]> L(new double[(size_t)n * n]);
-    double *Lp = L.get();
-    parallel_rows(0, n, nt, [&](int64_t i) {
-        for (int64_t j = 0; j <= i; ++j) Lp[i * n + j] = P(i, j);
-    });
-    const Simd simd = host_simd();
-    const bool avx = simd != Simd::portable;
-    const int64_t R = tile_rows(simd);
-    auto dotv = [avx](const double *a, const double *b, int64_t m) {
-        return avx ? dot_avx2(a, b, m) : dot(a, b, m);
-    };
-    // Right-looking blocked Cholesky, kNB columns per panel: factor the
-    // panel's diagonal block, solve the rows below it against that block,
-    // then subtract the panel's product from the trailing lower triangle
-    // (4 x 8 tiles by the same kernel as the inverse, against the panel
-    // transposed and negated, kGR rows per task so that each 8-column tile
-    // of it is reused from cache).
-    constexpr int64_t kNB = 128, kGR = 32;
-    std::vector<double> Pt;
-    for (int64_t j0 = 0; j0 < n; j0 += kNB) {
-        const int64_t j1 = std::min(n, j0 + kNB), nb = j1 - j0;
-        for (int64_t i = j0; i < j1; ++i)
-            for (int64_t j = j0; j <= i; ++j) {
-                const double v = Lp[i * n + j] - dotv(Lp + i * n + j0, Lp + j * n + j0, j - j0);
-                if (i == j) {
-                    if (!(v > 0.0) || !isfinite(v))
-                        return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is not positive definite");
-                    Lp[i * n + i] = sqrt(v);
-                } else {
-                    Lp[i * n + j] = v / Lp[j * n + j];
-                }
-            }
-        const int64_t m = n - j1;
-        if (m == 0) break;
-        parallel_rows(j1, n, nt, [&](int64_t i) {
-            double *li = Lp + i * n;
-            for (int64_t j = j0; j < j1; ++j)
-                li[j] = (li[j] - dotv(li + j0, Lp + j * n + j0, j - j0)) / Lp[j * n + j];
+    return host_guarded([&]() -> mq_status {
+        if (!H || !U_out) return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_matgptq_prepare");
+        if (K < 1 || K > 65536) return fail(MQ_ERR_INVALID_ARG, "need 1 <= K <= 65536");
+        if (!(damp >= 0.0)) return fail(MQ_ERR_INVALID_ARG, "damp must be >= 0");
+        // A = H + damp * mean(diag H) * I and J the reversal (J A J reverses
+        // rows and columns).  With J A J = L L^T (lower Cholesky), A = R R^T for
+        // the upper R = J L J, so A^-1 = R^-T R^-1 and U = R^-1 = J L^-1 J is the
+        // upper factor with U^T U = A^-1 (unique for a positive diagonal).
+        const int64_t n = K;
+        double mean = 0.0;
+        for (int64_t i = 0; i < n; ++i) mean += H[i * n + i];
+        mean /= (double)K;
+        const double add = damp * mean;
+        auto P = [&](int64_t i, int64_t j) {
+            return H[(n - 1 - i) * n + (n - 1 - j)] + (i == j ? add : 0.0);
+        };
+        const int nt = std::max(1, std::min<int>(64, (int)std::thread::hardware_concurrency()));
+        // L starts as the lower triangle of J A J and is factorised in place;
+        // its upper triangle is never read, so the buffer is not initialised
+        // (its pages are first touched by the threads that copy the rows)
+        std::unique_ptr<double[]> L(new double[(size_t)n * n]);
+        double *Lp = L.get();
+        parallel_rows(0, n, nt, [&](int64_t i) {
+            for (int64_t j = 0; j <= i; ++j) Lp[i * n + j] = P(i, j);
         });
-        // Pt: the panel's rows below j1, negated and transposed, in tiles of 8
-        // columns each contiguous (tile t, term p, column c at (t nb + p) 8 + c;
-        // the last tile padded with zeros)
-        const int64_t m8 = (m + 7) / 8 * 8;
-        Pt.resize((size_t)(nb * m8));
-        parallel_rows(0, m8, nt, [&](int64_t jj) {
-            double *dst = Pt.data() + (jj / 8) * nb * 8 + jj % 8;
-            if (jj >= m) {
-                for (int64_t p = 0; p < nb; ++p) dst[p * 8] = 0.0;
-                return;
-            }
-            const double *lj = Lp + (j1 + jj) * n + j0;
-            for (int64_t p = 0; p < nb; ++p) dst[p * 8] = -lj[p];
-        });
-        const int64_t ng = (m + kGR - 1) / kGR;
-        parallel_rows(0, ng, nt, [&](int64_t t) {
-            const int64_t g0 = j1 + (ng - 1 - t) * kGR;          // largest groups first
-            const int64_t g1 = std::min(n, g0 + kGR);
-            // chunks of kCC columns (their panel tiles stay in cache), each
-            // row tile of the group running along the chunk
-            constexpr int64_t kCC = 64;
-            for (int64_t jc = j1; jc < g1; jc += kCC)
-            for (int64_t i = g0; i < g1; i += R) {
-                for (int64_t jt = jc; jt < std::min(g1, jc + kCC); jt += 8) {
-                    if (jt > i + R - 1) break;                    // the rest lies above the diagonal
-                    const double *B = Pt.data() + (jt - j1) * nb;    // tile (jt - j1) / 8
-                    if (i + R <= g1 && jt + 8 <= n) {
-                        // writes of the tile's entries above the diagonal
-                        // land in L's unread upper triangle
-                        gemm_tile(simd, Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
+        const Simd simd = host_simd();
+        const bool avx = simd != Simd::portable;
+        const int64_t R = tile_rows(simd);
+        auto dotv = [avx](const double *a, const double *b, int64_t m) {
+            return avx ? dot_avx2(a, b, m) : dot(a, b, m);
+        };
+        // Right-looking blocked Cholesky, kNB columns per panel: factor the
+        // panel's diagonal block, solve the rows below it against that block,
+        // then subtract the panel's product from the trailing lower triangle
+        // (4 x 8 tiles by the same kernel as the inverse, against the panel
+        // transposed and negated, kGR rows per task so that each 8-column tile
+        // of it is reused from cache).
+        constexpr int64_t kNB = 128, kGR = 32;
+        std::vector<double> Pt;
+        for (int64_t j0 = 0; j0 < n; j0 += kNB) {
+            const int64_t j1 = std::min(n, j0 + kNB), nb = j1 - j0;
+            for (int64_t i = j0; i < j1; ++i)
+                for (int64_t j = j0; j <= i; ++j) {
+                    const double v = Lp[i * n + j] - dotv(Lp + i * n + j0, Lp + j * n + j0, j - j0);
+                    if (i == j) {
+                        if (!(v > 0.0) || !isfinite(v))
+                            return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is not positive definite");
+                        Lp[i * n + i] = sqrt(v);
                     } else {
-                        for (int64_t r = i; r < std::min(i + R, g1); ++r)
-                            for (int64_t c = jt; c < std::min(jt + 8, r + 1); ++c) {
-                                double v = 0.0;
-                                for (int64_t p = 0; p < nb; ++p) v += Lp[r * n + j0 + p] * B[p * 8 + (c - jt)];
-                                Lp[r * n + c] += v;
-                            }
+                        Lp[i * n + j] = v / Lp[j * n + j];
                     }
                 }
-            }
-        });
-    }
-    // M = L^-1 into U_out, then U = J M J: the 180-degree rotation of the
-    // matrix, i.e. the flat array reversed
-    parallel_rows(0, n, nt, [&](int64_t i) { std::fill(U_out + i * n, U_out + (i + 1) * n, 0.0); });
-    invert_lower(Lp, n, U_out, nt, simd);
-    std::reverse(U_out, U_out + (size_t)n * n);
-    for (int64_t i = 0; i < n; ++i)
-        if (!(U_out[i * n + i] > 0.0) || !isfinite(U_out[i * n + i])) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is too ill-conditioned to invert");
-    return MQ_OK;
+            const int64_t m = n - j1;
+            if (m == 0) break;
+            parallel_rows(j1, n, nt, [&](int64_t i) {
+                double *li = Lp + i * n;
+                for (int64_t j = j0; j < j1; ++j)
+                    li[j] = (li[j] - dotv(li + j0, Lp + j * n + j0, j - j0)) / Lp[j * n + j];
+            });
+            // Pt: the panel's rows below j1, negated and transposed, in tiles of 8
+            // columns each contiguous (tile t, term p, column c at (t nb + p) 8 + c;
+            // the last tile padded with zeros)
+            const int64_t m8 = (m + 7) / 8 * 8;
+            Pt.resize((size_t)(nb * m8));
+            parallel_rows(0, m8, nt, [&](int64_t jj) {
+                double *dst = Pt.data() + (jj / 8) * nb * 8 + jj % 8;
+                if (jj >= m) {
+                    for (int64_t p = 0; p < nb; ++p) dst[p * 8] = 0.0;
+                    return;
+                }
+                const double *lj = Lp + (j1 + jj) * n + j0;
+                for (int64_t p = 0; p < nb; ++p) dst[p * 8] = -lj[p];
+            });
+            const int64_t ng = (m + kGR - 1) / kGR;
+            parallel_rows(0, ng, nt, [&](int64_t t) {
+                const int64_t g0 = j1 + (ng - 1 - t) * kGR;          // largest groups first
+                const int64_t g1 = std::min(n, g0 + kGR);
+                // chunks of kCC columns (their panel tiles stay in cache), each
+                // row tile of the group running along the chunk
+                constexpr int64_t kCC = 64;
+                for (int64_t jc = j1; jc < g1; jc += kCC)
+                for (int64_t i = g0; i < g1; i += R) {
+                    for (int64_t jt = jc; jt < std::min(g1, jc + kCC); jt += 8) {
+                        if (jt > i + R - 1) break;                    // the rest lies above the diagonal
+                        const double *B = Pt.data() + (jt - j1) * nb;    // tile (jt - j1) / 8
+                        if (i + R <= g1 && jt + 8 <= n) {
+                            // writes of the tile's entries above the diagonal
+                            // land in L's unread upper triangle
+                            gemm_tile(simd, Lp + i * n + j0, n, B, 8, 0, nb, Lp + i * n + jt, n);
+                        } else {
+                            for (int64_t r = i; r < std::min(i + R, g1); ++r)
+                                for (int64_t c = jt; c < std::min(jt + 8, r + 1); ++c) {
+                                    double v = 0.0;
+                                    for (int64_t p = 0; p < nb; ++p) v += Lp[r * n + j0 + p] * B[p * 8 + (c - jt)];
+                                    Lp[r * n + c] += v;
+                                }
+                        }
+                    }
+                }
+            });
+        }
+        // M = L^-1 into U_out, then U = J M J: the 180-degree rotation of the
+        // matrix, i.e. the flat array reversed
+        parallel_rows(0, n, nt, [&](int64_t i) { std::fill(U_out + i * n, U_out + (i + 1) * n, 0.0); });
+        invert_lower(Lp, n, U_out, nt, simd);
+        std::reverse(U_out, U_out + (size_t)n * n);
+        for (int64_t i = 0; i < n; ++i)
+            if (!(U_out[i * n + i] > 0.0) || !isfinite(U_out[i * n + i])) return fail(MQ_ERR_UNSUPPORTED, "the damped Hessian is too ill-conditioned to invert");
+        return MQ_OK;
+    });
 }
 
 static mq_status quantize_common(const float *W, int64_t N, int64_t K, const double *U, const int32_t *rs,
                                  const double *lambdas, int n_r, const double *alphas, int n_alpha,
                                  int threads, uint8_t *codes_out, float *scales_out, float *zeros_out) {
-    if (!W || !U || !rs || !lambdas || !alphas || !codes_out || !scales_out)
-        return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_matgptq_quantize");
-    if (N < 1 || K < kGroup || K % kGroup) return fail(MQ_ERR_INVALID_ARG, "need N >= 1 and K a positive multiple of 128");
-    if (n_r < 1 || n_r > 8 || n_alpha < 1) return fail(MQ_ERR_INVALID_ARG, "need 1 <= n_r <= 8 and n_alpha >= 1");
-    double lsum = 0.0;
-    for (int i = 0; i < n_r; ++i) {
-        if (rs[i] < 1 || rs[i] > 8) return fail(MQ_ERR_INVALID_ARG, "bit widths must be in 1..8");
-        if (!(lambdas[i] >= 0.0) || !isfinite(lambdas[i])) return fail(MQ_ERR_INVALID_ARG, "lambdas must be finite and >= 0");
-        lsum += lambdas[i];
-    }
-    if (!(lsum > 0.0)) return fail(MQ_ERR_INVALID_ARG, "the lambdas must not all be zero");
-    for (int i = 0; i < n_alpha; ++i)
-        if (!(alphas[i] > 0.0) || !isfinite(alphas[i])) return fail(MQ_ERR_INVALID_ARG, "alphas must be finite and > 0");
-    for (int64_t k = 0; k < K; ++k)
-        if (!(U[k * K + k] != 0.0)) return fail(MQ_ERR_INVALID_ARG, "U has a zero on its diagonal");
-    for (int64_t i = 0; i < N * K; ++i)
-        if (!isfinite(W[i])) return fail(MQ_ERR_INVALID_ARG, "W holds a non-finite value");
-    const Objective obj(rs, lambdas, n_r);
-    const int nt = threads > 0 ? threads : (int)std::max(1u, std::thread::hardware_concurrency());
-    const int64_t nblocks = (N + kRowBlock - 1) / kRowBlock;
-    parallel_rows(0, nblocks, nt, [&](int64_t blk) {
-        quantize_rows(W, K, U, obj, alphas, n_alpha, lsum, blk * kRowBlock,
-                      std::min<int64_t>(N, (blk + 1) * kRowBlock), codes_out, scales_out, zeros_out);
+    return host_guarded([&]() -> mq_status {
+        if (!W || !U || !rs || !lambdas || !alphas || !codes_out || !scales_out)
+            return fail(MQ_ERR_INVALID_ARG, "NULL argument to mq_matgptq_quantize");
+        if (N < 1 || K < kGroup || K % kGroup) return fail(MQ_ERR_INVALID_ARG, "need N >= 1 and K a positive multiple of 128");
+        if (n_r < 1 || n_r > 8 || n_alpha < 1) return fail(MQ_ERR_INVALID_ARG, "need 1 <= n_r <= 8 and n_alpha >= 1");
+        double lsum = 0.0;
+        for (int i = 0; i < n_r; ++i) {
+            if (rs[i] < 1 || rs[i] > 8) return fail(MQ_ERR_INVALID_ARG, "bit widths must be in 1..8");
+            if (!(lambdas[i] >= 0.0) || !isfinite(lambdas[i])) return fail(MQ_ERR_INVALID_ARG, "lambdas must be finite and >= 0");
+            lsum += lambdas[i];
+        }
+        if (!(lsum > 0.0)) return fail(MQ_ERR_INVALID_ARG, "the lambdas must not all be zero");
+        for (int i = 0; i < n_alpha; ++i)
+            if (!(alphas[i] > 0.0) || !isfinite(alphas[i])) return fail(MQ_ERR_INVALID_ARG, "alphas must be finite and > 0");
+        for (int64_t k = 0; k < K; ++k)
+            if (!(U[k * K + k] != 0.0)) return fail(MQ_ERR_INVALID_ARG, "U has a zero on its diagonal");
+        for (int64_t i = 0; i < N * K; ++i)
+            if (!isfinite(W[i])) return fail(MQ_ERR_INVALID_ARG, "W holds a non-finite value");
+        const Objective obj(rs, lambdas, n_r);
+        const int nt = threads > 0 ? threads : (int)std::max(1u, std::thread::hardware_concurrency());
+        const int64_t nblocks = (N + kRowBlock - 1) / kRowBlock;
+        parallel_rows(0, nblocks, nt, [&](int64_t blk) {
+            quantize_rows(W, K, U, obj, alphas, n_alpha, lsum, blk * kRowBlock,
+                          std::min<int64_t>(N, (blk + 1) * kRowBlock), codes_out, scales_out, zeros_out);
+        });
+        return MQ_OK;
     });
-    return MQ_OK;
 }
 
 extern "C" mq_status mq_matgptq_quantize(const float *W, int64_t N, int64_t K, const double *U,
