@@ -6,6 +6,7 @@ import numpy as np
 import pytest
 
 import oracle
+import workloads as wl
 import nested_bit_weight_b200 as mq
 
 
@@ -213,5 +214,18 @@ def test_many_groups_and_a_ragged_row_block_match_the_oracle():
     W = _W(N, K, 102)
     c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U, alphas=(1.0, 0.85))
     codes, scales = mq.matgptq_quantize(W, U, alphas=(1.0, 0.85))
+    assert np.array_equal(codes, c_ref)
+    assert np.array_equal(scales, s_ref.astype(np.float32))
+
+
+def test_sixteen_groups_match_the_oracle():
+    # K = 2048: every group's feedback reaches fifteen later groups through
+    # the grouped update, and the window search runs over 16 scale choices
+    N, K = 3, 2048
+    H = wl.gen_hessian(K, 111, samples=K + 256)
+    U = oracle.matgptq_prepare(H)
+    W = wl.gen_float_weights(N, K, 112)
+    c_ref, s_ref = oracle.matgptq_quantize(W.astype(np.float64), U, alphas=(1.0, 0.9))
+    codes, scales = mq.matgptq_quantize(W, U, alphas=(1.0, 0.9))
     assert np.array_equal(codes, c_ref)
     assert np.array_equal(scales, s_ref.astype(np.float32))
