@@ -263,7 +263,8 @@ MQ_API mq_status mq_bitwidth_search(const mq_choice *choices, int n_layers, int 
  *     carried to the later columns of the row, w_j -= e / U[k][k] * U[k][j].
  *     codes_out N x K uint8, scales_out N x (K/128) fp32 (inputs of mq_pack).
  *     threads <= 0: one per hardware thread.  fp64 in a fixed order, so the
- *     result does not depend on the thread count.
+ *     result does not depend on the thread count (in the default
+ *     floating-point environment: round to nearest even).
  * Errors: MQ_ERR_INVALID_ARG for bad sizes, widths, lambdas (all zero, or
  * negative) or alphas, a non-finite weight, or a zero on U's diagonal;
  * MQ_ERR_UNSUPPORTED when the damped Hessian is not positive definite (or
